@@ -1,0 +1,476 @@
+"""Benchmark: causal attention forward + backward, bf16, TFLOP/s on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step is one pass of the whole path over one batch of the workload: the
+forward (one kernel) and the backward (D pre-pass, dK/dV kernel with dQ atomics,
+dQ conversion), all through the C ABI.  FLOPs are the causal counts (forward
+2*B*H*T^2*d, backward 2.5x that).  Inputs are synthetic (seeded bf16 Gaussian
+with the workload's shape and distribution) and resident in HBM; successive
+steps rotate over several input sets whose total is larger than the 126 MB L2.
+
+Prints ONE JSON line on rank 0.  With N > 1 (launched by torch.distributed.run)
+every rank runs its own batch (independent heads, no collective on the data
+path: weak scaling); the time is the max over ranks.
+
+--impl reference times the fp64 CPU oracle instead (the slow, plain reference
+this library is checked against) on a bounded sample of the workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from causal_attention_fwd_attn_b200 import workloads as wl  # noqa: E402
+
+METRIC = "causal attention fwd+bwd TFLOP/s (bf16) and % of B200 dense BF16 peak"
+UNIT = "TFLOP/s"
+DEFAULT_WORKLOAD = "gpt2small_b8h12t1024d64"
+L2_BYTES = 126 * 1024 * 1024
+PROFILES = os.path.join(ROOT, "profiles")
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {"bf16_tflops": p["bf16_tflops"], "bf16_tflops_sustained": p["bf16_tflops_sustained"],
+                "hbm_gbs": p["hbm_gbs"], "source": "measured"}
+    return {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0,
+            "source": "fallback"}
+
+
+def kernel_source_sha():
+    h = hashlib.sha256()
+    for name in ("attn_bwd.cu", "attn_fwd.cu", "sm100_ptx.cuh"):
+        with open(os.path.join(ROOT, "causal_attention_fwd_attn_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel, workload):
+    """DRAM bytes per launch from a committed ncu capture, if the kernel sources
+    are unchanged since it was taken (else None)."""
+    path = os.path.join(PROFILES, "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f)
+    e = rec.get(kernel, {}).get(workload)
+    if not e or e.get("source_sha") != kernel_source_sha():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+def find_workload(name):
+    for i, w in enumerate(wl.WORKLOADS):
+        if w.name == name:
+            return i, w
+    raise SystemExit(f"unknown workload {name}; choose from {[w.name for w in wl.WORKLOADS]}")
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (FileNotFoundError, OSError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        smax = max(float(r[2]) for r in rows if r[2].replace(".", "").isdigit())
+        loaded = [r for r in rows if _num(r[3]) and float(r[3]) > 200] or rows
+        sm_loaded = [float(r[1]) for r in loaded if r[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
+        return {"sm_mhz": statistics.median(sm_loaded or sm), "sm_max_mhz": smax,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def _num(x):
+    try:
+        float(x)
+        return True
+    except ValueError:
+        return False
+
+
+# ------------------------------------------------------------------- ours ----
+def run_ours(args, rank, world, local_rank):
+    from causal_attention_fwd_attn_b200 import _lib
+
+    ci, w = find_workload(args.workload)
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    B, H, T, d = w.B, w.H, w.T, w.d
+    scale = w.scale
+    set_bytes = 4 * B * H * T * d * 2
+    out_bytes = B * H * T * d * 2 * 4 + B * H * T * 4
+    n_sets = max(2, math.ceil(3 * L2_BYTES / set_bytes))
+    sets = []
+    for s in range(n_sets):
+        x = wl.make_inputs(ci, seed_offset=100 * s + 17 * rank)
+        sets.append({n: t.to(dev) for n, t in x.items()})
+    o = torch.empty((B, H, T, d), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((B, H, T), dtype=torch.float32, device=dev)
+    dq, dk, dv = (torch.empty((B, H, T, d), dtype=torch.bfloat16, device=dev) for _ in range(3))
+    ws_n = _lib.forge_attn_bwd_workspace_size(B, H, T, d)
+    ws = torch.empty(ws_n, dtype=torch.uint8, device=dev)
+    delta_p = ws.data_ptr()
+    acc_p = ws.data_ptr() + ((B * H * T * 4 + 255) // 256) * 256
+    stream = torch.cuda.current_stream(dev)
+    s = stream.cuda_stream
+
+    def step(x, ev=None):
+        q, k, v, dO = x["q"], x["k"], x["v"], x["dO"]
+        if ev:
+            ev[0].record(stream)
+        _lib.check(_lib.forge_attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                       lse.data_ptr(), B, H, T, d, scale, w.causal, s), "fwd")
+        if ev:
+            ev[1].record(stream)
+        _lib.check(_lib.forge_attn_bwd_preprocess(o.data_ptr(), dO.data_ptr(), delta_p, acc_p, B,
+                                                  H, T, d, 0, s), "pre")
+        if ev:
+            ev[2].record(stream)
+        _lib.check(_lib.forge_attn_bwd_dkdv(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                            dO.data_ptr(), lse.data_ptr(), delta_p, acc_p,
+                                            dk.data_ptr(), dv.data_ptr(), B, H, T, d, scale,
+                                            w.causal, 0, s), "dkdv")
+        if ev:
+            ev[3].record(stream)
+        _lib.check(_lib.forge_attn_bwd_dq_convert(acc_p, dq.data_ptr(), B, H, T, d, s), "cvt")
+        if ev:
+            ev[4].record(stream)
+
+    launches_per_step = 4
+    for i in range(args.warmup):
+        step(sets[i % n_sets])
+    torch.cuda.synchronize()
+    st, detail = _lib.forge_attn_check_device_error(s)
+    if st != _lib.OK:
+        raise RuntimeError(f"device wait timed out during warm-up: 0x{detail:08x}")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    vis = [v for v in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if v]
+    clocks = ClockSampler(vis[local_rank] if local_rank < len(vis) else str(local_rank))
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)  # let the sampler start before the timed region
+    t0.record(stream)
+    for i in range(args.steps):
+        step(sets[(args.warmup + i) % n_sets], evs[i])
+    t1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    clk = clocks.stop()
+    elapsed_ms = t0.elapsed_time(t1)
+    st, detail = _lib.forge_attn_check_device_error(s)
+    if st != _lib.OK:
+        raise RuntimeError(f"device wait timed out: 0x{detail:08x}")
+
+    per = {"fwd": [], "pre": [], "dkdv": [], "cvt": []}
+    for e in evs:
+        per["fwd"].append(e[0].elapsed_time(e[1]))
+        per["pre"].append(e[1].elapsed_time(e[2]))
+        per["dkdv"].append(e[2].elapsed_time(e[3]))
+        per["cvt"].append(e[3].elapsed_time(e[4]))
+    avg = {k: sum(v) / len(v) for k, v in per.items()}
+
+    t = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    max_ms = float(t.item())
+
+    # ---- end to end through the C ABI with host buffers (pinned) ----------------
+    e2e = run_e2e(args, w, ci, dev, stream, o, lse, dq, dk, dv, ws, world)
+
+    result = None
+    if rank == 0:
+        peaks = measured_peaks()
+        flops = w.flops_total()
+        value = flops * args.steps * world / (max_ms * 1e-3) / 1e12
+        dkdv_flops = w.flops_bwd()
+        achieved = dkdv_flops / (avg["dkdv"] * 1e-3) / 1e12
+        dominant = max(avg, key=avg.get)
+        traffic = recorded_traffic("attn_bwd_dkdv", w.name)
+        result = {
+            "metric": METRIC,
+            "value": round(value, 2),
+            "unit": UNIT,
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": round(max_ms / args.steps, 4),
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "bf16",
+            "data": "synthetic",
+            "config": {
+                "workload": w.name, "B": B, "H": H, "T": T, "d": d, "causal": w.causal,
+                "scale": "1/sqrt(d)", "inputs": "seeded iid Gaussian bf16, resident in HBM",
+                "l2": f"rotating {n_sets} input sets, {n_sets * set_bytes / 2**20:.0f} MiB of "
+                      f"inputs > 126 MB L2",
+                "parallelism": f"replicas x{world} (independent heads per GPU)",
+            },
+            "pct_of_peak": {"measured_bf16": round(100 * value / world / peaks["bf16_tflops"], 2),
+                            "spec_2250": round(100 * value / world / 2250.0, 2)},
+            "fwd_ms": round(avg["fwd"], 4),
+            "bwd_ms": round(avg["pre"] + avg["dkdv"] + avg["cvt"], 4),
+            "kernel_ms": {k: round(v, 4) for k, v in avg.items()},
+            "fwd_tflops": round(w.flops_fwd() / (avg["fwd"] * 1e-3) / 1e12, 1),
+            "bwd_tflops": round(w.flops_bwd() / ((avg["pre"] + avg["dkdv"] + avg["cvt"]) * 1e-3)
+                                / 1e12, 1),
+            "roofline": {
+                "kernel": "attn_bwd_dkdv",
+                "bound": "tensor",
+                "achieved": round(achieved, 1),
+                "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s",
+                "frac": round(achieved / peaks["bf16_tflops"], 4),
+                "traffic": traffic,
+                "peak_source": f"{peaks['source']} bf16_tflops (burst)",
+                "dominant_by_time": dominant,
+                "algorithmic_flops_per_launch": dkdv_flops,
+            },
+            "clocks": clk,
+            "e2e": e2e,
+            "gpu_launches": launches_per_step * args.steps,
+            "library": os.path.relpath(_lib.library_path(), ROOT),
+        }
+    return result
+
+
+def run_e2e(args, w, ci, dev, stream, o, lse, dq, dk, dv, ws, world):
+    """Same metric through the C ABI, with each step's inputs copied from pinned host
+    memory and its outputs copied back, all inside the timed region."""
+    from causal_attention_fwd_attn_b200 import _lib
+
+    B, H, T, d = w.B, w.H, w.T, w.d
+    x = wl.make_inputs(ci, seed_offset=7)
+    host_in = {n: t.pin_memory() for n, t in x.items()}
+    dev_in = {n: torch.empty_like(t, device=dev) for n, t in x.items()}
+    host_out = {"o": torch.empty_like(o, device="cpu").pin_memory(),
+                "lse": torch.empty_like(lse, device="cpu").pin_memory(),
+                "dq": torch.empty_like(dq, device="cpu").pin_memory(),
+                "dk": torch.empty_like(dk, device="cpu").pin_memory(),
+                "dv": torch.empty_like(dv, device="cpu").pin_memory()}
+    dev_out = {"o": o, "lse": lse, "dq": dq, "dk": dk, "dv": dv}
+    h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+    d2h = sum(t.numel() * t.element_size() for t in host_out.values())
+    s = stream.cuda_stream
+    ws_n = ws.numel()
+
+    def step():
+        for n in host_in:
+            dev_in[n].copy_(host_in[n], non_blocking=True)
+        q, k, v, dO = dev_in["q"], dev_in["k"], dev_in["v"], dev_in["dO"]
+        _lib.check(_lib.forge_attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                       lse.data_ptr(), B, H, T, d, w.scale, w.causal, s), "fwd")
+        _lib.check(_lib.forge_attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                       dO.data_ptr(), lse.data_ptr(), dq.data_ptr(),
+                                       dk.data_ptr(), dv.data_ptr(), ws.data_ptr(), ws_n, B, H,
+                                       T, d, w.scale, w.causal, s), "bwd")
+        for n in host_out:
+            host_out[n].copy_(dev_out[n], non_blocking=True)
+
+    steps = max(3, min(args.steps, 20))
+    for _ in range(2):
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(steps):
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1)
+    t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    ms = float(t.item())
+    value = w.flops_total() * steps * world / (ms * 1e-3) / 1e12
+    return {"value": round(value, 2), "unit": UNIT, "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "steps": steps, "ms_per_step": round(ms / steps, 4)}
+
+
+# ---------------------------------------------------------- CPU oracle leg ----
+def oracle_sample(w, ci, budget_s, threads):
+    """Time the fp64 oracle (forward + backward, the full T x T definition) on as
+    many heads of the workload as fit in about budget_s seconds on `threads` host
+    threads.  Returns (TFLOP/s in the workload's causal-FLOP convention, cores,
+    sample description)."""
+    import oracle
+
+    orc = oracle.default()
+    x = wl.make_inputs(ci)
+    heads = [(b, h) for b in range(w.B) for h in range(w.H)]
+    f = {n: x[n].double().numpy() for n in x}
+
+    def run(hs):
+        from concurrent.futures import ThreadPoolExecutor
+
+        def one(bh):
+            b, h = bh
+            orc.fwd_head(f["q"][b, h], f["k"][b, h], f["v"][b, h], w.scale, w.causal)
+            orc.bwd_head(f["q"][b, h], f["k"][b, h], f["v"][b, h], f["dO"][b, h], w.scale,
+                         w.causal)
+
+        t = time.perf_counter()
+        with ThreadPoolExecutor(max_workers=threads) as ex:
+            list(ex.map(one, hs))
+        return time.perf_counter() - t
+
+    # calibrate on one head per thread, then scale the sample to the budget (whole
+    # passes over the workload's heads are repeated when the workload is small)
+    first = heads[:min(threads, len(heads))]
+    t_first = run(first)
+    per_head = max(t_first, 1e-3) / len(first)
+    n = max(len(first), int(budget_s / per_head))
+    sample = [heads[j % len(heads)] for j in range(n)]
+    elapsed = run(sample)
+    flops_per_head = w.flops_total() / w.BH
+    value = flops_per_head * len(sample) / elapsed / 1e12
+    desc = (f"{len(sample)} head passes over the {w.BH} heads of {w.name} (T={w.T}, d={w.d}), "
+            f"fp64 oracle forward + backward, {elapsed:.1f} s on {threads} threads")
+    return value, threads, desc, elapsed
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    ci, w = find_workload(args.workload)
+    threads = os.cpu_count() or 1
+    steps_v = []
+    descs = []
+    budget = max(2.0, 150.0 / max(1, args.steps + args.warmup))
+    for i in range(args.warmup + args.steps):
+        v, cores, desc, el = oracle_sample(w, ci, budget, threads)
+        if i >= args.warmup:
+            steps_v.append((v, el))
+            descs.append(desc)
+    value = statistics.median(v for v, _ in steps_v)
+    ms = statistics.median(el for _, el in steps_v) * 1e3
+    return {
+        "impl": "reference",
+        "metric": METRIC, "value": round(value, 6), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 2),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "d": w.d,
+                   "causal": w.causal, "scale": "1/sqrt(d)",
+                   "note": "each step is a bounded sample of the workload's heads"},
+        "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": threads,
+                         "kind": "oracle", "sample": descs[-1]},
+        "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__,
+                                 formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--cpu-baseline-seconds", type=float, default=12.0,
+                    help="budget of the oracle sample timed beside the GPU run (rank 0, N=1)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be at least 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+
+    if args.impl == "reference":
+        res = run_reference(args, rank, world)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+
+    if world > 1:
+        import datetime
+
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group(
+            "nccl", timeout=datetime.timedelta(seconds=120),
+            device_id=torch.device("cuda", local_rank))
+    try:
+        res = run_ours(args, rank, world, local_rank)
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            ci, w = find_workload(args.workload)
+            v, cores, desc, _ = oracle_sample(w, ci, args.cpu_baseline_seconds,
+                                              os.cpu_count() or 1)
+            res["cpu_baseline"] = {"value": round(v, 6), "unit": UNIT, "cores": cores,
+                                   "kind": "oracle", "sample": desc}
+        elif rank == 0:
+            res["cpu_baseline"] = None
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.barrier()
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

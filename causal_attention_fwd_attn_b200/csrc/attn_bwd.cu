@@ -1,0 +1,687 @@
+// attn_bwd.cu -- fused causal attention backward for sm_100a.
+//
+// The Forge paper ("Building an LLM Training Framework from Scratch in C++ and
+// Metal on Apple Silicon") splits its backward into a pre-pass D = rowsum(dO o O)
+// in float, a dQ stage over queries and a dK/dV stage over key/value rows
+// (section "Ecosystem survey"), recomputes the probabilities from the saved
+// log-sum-exp (section "Attention kernel design"), and obtains the transposed
+// score matrices S^T = K Q^T and dP^T = V dO^T by exchanging operand roles
+// rather than moving data (same section).  Here:
+//
+//   attn_bwd_preprocess  D[i] = sum_k dO[i][k] O[i][k] (fp32), and the fp32 dQ
+//                        accumulator cleared.  Memory-bound, one thread per row.
+//   attn_bwd_dkdv        one CTA per (head, 128-key tile j), looping over the query
+//                        tiles i that see it (i >= j under the causal mask):
+//                          S^T  = K_j Q_i^T           (tcgen05, TMEM)
+//                          dP^T = V_j dO_i^T          (tcgen05, TMEM)
+//                          P^T  = exp2(S^T*scale*log2e - LSE_i*log2e)   (threads)
+//                          dS^T = P^T o (dP^T - D_i)                     (threads)
+//                          dV  += P^T dO_i ;  dK += dS^T Q_i             (tcgen05, TMEM)
+//                          dQ_i = dS K_j  (tcgen05 with dS^T read MN-major), then
+//                                 scale * dQ_i added to the fp32 accumulator with
+//                                 vector reductions (red.global.add.v4.f32).
+//                        The dQ stage of the paper is fused here: its partial sums
+//                        come out of the same recomputation, and reductions in L2
+//                        replace the paper's second pass over the scores.
+//   attn_bwd_dq_convert  dQ = bf16(accumulator).
+//
+// dkdv warp roles (320 threads):
+//   warp 0      producer: K_j, V_j once; Q_i, dO_i by TMA into staged rings; the
+//               LSE_i and D_i vectors (128 floats each) by plain loads into shared
+//               memory (queries past T get LSE = +inf, so their P is exactly 0).
+//   warp 1      MMA issuer (one thread).
+//   warps 2..9  compute: warp w owns TMEM lanes 32*(w%4).. (key rows of the tile)
+//               and half h = (w-2)/4 of the 128 query columns.  Each thread writes
+//               its 64 P^T and dS^T values bf16 into 128-byte-swizzled shared
+//               memory (the A operand of dV/dK, and the MN-major A operand of dQ),
+//               drains its half of dQ_i's columns for query row 32*(w%4)+lane,
+//               and stores its half of the dK/dV columns at the end.
+// Tensor memory: dV [0,d) | dK [d,2d) | S^T [2d,2d+128) | dP^T [2d+128,2d+256) |
+//   dQ_i [2d+256, 3d+256) for d = 64; for d = 128 dQ_i reuses the dP^T columns once
+//   dS^T has been formed (512 columns hold no more).
+#include "forge_internal.h"
+#include "sm100_ptx.cuh"
+
+namespace forge {
+namespace {
+
+constexpr int kBwdThreads = 320;
+constexpr int kComputeWarps = 8;
+constexpr float kLog2e = 1.4426950408889634f;
+
+enum : uint32_t {
+    kSiteKV = 1, kSiteQFull, kSiteDOFull, kSiteLdFull, kSiteQEmpty, kSiteDOEmpty, kSiteSFull,
+    kSiteSFree, kSiteDPFull, kSitePFull, kSitePFree, kSiteDSFull, kSiteDSFree, kSiteDQFull,
+    kSiteDQFree, kSiteAccDone, kSiteAlign
+};
+
+template <int D, bool PRECISE>
+struct BwdCfg {
+    static constexpr int kChunks = D / 64;
+    static constexpr int kChunkBytes = kTile * 128;        // 128 rows x 128 bytes
+    static constexpr int kTileBytes = kChunks * kChunkBytes;
+    static constexpr int kStagesQ = 2;
+    // Precise mode at d = 128 needs the room of one dO stage for the lo buffer.
+    static constexpr int kStagesDO = (D == 128 && PRECISE) ? 1 : 2;
+    // P^T and dS^T: [128 keys][128 queries] bf16 = two 64-query chunks; in precise
+    // mode each is a hi buffer followed by a lo buffer.
+    static constexpr int kScoreBytes = 2 * kChunkBytes;
+    static constexpr int kSplit = PRECISE ? 2 : 1;
+    // With d = 128 shared memory only holds one set of score buffers, used for P^T
+    // and then for dS^T.
+    static constexpr bool kSeparatePdS = (D == 64);
+    // With d = 64 dQ_i has tensor-memory columns of its own.
+    static constexpr bool kSeparateDQ = (D == 64);
+    static constexpr int kOffK = 0;
+    static constexpr int kOffV = kOffK + kTileBytes;
+    static constexpr int kOffQ = kOffV + kTileBytes;
+    static constexpr int kOffDO = kOffQ + kStagesQ * kTileBytes;
+    static constexpr int kOffP = kOffDO + kStagesDO * kTileBytes;
+    static constexpr int kOffDS = kSeparatePdS ? kOffP + kSplit * kScoreBytes : kOffP;
+    static constexpr int kOffLse = kOffDS + kSplit * kScoreBytes;
+    static constexpr int kOffDelta = kOffLse + kStagesQ * kTile * 4;
+    static constexpr int kOffBar = kOffDelta + kStagesQ * kTile * 4;
+    static constexpr int kSmemBytes = kOffBar + 256;
+    static_assert(kSmemBytes <= 232448, "shared memory budget");
+    static constexpr uint32_t kColDV = 0, kColDK = D, kColS = 2 * D, kColDP = 2 * D + 128;
+    static constexpr uint32_t kColDQ = kSeparateDQ ? 2 * D + 256 : kColDP;
+    static constexpr uint32_t kTmemCols = 512;
+    static_assert(kColDQ + D <= kTmemCols, "tensor memory budget");
+    static constexpr uint32_t kIdescScore = idesc_bf16_f32(128, 128, false, false);
+    static constexpr uint32_t kIdescGrad = idesc_bf16_f32(128, D, false, true);  // dV, dK
+    static constexpr uint32_t kIdescDQ = idesc_bf16_f32(128, D, true, true);     // dQ
+};
+
+struct BwdBarriers {
+    uint64_t kv_full;
+    uint64_t q_full[2];
+    uint64_t do_full[2];
+    uint64_t ld_full[2];
+    uint64_t q_empty[2];
+    uint64_t do_empty[2];
+    uint64_t s_full, s_free, dp_full, p_full, p_free, ds_full, ds_free, dq_full, dq_free;
+    uint64_t acc_done, mma_final;
+    uint32_t tmem_base;
+    int abort;
+};
+
+// Eight fp32 values as bf16 into a 16-byte chunk at base + off; in precise mode the
+// remainders x - bf16(x), rounded to bf16, go to the same place in the lo buffer
+// (base + lo_stride + off).
+template <bool PRECISE>
+__device__ __forceinline__ void store_split8(uint8_t* base, int lo_stride, uint32_t off,
+                                             const float* x) {
+    uint32_t h[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) h[e] = pack_bf16x2(x[2 * e], x[2 * e + 1]);
+    *reinterpret_cast<uint4*>(base + off) = make_uint4(h[0], h[1], h[2], h[3]);
+    if (PRECISE) {
+        uint32_t l[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+            l[e] = pack_bf16x2(x[2 * e] - bf16_lo_to_float(h[e]),
+                               x[2 * e + 1] - bf16_hi_to_float(h[e]));
+        *reinterpret_cast<uint4*>(base + lo_stride + off) = make_uint4(l[0], l[1], l[2], l[3]);
+    }
+}
+
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, uint32_t site,
+                                          volatile int* abort) {
+    return __all_sync(0xffffffffu, mbar_wait(bar, parity, site, abort));
+}
+
+// Fire-and-forget fp32 vector reduction into global memory (no value returned).
+__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b),
+                 "f"(c), "f"(d)
+                 : "memory");
+}
+
+template <int D, bool PRECISE>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmap_q,
+                         const __grid_constant__ CUtensorMap tmap_k,
+                         const __grid_constant__ CUtensorMap tmap_v,
+                         const __grid_constant__ CUtensorMap tmap_do,
+                         const float* __restrict__ lse, const float* __restrict__ delta,
+                         float* __restrict__ dq_accum, void* __restrict__ dk_out,
+                         void* __restrict__ dv_out, int T, int n_kvtiles, float scale,
+                         float scale_log2, int causal, int grad_f32) {
+    using C = BwdCfg<D, PRECISE>;
+    extern __shared__ __align__(1024) uint8_t smem[];
+    BwdBarriers* bars = reinterpret_cast<BwdBarriers*>(smem + C::kOffBar);
+    volatile int* abort = &bars->abort;
+    float* s_lse = reinterpret_cast<float*>(smem + C::kOffLse);
+    float* s_delta = reinterpret_cast<float*>(smem + C::kOffDelta);
+
+    const int bh = blockIdx.x;
+    const int kt = n_kvtiles - 1 - blockIdx.y;  // key tile; the most query tiles first
+    const int n_qtiles = n_kvtiles;
+    const int i_begin = causal ? kt : 0;
+    const int n_iter = n_qtiles - i_begin;
+    const uint32_t warp = warp_id();
+    const uint32_t lane = lane_id();
+
+    if (threadIdx.x == 0) {
+        mbar_init(&bars->kv_full, 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&bars->q_full[s], 1);
+            mbar_init(&bars->do_full[s], 1);
+            mbar_init(&bars->ld_full[s], 32);
+            mbar_init(&bars->q_empty[s], 1);
+            mbar_init(&bars->do_empty[s], 1);
+        }
+        mbar_init(&bars->s_full, 1);
+        mbar_init(&bars->s_free, kComputeWarps);
+        mbar_init(&bars->dp_full, 1);
+        mbar_init(&bars->p_full, kComputeWarps);
+        mbar_init(&bars->p_free, 1);
+        mbar_init(&bars->ds_full, kComputeWarps);
+        mbar_init(&bars->ds_free, 1);
+        mbar_init(&bars->dq_full, 1);
+        mbar_init(&bars->dq_free, kComputeWarps);
+        mbar_init(&bars->acc_done, 1);
+        mbar_init(&bars->mma_final, 1);
+        bars->abort = (smem_u32(smem) & 1023u) ? 1 : 0;
+        if (bars->abort) record_timeout(kSiteAlign);
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(&bars->tmem_base, C::kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = bars->tmem_base;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        int last_q[2] = {-1, -1}, last_do[2] = {-1, -1};
+        bool kv_issued = false;
+        if (!*abort) {
+            if (lane == 0) {
+                tma_prefetch_desc(&tmap_q);
+                tma_prefetch_desc(&tmap_k);
+                tma_prefetch_desc(&tmap_v);
+                tma_prefetch_desc(&tmap_do);
+                mbar_arrive_expect_tx(&bars->kv_full, 2 * C::kTileBytes);
+                for (int c = 0; c < C::kChunks; ++c) {
+                    tma_load_3d(smem + C::kOffK + c * C::kChunkBytes, &tmap_k, &bars->kv_full,
+                                64 * c, kt * kTile, bh);
+                    tma_load_3d(smem + C::kOffV + c * C::kChunkBytes, &tmap_v, &bars->kv_full,
+                                64 * c, kt * kTile, bh);
+                }
+            }
+            kv_issued = true;
+            for (int n = 0; n < n_iter; ++n) {
+                const int i = i_begin + n;
+                // Q_n and the LSE/D vectors of its query tile
+                const int sq = n & 1, uq = n >> 1;
+                if (uq > 0 && !warp_wait(&bars->q_empty[sq], (uq - 1) & 1, kSiteQEmpty, abort))
+                    break;
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(&bars->q_full[sq], C::kTileBytes);
+                    for (int c = 0; c < C::kChunks; ++c)
+                        tma_load_3d(smem + C::kOffQ + sq * C::kTileBytes + c * C::kChunkBytes,
+                                    &tmap_q, &bars->q_full[sq], 64 * c, i * kTile, bh);
+                }
+                last_q[sq] = uq;
+                // LSE (to log2 units) and D of the query tile; +inf / 0 past T
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int r = lane * 4 + e;
+                    const int q = i * kTile + r;
+                    float lv = INFINITY, dv = 0.f;
+                    if (q < T) {
+                        lv = lse[(size_t)bh * T + q] * kLog2e;
+                        dv = delta[(size_t)bh * T + q];
+                    }
+                    s_lse[sq * kTile + r] = lv;
+                    s_delta[sq * kTile + r] = dv;
+                }
+                mbar_arrive(&bars->ld_full[sq]);
+                // dO_n
+                const int sd = n % C::kStagesDO, ud = n / C::kStagesDO;
+                if (ud > 0 && !warp_wait(&bars->do_empty[sd], (ud - 1) & 1, kSiteDOEmpty, abort))
+                    break;
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(&bars->do_full[sd], C::kTileBytes);
+                    for (int c = 0; c < C::kChunks; ++c)
+                        tma_load_3d(smem + C::kOffDO + sd * C::kTileBytes + c * C::kChunkBytes,
+                                    &tmap_do, &bars->do_full[sd], 64 * c, i * kTile, bh);
+                }
+                last_do[sd] = ud;
+            }
+        }
+        if (*abort && lane == 0) {
+            if (kv_issued) mbar_wait_drain(&bars->kv_full, 0);
+            for (int s = 0; s < 2; ++s) {
+                if (last_q[s] >= 0) mbar_wait_drain(&bars->q_full[s], last_q[s] & 1);
+                if (last_do[s] >= 0) mbar_wait_drain(&bars->do_full[s], last_do[s] & 1);
+            }
+        }
+    } else if (warp == 1) {
+        // --------------------------------------------------------- MMA issuer
+        if (lane == 0 && !*abort) {
+            const uint32_t tS = tmem + C::kColS;
+            const uint32_t tDP = tmem + C::kColDP;
+            const uint32_t tDQ = tmem + C::kColDQ;
+            const uint32_t tDV = tmem + C::kColDV;
+            const uint32_t tDK = tmem + C::kColDK;
+            const uint32_t k_addr = smem_u32(smem + C::kOffK);
+            const uint32_t v_addr = smem_u32(smem + C::kOffV);
+            const uint32_t p_addr = smem_u32(smem + C::kOffP);
+            const uint32_t ds_addr = smem_u32(smem + C::kOffDS);
+            bool ok = mbar_wait(&bars->kv_full, 0, kSiteKV, abort);
+
+            // S^T = K Q^T  or  dP^T = V dO^T: M = 128 keys, N = 128 queries, K = d
+            auto score_mma = [&](uint32_t d_tmem, uint32_t a_addr, uint32_t b_addr) {
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * C::kChunkBytes + (kk & 3) * 32;
+                    mma_ss(d_tmem, sdesc_sw128(a_addr + off, 16, 1024),
+                           sdesc_sw128(b_addr + off, 16, 1024), C::kIdescScore, kk > 0 ? 1u : 0u);
+                }
+            };
+            // dV += P^T dO  or  dK += dS^T Q: M = 128 keys, N = d, K = 128 queries
+            auto grad_mma = [&](uint32_t d_tmem, uint32_t a_addr, uint32_t b_addr, bool acc) {
+#pragma unroll
+                for (int kk = 0; kk < kTile / 16; ++kk) {
+                    const uint32_t aoff = (kk >> 2) * C::kChunkBytes + (kk & 3) * 32;
+                    mma_ss(d_tmem, sdesc_sw128(a_addr + aoff, 16, 1024),
+                           sdesc_sw128(b_addr + kk * 2048, C::kChunkBytes, 1024), C::kIdescGrad,
+                           (acc || kk > 0) ? 1u : 0u);
+                }
+            };
+            // dQ_i = dS K: M = 128 queries (dS^T read MN-major), N = d, K = 128 keys
+            auto dq_mma = [&](uint32_t a_addr, bool acc) {
+#pragma unroll
+                for (int kk = 0; kk < kTile / 16; ++kk)
+                    mma_ss(tDQ, sdesc_sw128(a_addr + kk * 2048, C::kChunkBytes, 1024),
+                           sdesc_sw128(k_addr + kk * 2048, C::kChunkBytes, 1024), C::kIdescDQ,
+                           (acc || kk > 0) ? 1u : 0u);
+            };
+            auto q_stage = [&](int n) {
+                return smem_u32(smem + C::kOffQ + (n & 1) * C::kTileBytes);
+            };
+            auto do_stage = [&](int n) {
+                return smem_u32(smem + C::kOffDO + (n % C::kStagesDO) * C::kTileBytes);
+            };
+
+            // prologue: S_0, dP_0
+            if (ok) ok = mbar_wait(&bars->q_full[0], 0, kSiteQFull, abort);
+            if (ok) {
+                tc_fence_after();
+                score_mma(tS, k_addr, q_stage(0));
+                mma_commit(&bars->s_full);
+            }
+            if (ok) ok = mbar_wait(&bars->do_full[0], 0, kSiteDOFull, abort);
+            if (ok) {
+                tc_fence_after();
+                score_mma(tDP, v_addr, do_stage(0));
+                mma_commit(&bars->dp_full);
+            }
+            for (int n = 0; ok && n < n_iter; ++n) {
+                const int st = n & 1;
+                // S_{n+1} as soon as the compute warps hold S_n in registers
+                if (n + 1 < n_iter) {
+                    if (!mbar_wait(&bars->s_free, n & 1, kSiteSFree, abort)) { ok = false; break; }
+                    if (!mbar_wait(&bars->q_full[(n + 1) & 1], ((n + 1) >> 1) & 1, kSiteQFull,
+                                   abort)) { ok = false; break; }
+                    tc_fence_after();
+                    score_mma(tS, k_addr, q_stage(n + 1));
+                    mma_commit(&bars->s_full);
+                }
+                // dV += P^T dO_n
+                if (!mbar_wait(&bars->p_full, n & 1, kSitePFull, abort)) { ok = false; break; }
+                tc_fence_after();
+                grad_mma(tDV, p_addr, do_stage(n), n > 0);
+                if (PRECISE) grad_mma(tDV, p_addr + C::kScoreBytes, do_stage(n), true);
+                mma_commit(&bars->p_free);
+                mma_commit(&bars->do_empty[n % C::kStagesDO]);
+                // dK += dS^T Q_n ; dQ_n = dS K
+                if (!mbar_wait(&bars->ds_full, n & 1, kSiteDSFull, abort)) { ok = false; break; }
+                tc_fence_after();
+                grad_mma(tDK, ds_addr, q_stage(n), n > 0);
+                if (PRECISE) grad_mma(tDK, ds_addr + C::kScoreBytes, q_stage(n), true);
+                // separate dQ columns: free once dQ_{n-1} is drained; shared with dP^T:
+                // dP_n has been read (ds_full)
+                if (C::kSeparateDQ && n > 0 &&
+                    !mbar_wait(&bars->dq_free, (n - 1) & 1, kSiteDQFree, abort)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                dq_mma(ds_addr, false);
+                if (PRECISE) dq_mma(ds_addr + C::kScoreBytes, true);
+                mma_commit(&bars->dq_full);
+                mma_commit(&bars->ds_free);
+                mma_commit(&bars->q_empty[st]);
+                // dP_{n+1}: its columns are free once dS_n is formed (separate dQ) or
+                // once dQ_n has left tensor memory (shared columns)
+                if (n + 1 < n_iter) {
+                    if (!C::kSeparateDQ &&
+                        !mbar_wait(&bars->dq_free, n & 1, kSiteDQFree, abort)) {
+                        ok = false;
+                        break;
+                    }
+                    if (!mbar_wait(&bars->do_full[(n + 1) % C::kStagesDO],
+                                   ((n + 1) / C::kStagesDO) & 1, kSiteDOFull, abort)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    score_mma(tDP, v_addr, do_stage(n + 1));
+                    mma_commit(&bars->dp_full);
+                }
+            }
+            if (ok) mma_commit(&bars->acc_done);
+            mma_commit(&bars->mma_final);
+            mbar_wait_drain(&bars->mma_final, 0);
+        }
+    } else {
+        // ----------------------------------------------------------- compute
+        const uint32_t quarter = warp & 3;
+        const uint32_t half = (warp - 2) >> 2;          // which 64 query columns
+        const uint32_t row = (quarter << 5) + lane;      // key row (and dQ query row)
+        const uint32_t lane_off = (quarter << 5) << 16;
+        uint8_t* p_smem = smem + C::kOffP + half * C::kChunkBytes;
+        uint8_t* ds_smem = smem + C::kOffDS + half * C::kChunkBytes;
+        const int c0 = half * 64;                        // first query column owned
+        bool ok = !*abort;
+
+        // dQ_m rows -> accumulator: this thread's query row, its half of the d columns
+        auto drain_dq = [&](int m) -> bool {
+            if (!warp_wait(&bars->dq_full, m & 1, kSiteDQFull, abort)) return false;
+            tc_fence_after();
+            uint32_t r[D / 2];
+#pragma unroll
+            for (int c = 0; c < D / 64; ++c)
+                tmem_ld32(tmem + lane_off + C::kColDQ + half * (D / 2) + c * 32, r + c * 32);
+            tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->dq_free);
+            const int q = (i_begin + m) * kTile + (int)row;
+            if (q < T) {
+                float* dst = dq_accum + ((size_t)bh * T + q) * D + half * (D / 2);
+#pragma unroll
+                for (int e = 0; e < D / 8; ++e)
+                    red_add_v4(dst + 4 * e, __uint_as_float(r[4 * e]) * scale,
+                               __uint_as_float(r[4 * e + 1]) * scale,
+                               __uint_as_float(r[4 * e + 2]) * scale,
+                               __uint_as_float(r[4 * e + 3]) * scale);
+            }
+            return true;
+        };
+
+        for (int n = 0; ok && n < n_iter; ++n) {
+            const int st = n & 1;
+            const int i = i_begin + n;
+            const bool diag = causal && (i == kt);
+            // ---- P^T for 64 query columns
+            if (!warp_wait(&bars->s_full, n & 1, kSiteSFull, abort)) { ok = false; break; }
+            tc_fence_after();
+            uint32_t sraw[64];
+            tmem_ld32(tmem + lane_off + C::kColS + c0, sraw);
+            tmem_ld32(tmem + lane_off + C::kColS + c0 + 32, sraw + 32);
+            tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->s_free);
+            if (!warp_wait(&bars->ld_full[st], (n >> 1) & 1, kSiteLdFull, abort)) { ok = false; break; }
+            const float* lse_t = s_lse + st * kTile + c0;
+            float p[64];
+#pragma unroll
+            for (int c = 0; c < 64; ++c) {
+                float x = ex2_approx(__uint_as_float(sraw[c]) * scale_log2 - lse_t[c]);
+                if (diag && c0 + c < (int)row) x = 0.f;  // query precedes the key row
+                p[c] = x;
+            }
+            // the P^T buffer must no longer be read by the previous iteration's MMAs
+            if (n > 0) {
+                uint64_t* fb = C::kSeparatePdS ? &bars->p_free : &bars->ds_free;
+                if (!warp_wait(fb, (n - 1) & 1, kSitePFree, abort)) { ok = false; break; }
+            }
+#pragma unroll
+            for (int ch = 0; ch < 8; ++ch)  // 8 chunks of 8 queries
+                store_split8<PRECISE>(p_smem, C::kScoreBytes, sw128_offset(row, ch), p + ch * 8);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->p_full);
+
+            // ---- with its own columns, dQ_{n-1} drains while dP_n / dV_n run
+            if (C::kSeparateDQ && n > 0 && !drain_dq(n - 1)) { ok = false; break; }
+
+            // ---- dS^T = P^T o (dP^T - D), 32 queries at a time
+            if (!warp_wait(&bars->dp_full, n & 1, kSiteDPFull, abort)) { ok = false; break; }
+            {
+                // dS^T buffer: free once dK/dQ of the previous iteration (separate
+                // buffers) or dV of this one (shared buffer) have read it
+                bool w = true;
+                if (C::kSeparatePdS) {
+                    if (n > 0) w = warp_wait(&bars->ds_free, (n - 1) & 1, kSiteDSFree, abort);
+                } else {
+                    w = warp_wait(&bars->p_free, n & 1, kSitePFree, abort);
+                }
+                if (!w) { ok = false; break; }
+            }
+            tc_fence_after();
+            const float* d_t = s_delta + st * kTile + c0;
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+                uint32_t dp[32];
+                tmem_ld32(tmem + lane_off + C::kColDP + c0 + c * 32, dp);
+                tmem_wait_ld();
+#pragma unroll
+                for (int ch = 0; ch < 4; ++ch) {  // 4 chunks of 8 queries
+                    float ds[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const int qc = c * 32 + ch * 8 + e;
+                        ds[e] = p[qc] * (__uint_as_float(dp[ch * 8 + e]) - d_t[qc]);
+                    }
+                    store_split8<PRECISE>(ds_smem, C::kScoreBytes, sw128_offset(row, c * 4 + ch),
+                                          ds);
+                }
+            }
+            tc_fence_before();
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->ds_full);
+
+            // ---- sharing its columns with dP^T, dQ_n drains before dP_{n+1}
+            if (!C::kSeparateDQ && !drain_dq(n)) { ok = false; break; }
+        }
+        if (ok && C::kSeparateDQ && !drain_dq(n_iter - 1)) ok = false;
+
+        // ------------------------------------------------ dK / dV epilogue
+        if (ok && warp_wait(&bars->acc_done, 0, kSiteAccDone, abort)) {
+            tc_fence_after();
+            const int key = kt * kTile + (int)row;
+            const size_t base = ((size_t)bh * T + key) * D + half * (D / 2);
+#pragma unroll
+            for (int which = 0; which < 2; ++which) {
+                const uint32_t col = (which == 0 ? C::kColDV : C::kColDK) + half * (D / 2);
+                const float mul = which == 0 ? 1.f : scale;
+                void* out = which == 0 ? dv_out : dk_out;
+#pragma unroll
+                for (int c = 0; c < D / 64; ++c) {
+                    uint32_t r[32];
+                    tmem_ld32(tmem + lane_off + col + c * 32, r);
+                    tmem_wait_ld();
+                    if (key < T) {
+                        if (grad_f32) {
+                            float* o = reinterpret_cast<float*>(out) + base + c * 32;
+#pragma unroll
+                            for (int e = 0; e < 8; ++e)
+                                reinterpret_cast<float4*>(o)[e] = make_float4(
+                                    __uint_as_float(r[4 * e]) * mul,
+                                    __uint_as_float(r[4 * e + 1]) * mul,
+                                    __uint_as_float(r[4 * e + 2]) * mul,
+                                    __uint_as_float(r[4 * e + 3]) * mul);
+                        } else {
+                            uint4* o = reinterpret_cast<uint4*>(
+                                reinterpret_cast<__nv_bfloat16*>(out) + base + c * 32);
+#pragma unroll
+                            for (int e = 0; e < 4; ++e)
+                                o[e] = make_uint4(
+                                    pack_bf16x2(__uint_as_float(r[8 * e]) * mul,
+                                                __uint_as_float(r[8 * e + 1]) * mul),
+                                    pack_bf16x2(__uint_as_float(r[8 * e + 2]) * mul,
+                                                __uint_as_float(r[8 * e + 3]) * mul),
+                                    pack_bf16x2(__uint_as_float(r[8 * e + 4]) * mul,
+                                                __uint_as_float(r[8 * e + 5]) * mul),
+                                    pack_bf16x2(__uint_as_float(r[8 * e + 6]) * mul,
+                                                __uint_as_float(r[8 * e + 7]) * mul));
+                        }
+                    }
+                }
+            }
+        }
+    }
+
+    // ------------------------------------------------------------- teardown
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, C::kTmemCols);
+    }
+}
+
+// D = rowsum(dO o O) per row (fp32), and the dQ accumulator cleared.  O is bf16 or
+// fp32 (TO); dO is bf16.
+template <int D, typename TO>
+__global__ void __launch_bounds__(256) attn_bwd_preprocess_kernel(
+    const TO* __restrict__ o, const __nv_bfloat16* __restrict__ dO, float* __restrict__ delta,
+    float* __restrict__ dq_accum, long long rows) {
+    const long long r = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (r >= rows) return;
+    const uint4* g4 = reinterpret_cast<const uint4*>(dO + r * D);
+    float acc = 0.f;
+#pragma unroll
+    for (int e = 0; e < D / 8; ++e) {
+        const uint4 b = g4[e];
+        const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&b);
+        float fo[8];
+        if constexpr (sizeof(TO) == 2) {
+            const uint4 a = reinterpret_cast<const uint4*>(o + r * D)[e];
+            const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a);
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+                const float2 f = __bfloat1622float2(a2[h]);
+                fo[2 * h] = f.x;
+                fo[2 * h + 1] = f.y;
+            }
+        } else {
+            const float4 a0 = reinterpret_cast<const float4*>(o + r * D)[2 * e];
+            const float4 a1 = reinterpret_cast<const float4*>(o + r * D)[2 * e + 1];
+            fo[0] = a0.x; fo[1] = a0.y; fo[2] = a0.z; fo[3] = a0.w;
+            fo[4] = a1.x; fo[5] = a1.y; fo[6] = a1.z; fo[7] = a1.w;
+        }
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+            const float2 fb = __bfloat1622float2(b2[h]);
+            acc = fmaf(fo[2 * h], fb.x, acc);
+            acc = fmaf(fo[2 * h + 1], fb.y, acc);
+        }
+    }
+    delta[r] = acc;
+    if (dq_accum) {
+        float4* z = reinterpret_cast<float4*>(dq_accum + r * D);
+#pragma unroll
+        for (int e = 0; e < D / 4; ++e) z[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+}
+
+// dQ = bf16(accumulator), 8 elements per thread.
+__global__ void __launch_bounds__(256) attn_bwd_dq_convert_kernel(const float* __restrict__ acc,
+                                                                  __nv_bfloat16* __restrict__ dq,
+                                                                  long long n8) {
+    const long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (t >= n8) return;
+    const float4 a = reinterpret_cast<const float4*>(acc)[2 * t];
+    const float4 b = reinterpret_cast<const float4*>(acc)[2 * t + 1];
+    reinterpret_cast<uint4*>(dq)[t] = make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w),
+                                                 pack_bf16x2(b.x, b.y), pack_bf16x2(b.z, b.w));
+}
+
+template <int D, bool PRECISE>
+cudaError_t launch_dkdv_dp(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                           const CUtensorMap& tdo, const float* lse, const float* delta,
+                           float* dq_accum, void* dk, void* dv, int BH, int T, float scale,
+                           int causal, int grad_f32, cudaStream_t stream) {
+    using C = BwdCfg<D, PRECISE>;
+    static bool configured = false;
+    if (!configured) {
+        cudaError_t e = cudaFuncSetAttribute(attn_bwd_dkdv_kernel<D, PRECISE>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             C::kSmemBytes);
+        if (e != cudaSuccess) return e;
+        configured = true;
+    }
+    const int n_kvtiles = (T + kTile - 1) / kTile;
+    dim3 grid(BH, n_kvtiles);
+    attn_bwd_dkdv_kernel<D, PRECISE><<<grid, kBwdThreads, C::kSmemBytes, stream>>>(
+        tq, tk, tv, tdo, lse, delta, dq_accum, dk, dv, T, n_kvtiles, scale, scale * kLog2e,
+        causal, grad_f32);
+    return cudaGetLastError();
+}
+
+template <int D, typename TO>
+void launch_pre(const void* o, const void* dO, float* delta, float* dq_accum, long long rows,
+                cudaStream_t stream) {
+    const int threads = 256;
+    const unsigned blocks = (unsigned)((rows + threads - 1) / threads);
+    attn_bwd_preprocess_kernel<D, TO><<<blocks, threads, 0, stream>>>(
+        static_cast<const TO*>(o), static_cast<const __nv_bfloat16*>(dO), delta, dq_accum, rows);
+}
+
+}  // namespace
+
+cudaError_t launch_bwd_preprocess(const void* o, const void* dO, float* delta, float* dq_accum,
+                                  int BH, int T, int d, int o_f32, cudaStream_t stream) {
+    const long long rows = (long long)BH * T;
+    if (d == 64) {
+        if (o_f32) launch_pre<64, float>(o, dO, delta, dq_accum, rows, stream);
+        else launch_pre<64, __nv_bfloat16>(o, dO, delta, dq_accum, rows, stream);
+    } else {
+        if (o_f32) launch_pre<128, float>(o, dO, delta, dq_accum, rows, stream);
+        else launch_pre<128, __nv_bfloat16>(o, dO, delta, dq_accum, rows, stream);
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_bwd_dkdv(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                            const CUtensorMap& tdo, const float* lse, const float* delta,
+                            float* dq_accum, void* dk, void* dv, int BH, int T, int d,
+                            float scale, int causal, int grad_f32, int precise,
+                            cudaStream_t stream) {
+    if (d == 64) {
+        if (precise)
+            return launch_dkdv_dp<64, true>(tq, tk, tv, tdo, lse, delta, dq_accum, dk, dv, BH, T,
+                                            scale, causal, grad_f32, stream);
+        return launch_dkdv_dp<64, false>(tq, tk, tv, tdo, lse, delta, dq_accum, dk, dv, BH, T,
+                                         scale, causal, grad_f32, stream);
+    }
+    if (precise)
+        return launch_dkdv_dp<128, true>(tq, tk, tv, tdo, lse, delta, dq_accum, dk, dv, BH, T,
+                                         scale, causal, grad_f32, stream);
+    return launch_dkdv_dp<128, false>(tq, tk, tv, tdo, lse, delta, dq_accum, dk, dv, BH, T,
+                                      scale, causal, grad_f32, stream);
+}
+
+cudaError_t launch_bwd_dq_convert(const float* dq_accum, void* dq, long long n,
+                                  cudaStream_t stream) {
+    const long long n8 = n / 8;  // d is a multiple of 8, so n is too
+    const int threads = 256;
+    const unsigned blocks = (unsigned)((n8 + threads - 1) / threads);
+    attn_bwd_dq_convert_kernel<<<blocks, threads, 0, stream>>>(
+        dq_accum, static_cast<__nv_bfloat16*>(dq), n8);
+    return cudaGetLastError();
+}
+
+}  // namespace forge

@@ -1,0 +1,41 @@
+// forge_internal.h -- declarations shared by the library's translation units
+// (kernel launchers and the C ABI).  Not installed; not part of the ABI.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace forge {
+
+// Tile geometry common to all attention kernels: 128 query rows x 128 keys.
+constexpr int kTile = 128;
+
+// Launchers.  Tensor maps describe bf16 [B*H][T][d] tensors with a
+// {64, 128, 1} box and 128-byte swizzle.
+cudaError_t launch_attn_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                            const CUtensorMap& to, void* o, float* lse, int BH, int T, int d,
+                            float scale, int causal, int o_f32, int precise, cudaStream_t stream);
+
+cudaError_t launch_bwd_preprocess(const void* o, const void* dO, float* delta, float* dq_accum,
+                                  int BH, int T, int d, int o_f32, cudaStream_t stream);
+
+cudaError_t launch_bwd_dkdv(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                            const CUtensorMap& tdo, const float* lse, const float* delta,
+                            float* dq_accum, void* dk, void* dv, int BH, int T, int d,
+                            float scale, int causal, int grad_f32, int precise,
+                            cudaStream_t stream);
+
+cudaError_t launch_bwd_dq_convert(const float* dq_accum, void* dq, long long n,
+                                  cudaStream_t stream);
+
+cudaError_t launch_probe_mma(const CUtensorMap& ta, const CUtensorMap& tb, const void* a_raw,
+                             float* d_out, int N, int K, int mode, cudaStream_t stream);
+
+cudaError_t launch_probe_wait_timeout(unsigned long long limit_ns, cudaStream_t stream);
+
+// Device error word accessors (defined next to the word itself).
+cudaError_t read_and_clear_device_error(unsigned int* value, cudaStream_t stream);
+
+}  // namespace forge

@@ -1,0 +1,69 @@
+"""Shared helpers of the GPU tests: run the CUDA path through the C ABI and
+compare with the oracle under the stated tolerances."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+from causal_attention_fwd_attn_b200 import _lib
+from causal_attention_fwd_attn_b200 import workloads as wl
+
+# Tolerances: relative L2 <= 1e-2 and max abs <= 2e-2 on O, dQ, dK, dV; both <= 1e-3
+# on LSE.
+TOL = {"o": (1e-2, 2e-2), "dq": (1e-2, 2e-2), "dk": (1e-2, 2e-2), "dv": (1e-2, 2e-2),
+       "lse": (1e-3, 1e-3)}
+
+
+def errors(gpu, ref):
+    g = np.asarray(gpu, dtype=np.float64)
+    r = np.asarray(ref, dtype=np.float64)
+    den = np.linalg.norm(r)
+    rel = np.linalg.norm(g - r) / den if den > 0 else np.linalg.norm(g - r)
+    return float(rel), float(np.max(np.abs(g - r))) if g.size else 0.0
+
+
+def assert_close(name, gpu, ref, what=""):
+    rel, mx = errors(gpu, ref)
+    trel, tabs = TOL[name]
+    assert np.all(np.isfinite(np.asarray(gpu, dtype=np.float64))), f"{what} {name}: non-finite"
+    assert rel <= trel and mx <= tabs, \
+        f"{what} {name}: rel-L2 {rel:.3e} (tol {trel}), max-abs {mx:.3e} (tol {tabs})"
+    return rel, mx
+
+
+def run_gpu(x, scale, causal, o_dtype=torch.bfloat16, grad_dtype=torch.bfloat16, bwd=True,
+            precise=False):
+    """Forward (and backward) through the C ABI on cuda:0.  x: dict of CPU bf16 tensors.
+    With an fp32 O the backward reads that fp32 O for its D pre-pass."""
+    dev = torch.device("cuda", 0)
+    q, k, v, dO = (x[n].to(dev) for n in ("q", "k", "v", "dO"))
+    B, H, T, d = q.shape
+    s = torch.cuda.current_stream(dev).cuda_stream
+    pflag = _lib.PRECISE if precise else 0
+    o = torch.empty((B, H, T, d), dtype=o_dtype, device=dev)
+    lse = torch.empty((B, H, T), dtype=torch.float32, device=dev)
+    fflags = (_lib.OUT_F32 if o_dtype == torch.float32 else 0) | pflag
+    _lib.check(_lib.forge_attn_fwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                      lse.data_ptr(), B, H, T, d, scale, causal, fflags, s),
+               "fwd")
+    out = {"o": o, "lse": lse}
+    if bwd:
+        ws_n = _lib.forge_attn_bwd_workspace_size(B, H, T, d)
+        ws = torch.empty(ws_n, dtype=torch.uint8, device=dev)
+        dq, dk, dv = (torch.empty((B, H, T, d), dtype=grad_dtype, device=dev) for _ in range(3))
+        bflags = ((_lib.OUT_F32 if grad_dtype == torch.float32 else 0)
+                  | (_lib.O_IN_F32 if o_dtype == torch.float32 else 0) | pflag)
+        _lib.check(_lib.forge_attn_bwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                          o.data_ptr(), dO.data_ptr(), lse.data_ptr(),
+                                          dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                                          ws.data_ptr(), ws_n, B, H, T, d, scale, causal,
+                                          bflags, s), "bwd")
+        out.update(dq=dq, dk=dk, dv=dv)
+    torch.cuda.synchronize()
+    st, detail = _lib.forge_attn_check_device_error(s)
+    assert st == _lib.OK, f"device wait timed out: 0x{detail:08x}"
+    return {n: t.float().cpu().numpy() for n, t in out.items()}
+
+
+def as_f64(x):
+    return {n: t.double().numpy() for n, t in x.items()}
