@@ -34,6 +34,7 @@ EXPORTED = [
     "forge_attn_bwd_ex", "forge_attn_bwd_preprocess", "forge_attn_bwd_dkdv",
     "forge_attn_bwd_dq_convert", "forge_attn_status_string", "forge_attn_check_device_error",
     "forge_attn_version", "forge_probe_mma", "forge_probe_wait_timeout",
+    "forge_attn_bwd_noalloc",
 ]
 
 _vp = ctypes.c_void_p
@@ -58,6 +59,8 @@ _SIGNATURES = {
     "forge_attn_version": (_i, []),
     "forge_probe_mma": (_i, [_vp, _vp, _vp, _i, _i, _i, _vp]),
     "forge_probe_wait_timeout": (_i, [ctypes.c_ulonglong, _vp]),
+    "forge_attn_bwd_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i,
+                                    _f, _i, _vp]),
 }
 
 _lib = None
@@ -138,6 +141,14 @@ def forge_attn_bwd_dkdv(q, k, v, dO, lse, delta, dq_accum, dk, dv, B, H, T, d, s
 
 def forge_attn_bwd_dq_convert(dq_accum, dq, B, H, T, d, stream):
     return load().forge_attn_bwd_dq_convert(dq_accum, dq, B, H, T, d, stream)
+
+
+def forge_attn_bwd_noalloc(q, k, v, o, dO, lse, dq, dk, dv, B, H, T, d, scale, causal, stream):
+    return load().forge_attn_bwd_noalloc(q, k, v, o, dO, lse, dq, dk, dv, B, H, T, d, scale,
+                                         causal, stream)
+
+
+NOALLOC_SCRATCH_BYTES = 64 << 20
 
 
 def forge_attn_check_device_error(stream):

@@ -146,6 +146,37 @@ int forge_attn_bwd_dkdv(const void* q, const void* k, const void* v, const void*
 int forge_attn_bwd_dq_convert(const float* dq_accum, void* dq, int B, int H, int T, int d,
                               void* stream);
 
+/*
+ * Bytes of the fixed device array that forge_attn_bwd_noalloc uses in place of a
+ * workspace: 64 MiB, enough for B*H*T*(d+1) up to about 16.7 million (for example
+ * B=4 H=16 T=2048 d=64, or B=1 H=16 T=4096 d=64).
+ */
+#define FORGE_ATTN_NOALLOC_SCRATCH_BYTES (64u << 20)
+
+/*
+ * forge_attn_bwd for callers that cannot allocate device memory (a process whose
+ * memory budget is fixed at start-up, a plugin that is handed raw device pointers
+ * but no allocator, a latency-critical loop that must not call the allocator).
+ * The paper has no counterpart; this is a property of this library, not of the
+ * method.  Same arguments, results and launch sequence as forge_attn_bwd, minus the
+ * workspace: D and the fp32 dQ accumulator live in a file-scope __device__ array of
+ * FORGE_ATTN_NOALLOC_SCRATCH_BYTES that every GPU which loads the library holds
+ * until the process exits.  No cudaMalloc, cudaFree or allocating library call is
+ * made.
+ *   - Sizes whose forge_attn_bwd_workspace_size() exceeds the array are refused
+ *     with FORGE_ATTN_ERR_WORKSPACE before any launch.
+ *   - The first call on a device looks up the array's device address (once per
+ *     device, with that device current); make that first call before any stream
+ *     capture begins.
+ *   - All calls on a device share the array, which keeps the last call's contents;
+ *     each call rewrites D and clears the accumulator first.  Calls whose kernels
+ *     can overlap on the GPU (unordered streams) race on the array and must not be
+ *     issued.
+ */
+int forge_attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
+                           const void* dO, const float* lse, void* dq, void* dk, void* dv,
+                           int B, int H, int T, int d, float scale, int causal, void* stream);
+
 /* Human-readable name of a status code (static string, never NULL). */
 const char* forge_attn_status_string(int status);
 
