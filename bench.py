@@ -162,8 +162,8 @@ def run_ours(args, rank, world, local_rank):
     dq, dk, dv = (torch.empty((B, H, T, d), dtype=torch.bfloat16, device=dev) for _ in range(3))
     ws_n = _lib.forge_attn_bwd_workspace_size(B, H, T, d)
     ws = torch.empty(ws_n, dtype=torch.uint8, device=dev)
-    delta_p = ws.data_ptr()
-    acc_p = ws.data_ptr() + ((B * H * T * 4 + 255) // 256) * 256
+    rowstats_p = ws.data_ptr()
+    acc_p = ws.data_ptr() + _lib.rowstats_bytes(B, H, T)
     stream = torch.cuda.current_stream(dev)
     s = stream.cuda_stream
 
@@ -175,14 +175,14 @@ def run_ours(args, rank, world, local_rank):
                                        lse.data_ptr(), B, H, T, d, scale, w.causal, s), "fwd")
         if ev:
             ev[1].record(stream)
-        _lib.check(_lib.forge_attn_bwd_preprocess(o.data_ptr(), dO.data_ptr(), delta_p, acc_p, B,
-                                                  H, T, d, 0, s), "pre")
+        _lib.check(_lib.forge_attn_bwd_preprocess(o.data_ptr(), dO.data_ptr(), lse.data_ptr(),
+                                                  rowstats_p, acc_p, B, H, T, d, 0, s), "pre")
         if ev:
             ev[2].record(stream)
         _lib.check(_lib.forge_attn_bwd_dkdv(q.data_ptr(), k.data_ptr(), v.data_ptr(),
-                                            dO.data_ptr(), lse.data_ptr(), delta_p, acc_p,
-                                            dk.data_ptr(), dv.data_ptr(), B, H, T, d, scale,
-                                            w.causal, 0, s), "dkdv")
+                                            dO.data_ptr(), rowstats_p, acc_p, dk.data_ptr(),
+                                            dv.data_ptr(), B, H, T, d, scale, w.causal, 0, s),
+                   "dkdv")
         if ev:
             ev[3].record(stream)
         _lib.check(_lib.forge_attn_bwd_dq_convert(acc_p, dq.data_ptr(), B, H, T, d, s), "cvt")

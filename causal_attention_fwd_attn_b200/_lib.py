@@ -50,9 +50,9 @@ _SIGNATURES = {
                             _i, _f, _i, _vp]),
     "forge_attn_bwd_ex": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _i, _i,
                                _i, _i, _f, _i, _i, _vp]),
-    "forge_attn_bwd_preprocess": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp]),
-    "forge_attn_bwd_dkdv": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i,
-                                 _f, _i, _i, _vp]),
+    "forge_attn_bwd_preprocess": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp]),
+    "forge_attn_bwd_dkdv": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i,
+                                 _i, _vp]),
     "forge_attn_bwd_dq_convert": (_i, [_vp, _vp, _i, _i, _i, _i, _vp]),
     "forge_attn_status_string": (ctypes.c_char_p, [_i]),
     "forge_attn_check_device_error": (_i, [_vp, ctypes.POINTER(ctypes.c_uint)]),
@@ -129,14 +129,21 @@ def forge_attn_bwd_ex(q, k, v, o, dO, lse, dq, dk, dv, workspace, workspace_byte
                                     workspace_bytes, B, H, T, d, scale, causal, flags, stream)
 
 
-def forge_attn_bwd_preprocess(o, dO, delta, dq_accum, B, H, T, d, flags, stream):
-    return load().forge_attn_bwd_preprocess(o, dO, delta, dq_accum, B, H, T, d, flags, stream)
+def forge_attn_bwd_preprocess(o, dO, lse, rowstats, dq_accum, B, H, T, d, flags, stream):
+    return load().forge_attn_bwd_preprocess(o, dO, lse, rowstats, dq_accum, B, H, T, d, flags,
+                                            stream)
 
 
-def forge_attn_bwd_dkdv(q, k, v, dO, lse, delta, dq_accum, dk, dv, B, H, T, d, scale, causal,
+def forge_attn_bwd_dkdv(q, k, v, dO, rowstats, dq_accum, dk, dv, B, H, T, d, scale, causal,
                         flags, stream):
-    return load().forge_attn_bwd_dkdv(q, k, v, dO, lse, delta, dq_accum, dk, dv, B, H, T, d,
+    return load().forge_attn_bwd_dkdv(q, k, v, dO, rowstats, dq_accum, dk, dv, B, H, T, d,
                                       scale, causal, flags, stream)
+
+
+def rowstats_bytes(B, H, T):
+    """Bytes of the padded row statistics at the start of the backward workspace."""
+    t_pad = -(-T // 128) * 128
+    return -(-(2 * B * H * t_pad * 4) // 256) * 256
 
 
 def forge_attn_bwd_dq_convert(dq_accum, dq, B, H, T, d, stream):

@@ -48,7 +48,9 @@ def up_to_date() -> bool:
 def build(force: bool = False, ptxas_info: bool = False, verbose: bool = False) -> str:
     if not force and not ptxas_info and up_to_date():
         return LIBRARY
-    cmd = [nvcc_path(), *ARCH, "-O3", "-lineinfo", "-std=c++17", "-rdc=true", "-shared",
+    # No relocatable device code: ptxas then honours per-warpgroup register budgets
+    # (setmaxnreg), which the forward's softmax warpgroups rely on.
+    cmd = [nvcc_path(), *ARCH, "-O3", "-lineinfo", "-std=c++17", "-shared",
            "-Xcompiler", "-fPIC", "-I", INCLUDE, "-o", LIBRARY + ".tmp"]
     if ptxas_info:
         cmd += ["-Xptxas", "-v"]

@@ -8,8 +8,10 @@
 // score matrices S^T = K Q^T and dP^T = V dO^T by exchanging operand roles
 // rather than moving data (same section).  Here:
 //
-//   attn_bwd_preprocess  D[i] = sum_k dO[i][k] O[i][k] (fp32), and the fp32 dQ
-//                        accumulator cleared.  Memory-bound, one thread per row.
+//   attn_bwd_preprocess  D[i] = sum_k dO[i][k] O[i][k] (fp32), LSE[i] * log2(e), both
+//                        padded per head to a whole number of 128-row tiles (D = 0,
+//                        LSE = +inf past T, so those queries get P = 0), and the fp32
+//                        dQ accumulator cleared.  Memory-bound.
 //   attn_bwd_dkdv        one CTA per (head, 128-key tile j), looping over the query
 //                        tiles i that see it (i >= j under the causal mask):
 //                          S^T  = K_j Q_i^T           (tcgen05, TMEM)
@@ -18,17 +20,19 @@
 //                          dS^T = P^T o (dP^T - D_i)                     (threads)
 //                          dV  += P^T dO_i ;  dK += dS^T Q_i             (tcgen05, TMEM)
 //                          dQ_i = dS K_j  (tcgen05 with dS^T read MN-major), then
-//                                 scale * dQ_i added to the fp32 accumulator with
-//                                 vector reductions (red.global.add.v4.f32).
+//                                 scale * dQ_i added to the fp32 accumulator: staged
+//                                 in shared memory and added by TMA reduce-add
+//                                 (d = 64), or with red.global.add.v4.f32 (d = 128 and
+//                                 precise mode, whose shared memory is full).
 //                        The dQ stage of the paper is fused here: its partial sums
 //                        come out of the same recomputation, and reductions in L2
 //                        replace the paper's second pass over the scores.
 //   attn_bwd_dq_convert  dQ = bf16(accumulator).
 //
 // dkdv warp roles (320 threads):
-//   warp 0      producer: K_j, V_j once; Q_i, dO_i by TMA into staged rings; the
-//               LSE_i and D_i vectors (128 floats each) by plain loads into shared
-//               memory (queries past T get LSE = +inf, so their P is exactly 0).
+//   warp 0      producer (one thread): K_j, V_j once; Q_i, dO_i by TMA into staged
+//               rings; the LSE_i and D_i vectors (128 floats each) by 1-D bulk copies
+//               from the padded row statistics, counted on Q_i's barrier.
 //   warp 1      MMA issuer (one thread).
 //   warps 2..9  compute: warp w owns TMEM lanes 32*(w%4).. (key rows of the tile)
 //               and half h = (w-2)/4 of the 128 query columns.  Each thread writes
@@ -50,7 +54,7 @@ constexpr int kComputeWarps = 8;
 constexpr float kLog2e = 1.4426950408889634f;
 
 enum : uint32_t {
-    kSiteKV = 1, kSiteQFull, kSiteDOFull, kSiteLdFull, kSiteQEmpty, kSiteDOEmpty, kSiteSFull,
+    kSiteKV = 1, kSiteQFull, kSiteDOFull, kSiteQEmpty, kSiteDOEmpty, kSiteSFull,
     kSiteSFree, kSiteDPFull, kSitePFull, kSitePFree, kSiteDSFull, kSiteDSFree, kSiteDQFull,
     kSiteDQFree, kSiteAccDone, kSiteAlign
 };
@@ -60,7 +64,9 @@ struct BwdCfg {
     static constexpr int kChunks = D / 64;
     static constexpr int kChunkBytes = kTile * 128;        // 128 rows x 128 bytes
     static constexpr int kTileBytes = kChunks * kChunkBytes;
-    static constexpr int kStagesQ = 2;
+    // dQ through shared memory and a TMA reduce where there is room (d = 64 default)
+    static constexpr bool kTmaDQ = (D == 64 && !PRECISE);
+    static constexpr int kStagesQ = kTmaDQ ? 3 : 2;
     // Precise mode at d = 128 needs the room of one dO stage for the lo buffer.
     static constexpr int kStagesDO = (D == 128 && PRECISE) ? 1 : 2;
     // P^T and dS^T: [128 keys][128 queries] bf16 = two 64-query chunks; in precise
@@ -72,13 +78,16 @@ struct BwdCfg {
     static constexpr bool kSeparatePdS = (D == 64);
     // With d = 64 dQ_i has tensor-memory columns of its own.
     static constexpr bool kSeparateDQ = (D == 64);
+    // dQ staging for the TMA reduce: per column half, [128 rows][32 fp32] swizzled
+    static constexpr int kDQStageBytes = kTile * 32 * 4;
     static constexpr int kOffK = 0;
     static constexpr int kOffV = kOffK + kTileBytes;
     static constexpr int kOffQ = kOffV + kTileBytes;
     static constexpr int kOffDO = kOffQ + kStagesQ * kTileBytes;
     static constexpr int kOffP = kOffDO + kStagesDO * kTileBytes;
     static constexpr int kOffDS = kSeparatePdS ? kOffP + kSplit * kScoreBytes : kOffP;
-    static constexpr int kOffLse = kOffDS + kSplit * kScoreBytes;
+    static constexpr int kOffDQS = kOffDS + kSplit * kScoreBytes;
+    static constexpr int kOffLse = kOffDQS + (kTmaDQ ? 2 * kDQStageBytes : 0);
     static constexpr int kOffDelta = kOffLse + kStagesQ * kTile * 4;
     static constexpr int kOffBar = kOffDelta + kStagesQ * kTile * 4;
     static constexpr int kSmemBytes = kOffBar + 256;
@@ -94,10 +103,9 @@ struct BwdCfg {
 
 struct BwdBarriers {
     uint64_t kv_full;
-    uint64_t q_full[2];
+    uint64_t q_full[3];
     uint64_t do_full[2];
-    uint64_t ld_full[2];
-    uint64_t q_empty[2];
+    uint64_t q_empty[3];
     uint64_t do_empty[2];
     uint64_t s_full, s_free, dp_full, p_full, p_free, ds_full, ds_free, dq_full, dq_free;
     uint64_t acc_done, mma_final;
@@ -143,10 +151,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                          const __grid_constant__ CUtensorMap tmap_k,
                          const __grid_constant__ CUtensorMap tmap_v,
                          const __grid_constant__ CUtensorMap tmap_do,
-                         const float* __restrict__ lse, const float* __restrict__ delta,
-                         float* __restrict__ dq_accum, void* __restrict__ dk_out,
-                         void* __restrict__ dv_out, int T, int n_kvtiles, float scale,
-                         float scale_log2, int causal, int grad_f32) {
+                         const __grid_constant__ CUtensorMap tmap_dq,
+                         const float* __restrict__ rowstats, float* __restrict__ dq_accum,
+                         void* __restrict__ dk_out, void* __restrict__ dv_out, int T, int BH,
+                         int n_kvtiles, float scale, float scale_log2, int causal, int grad_f32) {
     using C = BwdCfg<D, PRECISE>;
     extern __shared__ __align__(1024) uint8_t smem[];
     BwdBarriers* bars = reinterpret_cast<BwdBarriers*>(smem + C::kOffBar);
@@ -155,8 +163,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     float* s_delta = reinterpret_cast<float*>(smem + C::kOffDelta);
 
     const int bh = blockIdx.x;
-    const int kt = n_kvtiles - 1 - blockIdx.y;  // key tile; the most query tiles first
+    const int kt = blockIdx.y;  // key tile: tile 0 sees the most query tiles, so it goes first
     const int n_qtiles = n_kvtiles;
+    const int t_pad = n_qtiles * kTile;  // row-statistics stride per head
     const int i_begin = causal ? kt : 0;
     const int n_iter = n_qtiles - i_begin;
     const uint32_t warp = warp_id();
@@ -164,11 +173,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
     if (threadIdx.x == 0) {
         mbar_init(&bars->kv_full, 1);
-        for (int s = 0; s < 2; ++s) {
+        for (int s = 0; s < 3; ++s) {
             mbar_init(&bars->q_full[s], 1);
-            mbar_init(&bars->do_full[s], 1);
-            mbar_init(&bars->ld_full[s], 32);
             mbar_init(&bars->q_empty[s], 1);
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&bars->do_full[s], 1);
             mbar_init(&bars->do_empty[s], 1);
         }
         mbar_init(&bars->s_full, 1);
@@ -197,10 +207,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
-        int last_q[2] = {-1, -1}, last_do[2] = {-1, -1};
-        bool kv_issued = false;
-        if (!*abort) {
-            if (lane == 0) {
+        if (lane == 0) {
+            int last_q[3] = {-1, -1, -1}, last_do[2] = {-1, -1};
+            bool kv_issued = false;
+            if (!*abort) {
                 tma_prefetch_desc(&tmap_q);
                 tma_prefetch_desc(&tmap_k);
                 tma_prefetch_desc(&tmap_v);
@@ -212,53 +222,42 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     tma_load_3d(smem + C::kOffV + c * C::kChunkBytes, &tmap_v, &bars->kv_full,
                                 64 * c, kt * kTile, bh);
                 }
-            }
-            kv_issued = true;
-            for (int n = 0; n < n_iter; ++n) {
-                const int i = i_begin + n;
-                // Q_n and the LSE/D vectors of its query tile
-                const int sq = n & 1, uq = n >> 1;
-                if (uq > 0 && !warp_wait(&bars->q_empty[sq], (uq - 1) & 1, kSiteQEmpty, abort))
-                    break;
-                if (lane == 0) {
-                    mbar_arrive_expect_tx(&bars->q_full[sq], C::kTileBytes);
+                kv_issued = true;
+                const float* lse2_head = rowstats + (size_t)bh * t_pad;
+                const float* delta_head = rowstats + (size_t)BH * t_pad + (size_t)bh * t_pad;
+                for (int n = 0; n < n_iter; ++n) {
+                    const int i = i_begin + n;
+                    // Q_n with the LSE and D vectors of its query tile
+                    const int sq = n % C::kStagesQ, uq = n / C::kStagesQ;
+                    if (uq > 0 && !mbar_wait(&bars->q_empty[sq], (uq - 1) & 1, kSiteQEmpty, abort))
+                        break;
+                    mbar_arrive_expect_tx(&bars->q_full[sq], C::kTileBytes + 2 * kTile * 4);
                     for (int c = 0; c < C::kChunks; ++c)
                         tma_load_3d(smem + C::kOffQ + sq * C::kTileBytes + c * C::kChunkBytes,
                                     &tmap_q, &bars->q_full[sq], 64 * c, i * kTile, bh);
-                }
-                last_q[sq] = uq;
-                // LSE (to log2 units) and D of the query tile; +inf / 0 past T
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int r = lane * 4 + e;
-                    const int q = i * kTile + r;
-                    float lv = INFINITY, dv = 0.f;
-                    if (q < T) {
-                        lv = lse[(size_t)bh * T + q] * kLog2e;
-                        dv = delta[(size_t)bh * T + q];
-                    }
-                    s_lse[sq * kTile + r] = lv;
-                    s_delta[sq * kTile + r] = dv;
-                }
-                mbar_arrive(&bars->ld_full[sq]);
-                // dO_n
-                const int sd = n % C::kStagesDO, ud = n / C::kStagesDO;
-                if (ud > 0 && !warp_wait(&bars->do_empty[sd], (ud - 1) & 1, kSiteDOEmpty, abort))
-                    break;
-                if (lane == 0) {
+                    bulk_load(s_lse + sq * kTile, lse2_head + i * kTile, kTile * 4,
+                              &bars->q_full[sq]);
+                    bulk_load(s_delta + sq * kTile, delta_head + i * kTile, kTile * 4,
+                              &bars->q_full[sq]);
+                    last_q[sq] = uq;
+                    // dO_n
+                    const int sd = n % C::kStagesDO, ud = n / C::kStagesDO;
+                    if (ud > 0 &&
+                        !mbar_wait(&bars->do_empty[sd], (ud - 1) & 1, kSiteDOEmpty, abort))
+                        break;
                     mbar_arrive_expect_tx(&bars->do_full[sd], C::kTileBytes);
                     for (int c = 0; c < C::kChunks; ++c)
                         tma_load_3d(smem + C::kOffDO + sd * C::kTileBytes + c * C::kChunkBytes,
                                     &tmap_do, &bars->do_full[sd], 64 * c, i * kTile, bh);
+                    last_do[sd] = ud;
                 }
-                last_do[sd] = ud;
             }
-        }
-        if (*abort && lane == 0) {
-            if (kv_issued) mbar_wait_drain(&bars->kv_full, 0);
-            for (int s = 0; s < 2; ++s) {
-                if (last_q[s] >= 0) mbar_wait_drain(&bars->q_full[s], last_q[s] & 1);
-                if (last_do[s] >= 0) mbar_wait_drain(&bars->do_full[s], last_do[s] & 1);
+            if (*abort) {
+                if (kv_issued) mbar_wait_drain(&bars->kv_full, 0);
+                for (int s = 0; s < 3; ++s)
+                    if (last_q[s] >= 0) mbar_wait_drain(&bars->q_full[s], last_q[s] & 1);
+                for (int s = 0; s < 2; ++s)
+                    if (last_do[s] >= 0) mbar_wait_drain(&bars->do_full[s], last_do[s] & 1);
             }
         }
     } else if (warp == 1) {
@@ -303,7 +302,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                            (acc || kk > 0) ? 1u : 0u);
             };
             auto q_stage = [&](int n) {
-                return smem_u32(smem + C::kOffQ + (n & 1) * C::kTileBytes);
+                return smem_u32(smem + C::kOffQ + (n % C::kStagesQ) * C::kTileBytes);
             };
             auto do_stage = [&](int n) {
                 return smem_u32(smem + C::kOffDO + (n % C::kStagesDO) * C::kTileBytes);
@@ -323,12 +322,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 mma_commit(&bars->dp_full);
             }
             for (int n = 0; ok && n < n_iter; ++n) {
-                const int st = n & 1;
                 // S_{n+1} as soon as the compute warps hold S_n in registers
                 if (n + 1 < n_iter) {
                     if (!mbar_wait(&bars->s_free, n & 1, kSiteSFree, abort)) { ok = false; break; }
-                    if (!mbar_wait(&bars->q_full[(n + 1) & 1], ((n + 1) >> 1) & 1, kSiteQFull,
-                                   abort)) { ok = false; break; }
+                    if (!mbar_wait(&bars->q_full[(n + 1) % C::kStagesQ],
+                                   ((n + 1) / C::kStagesQ) & 1, kSiteQFull, abort)) {
+                        ok = false;
+                        break;
+                    }
                     tc_fence_after();
                     score_mma(tS, k_addr, q_stage(n + 1));
                     mma_commit(&bars->s_full);
@@ -357,7 +358,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 if (PRECISE) dq_mma(ds_addr + C::kScoreBytes, true);
                 mma_commit(&bars->dq_full);
                 mma_commit(&bars->ds_free);
-                mma_commit(&bars->q_empty[st]);
+                mma_commit(&bars->q_empty[n % C::kStagesQ]);
                 // dP_{n+1}: its columns are free once dS_n is formed (separate dQ) or
                 // once dQ_n has left tensor memory (shared columns)
                 if (n + 1 < n_iter) {
@@ -388,10 +389,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const uint32_t lane_off = (quarter << 5) << 16;
         uint8_t* p_smem = smem + C::kOffP + half * C::kChunkBytes;
         uint8_t* ds_smem = smem + C::kOffDS + half * C::kChunkBytes;
+        uint8_t* dq_stage = smem + C::kOffDQS + half * C::kDQStageBytes;
+        const bool leader = lane == 0 && quarter == 2;   // warps 2 and 6: one per half
         const int c0 = half * 64;                        // first query column owned
         bool ok = !*abort;
 
-        // dQ_m rows -> accumulator: this thread's query row, its half of the d columns
+        // dQ_m: this thread's query row, its half of the d columns, times scale,
+        // into the fp32 accumulator
         auto drain_dq = [&](int m) -> bool {
             if (!warp_wait(&bars->dq_full, m & 1, kSiteDQFull, abort)) return false;
             tc_fence_after();
@@ -403,21 +407,40 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars->dq_free);
-            const int q = (i_begin + m) * kTile + (int)row;
-            if (q < T) {
-                float* dst = dq_accum + ((size_t)bh * T + q) * D + half * (D / 2);
+            const int i = i_begin + m;
+            if constexpr (C::kTmaDQ) {
+                // staging must have been read by this half's previous reduce
+                if (leader) tma_store_wait_all_read();
+                named_bar_sync(2 + half, 128);
 #pragma unroll
-                for (int e = 0; e < D / 8; ++e)
-                    red_add_v4(dst + 4 * e, __uint_as_float(r[4 * e]) * scale,
-                               __uint_as_float(r[4 * e + 1]) * scale,
-                               __uint_as_float(r[4 * e + 2]) * scale,
-                               __uint_as_float(r[4 * e + 3]) * scale);
+                for (int ch = 0; ch < 8; ++ch)
+                    *reinterpret_cast<float4*>(dq_stage + sw128_offset(row, ch)) = make_float4(
+                        __uint_as_float(r[4 * ch]) * scale, __uint_as_float(r[4 * ch + 1]) * scale,
+                        __uint_as_float(r[4 * ch + 2]) * scale,
+                        __uint_as_float(r[4 * ch + 3]) * scale);
+                fence_proxy_async_smem();
+                named_bar_sync(2 + half, 128);
+                if (leader) {
+                    tma_reduce_add_3d(&tmap_dq, dq_stage, 32 * half, i * kTile, bh);
+                    tma_store_commit();
+                }
+            } else {
+                const int q = i * kTile + (int)row;
+                if (q < T) {
+                    float* dst = dq_accum + ((size_t)bh * T + q) * D + half * (D / 2);
+#pragma unroll
+                    for (int e = 0; e < D / 8; ++e)
+                        red_add_v4(dst + 4 * e, __uint_as_float(r[4 * e]) * scale,
+                                   __uint_as_float(r[4 * e + 1]) * scale,
+                                   __uint_as_float(r[4 * e + 2]) * scale,
+                                   __uint_as_float(r[4 * e + 3]) * scale);
+                }
             }
             return true;
         };
 
         for (int n = 0; ok && n < n_iter; ++n) {
-            const int st = n & 1;
+            const int sq = n % C::kStagesQ;
             const int i = i_begin + n;
             const bool diag = causal && (i == kt);
             // ---- P^T for 64 query columns
@@ -430,14 +453,24 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars->s_free);
-            if (!warp_wait(&bars->ld_full[st], (n >> 1) & 1, kSiteLdFull, abort)) { ok = false; break; }
-            const float* lse_t = s_lse + st * kTile + c0;
+            // LSE_i and D_i arrived with Q_i
+            if (!warp_wait(&bars->q_full[sq], (n / C::kStagesQ) & 1, kSiteQFull, abort)) {
+                ok = false;
+                break;
+            }
+            const float4* lse4 = reinterpret_cast<const float4*>(s_lse + sq * kTile + c0);
             float p[64];
 #pragma unroll
-            for (int c = 0; c < 64; ++c) {
-                float x = ex2_approx(__uint_as_float(sraw[c]) * scale_log2 - lse_t[c]);
-                if (diag && c0 + c < (int)row) x = 0.f;  // query precedes the key row
-                p[c] = x;
+            for (int c4 = 0; c4 < 16; ++c4) {
+                const float4 l = lse4[c4];
+                const float lv[4] = {l.x, l.y, l.z, l.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int c = 4 * c4 + e;
+                    float x = ex2_approx(fmaf(__uint_as_float(sraw[c]), scale_log2, -lv[e]));
+                    if (diag && c0 + c < (int)row) x = 0.f;  // query precedes the key row
+                    p[c] = x;
+                }
             }
             // the P^T buffer must no longer be read by the previous iteration's MMAs
             if (n > 0) {
@@ -468,7 +501,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 if (!w) { ok = false; break; }
             }
             tc_fence_after();
-            const float* d_t = s_delta + st * kTile + c0;
+            const float4* d4 = reinterpret_cast<const float4*>(s_delta + sq * kTile + c0);
 #pragma unroll
             for (int c = 0; c < 2; ++c) {
                 uint32_t dp[32];
@@ -476,11 +509,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 tmem_wait_ld();
 #pragma unroll
                 for (int ch = 0; ch < 4; ++ch) {  // 4 chunks of 8 queries
+                    const float4 da = d4[c * 8 + ch * 2], db = d4[c * 8 + ch * 2 + 1];
+                    const float dv8[8] = {da.x, da.y, da.z, da.w, db.x, db.y, db.z, db.w};
                     float ds[8];
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
                         const int qc = c * 32 + ch * 8 + e;
-                        ds[e] = p[qc] * (__uint_as_float(dp[ch * 8 + e]) - d_t[qc]);
+                        ds[e] = p[qc] * (__uint_as_float(dp[ch * 8 + e]) - dv8[e]);
                     }
                     store_split8<PRECISE>(ds_smem, C::kScoreBytes, sw128_offset(row, c * 4 + ch),
                                           ds);
@@ -495,6 +530,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             if (!C::kSeparateDQ && !drain_dq(n)) { ok = false; break; }
         }
         if (ok && C::kSeparateDQ && !drain_dq(n_iter - 1)) ok = false;
+        if (C::kTmaDQ && leader) tma_store_wait_all();  // reduces done before the CTA exits
 
         // ------------------------------------------------ dK / dV epilogue
         if (ok && warp_wait(&bars->acc_done, 0, kSiteAccDone, abort)) {
@@ -552,23 +588,31 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
 }
 
-// D = rowsum(dO o O) per row (fp32), and the dQ accumulator cleared.  O is bf16 or
-// fp32 (TO); dO is bf16.
+// Row statistics of the backward, padded per head to t_pad = 128 * ceil(T / 128) rows:
+// rowstats[0][bh][t] = LSE * log2(e) and rowstats[1][bh][t] = D = rowsum(dO o O)
+// (fp32; +inf and 0 past T), and the dQ accumulator cleared.  O is bf16 or fp32
+// (TO); dO is bf16.  A group of D/8 consecutive threads covers one row, 8 elements
+// each, so every load of a warp is one contiguous span.
 template <int D, typename TO>
 __global__ void __launch_bounds__(256) attn_bwd_preprocess_kernel(
-    const TO* __restrict__ o, const __nv_bfloat16* __restrict__ dO, float* __restrict__ delta,
-    float* __restrict__ dq_accum, long long rows) {
-    const long long r = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-    if (r >= rows) return;
-    const uint4* g4 = reinterpret_cast<const uint4*>(dO + r * D);
+    const TO* __restrict__ o, const __nv_bfloat16* __restrict__ dO,
+    const float* __restrict__ lse, float* __restrict__ rowstats, float* __restrict__ dq_accum,
+    int T, int t_pad, long long padded_rows) {
+    constexpr int kGroup = D / 8;  // threads per row
+    const long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    const long long pr = t / kGroup;  // padded row index
+    const int part = (int)(t % kGroup);
+    const long long bh = pr / t_pad;
+    const int tr = (int)(pr % t_pad);
+    const bool valid = pr < padded_rows && tr < T;
+    const long long r = bh * T + tr;  // row in the [B*H][T] tensors
     float acc = 0.f;
-#pragma unroll
-    for (int e = 0; e < D / 8; ++e) {
-        const uint4 b = g4[e];
+    if (valid) {
+        const uint4 b = reinterpret_cast<const uint4*>(dO + r * D)[part];
         const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&b);
         float fo[8];
         if constexpr (sizeof(TO) == 2) {
-            const uint4 a = reinterpret_cast<const uint4*>(o + r * D)[e];
+            const uint4 a = reinterpret_cast<const uint4*>(o + r * D)[part];
             const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a);
 #pragma unroll
             for (int h = 0; h < 4; ++h) {
@@ -577,8 +621,8 @@ __global__ void __launch_bounds__(256) attn_bwd_preprocess_kernel(
                 fo[2 * h + 1] = f.y;
             }
         } else {
-            const float4 a0 = reinterpret_cast<const float4*>(o + r * D)[2 * e];
-            const float4 a1 = reinterpret_cast<const float4*>(o + r * D)[2 * e + 1];
+            const float4 a0 = reinterpret_cast<const float4*>(o + r * D)[2 * part];
+            const float4 a1 = reinterpret_cast<const float4*>(o + r * D)[2 * part + 1];
             fo[0] = a0.x; fo[1] = a0.y; fo[2] = a0.z; fo[3] = a0.w;
             fo[4] = a1.x; fo[5] = a1.y; fo[6] = a1.z; fo[7] = a1.w;
         }
@@ -588,12 +632,17 @@ __global__ void __launch_bounds__(256) attn_bwd_preprocess_kernel(
             acc = fmaf(fo[2 * h], fb.x, acc);
             acc = fmaf(fo[2 * h + 1], fb.y, acc);
         }
+        if (dq_accum) {
+            float4* z = reinterpret_cast<float4*>(dq_accum + r * D) + 2 * part;
+            z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+            z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
     }
-    delta[r] = acc;
-    if (dq_accum) {
-        float4* z = reinterpret_cast<float4*>(dq_accum + r * D);
 #pragma unroll
-        for (int e = 0; e < D / 4; ++e) z[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int off = kGroup / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (pr < padded_rows && part == 0) {
+        rowstats[pr] = valid ? lse[r] * kLog2e : INFINITY;
+        rowstats[padded_rows + pr] = valid ? acc : 0.f;
     }
 }
 
@@ -611,7 +660,7 @@ __global__ void __launch_bounds__(256) attn_bwd_dq_convert_kernel(const float* _
 
 template <int D, bool PRECISE>
 cudaError_t launch_dkdv_dp(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                           const CUtensorMap& tdo, const float* lse, const float* delta,
+                           const CUtensorMap& tdo, const CUtensorMap& tdq, const float* rowstats,
                            float* dq_accum, void* dk, void* dv, int BH, int T, float scale,
                            int causal, int grad_f32, cudaStream_t stream) {
     using C = BwdCfg<D, PRECISE>;
@@ -626,51 +675,55 @@ cudaError_t launch_dkdv_dp(const CUtensorMap& tq, const CUtensorMap& tk, const C
     const int n_kvtiles = (T + kTile - 1) / kTile;
     dim3 grid(BH, n_kvtiles);
     attn_bwd_dkdv_kernel<D, PRECISE><<<grid, kBwdThreads, C::kSmemBytes, stream>>>(
-        tq, tk, tv, tdo, lse, delta, dq_accum, dk, dv, T, n_kvtiles, scale, scale * kLog2e,
+        tq, tk, tv, tdo, tdq, rowstats, dq_accum, dk, dv, T, BH, n_kvtiles, scale, scale * kLog2e,
         causal, grad_f32);
     return cudaGetLastError();
 }
 
 template <int D, typename TO>
-void launch_pre(const void* o, const void* dO, float* delta, float* dq_accum, long long rows,
-                cudaStream_t stream) {
+void launch_pre(const void* o, const void* dO, const float* lse, float* rowstats,
+                float* dq_accum, int BH, int T, cudaStream_t stream) {
+    const int t_pad = ((T + kTile - 1) / kTile) * kTile;
+    const long long padded_rows = (long long)BH * t_pad;
     const int threads = 256;
-    const unsigned blocks = (unsigned)((rows + threads - 1) / threads);
+    const long long total = padded_rows * (D / 8);
+    const unsigned blocks = (unsigned)((total + threads - 1) / threads);
     attn_bwd_preprocess_kernel<D, TO><<<blocks, threads, 0, stream>>>(
-        static_cast<const TO*>(o), static_cast<const __nv_bfloat16*>(dO), delta, dq_accum, rows);
+        static_cast<const TO*>(o), static_cast<const __nv_bfloat16*>(dO), lse, rowstats, dq_accum,
+        T, t_pad, padded_rows);
 }
 
 }  // namespace
 
-cudaError_t launch_bwd_preprocess(const void* o, const void* dO, float* delta, float* dq_accum,
-                                  int BH, int T, int d, int o_f32, cudaStream_t stream) {
-    const long long rows = (long long)BH * T;
+cudaError_t launch_bwd_preprocess(const void* o, const void* dO, const float* lse,
+                                  float* rowstats, float* dq_accum, int BH, int T, int d,
+                                  int o_f32, cudaStream_t stream) {
     if (d == 64) {
-        if (o_f32) launch_pre<64, float>(o, dO, delta, dq_accum, rows, stream);
-        else launch_pre<64, __nv_bfloat16>(o, dO, delta, dq_accum, rows, stream);
+        if (o_f32) launch_pre<64, float>(o, dO, lse, rowstats, dq_accum, BH, T, stream);
+        else launch_pre<64, __nv_bfloat16>(o, dO, lse, rowstats, dq_accum, BH, T, stream);
     } else {
-        if (o_f32) launch_pre<128, float>(o, dO, delta, dq_accum, rows, stream);
-        else launch_pre<128, __nv_bfloat16>(o, dO, delta, dq_accum, rows, stream);
+        if (o_f32) launch_pre<128, float>(o, dO, lse, rowstats, dq_accum, BH, T, stream);
+        else launch_pre<128, __nv_bfloat16>(o, dO, lse, rowstats, dq_accum, BH, T, stream);
     }
     return cudaGetLastError();
 }
 
 cudaError_t launch_bwd_dkdv(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                            const CUtensorMap& tdo, const float* lse, const float* delta,
+                            const CUtensorMap& tdo, const CUtensorMap& tdq, const float* rowstats,
                             float* dq_accum, void* dk, void* dv, int BH, int T, int d,
                             float scale, int causal, int grad_f32, int precise,
                             cudaStream_t stream) {
     if (d == 64) {
         if (precise)
-            return launch_dkdv_dp<64, true>(tq, tk, tv, tdo, lse, delta, dq_accum, dk, dv, BH, T,
-                                            scale, causal, grad_f32, stream);
-        return launch_dkdv_dp<64, false>(tq, tk, tv, tdo, lse, delta, dq_accum, dk, dv, BH, T,
+            return launch_dkdv_dp<64, true>(tq, tk, tv, tdo, tdq, rowstats, dq_accum, dk, dv, BH,
+                                            T, scale, causal, grad_f32, stream);
+        return launch_dkdv_dp<64, false>(tq, tk, tv, tdo, tdq, rowstats, dq_accum, dk, dv, BH, T,
                                          scale, causal, grad_f32, stream);
     }
     if (precise)
-        return launch_dkdv_dp<128, true>(tq, tk, tv, tdo, lse, delta, dq_accum, dk, dv, BH, T,
+        return launch_dkdv_dp<128, true>(tq, tk, tv, tdo, tdq, rowstats, dq_accum, dk, dv, BH, T,
                                          scale, causal, grad_f32, stream);
-    return launch_dkdv_dp<128, false>(tq, tk, tv, tdo, lse, delta, dq_accum, dk, dv, BH, T,
+    return launch_dkdv_dp<128, false>(tq, tk, tv, tdo, tdq, rowstats, dq_accum, dk, dv, BH, T,
                                       scale, causal, grad_f32, stream);
 }
 
@@ -682,6 +735,10 @@ cudaError_t launch_bwd_dq_convert(const float* dq_accum, void* dq, long long n,
     attn_bwd_dq_convert_kernel<<<blocks, threads, 0, stream>>>(
         dq_accum, static_cast<__nv_bfloat16*>(dq), n8);
     return cudaGetLastError();
+}
+
+cudaError_t read_and_clear_device_error_bwd(unsigned int* value) {
+    return read_and_clear_unit_error(value);
 }
 
 }  // namespace forge

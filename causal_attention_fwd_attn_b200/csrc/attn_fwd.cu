@@ -86,7 +86,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                     const __grid_constant__ CUtensorMap tmap_v,
                     const __grid_constant__ CUtensorMap tmap_o, void* __restrict__ o_f32_out,
                     float* __restrict__ lse_out, int T, int n_qtiles, float scale_log2,
-                    int causal, int o_f32) {
+                    int negate_scores, int causal, int o_f32) {
     using C = FwdCfg<D>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -169,6 +169,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             const uint32_t tS = tmem + C::kColS;
             const uint32_t tO = tmem + C::kColO;
             const uint32_t q_addr = smem_u32(smem + C::kOffQ);
+            // bit 13 of the instruction descriptor negates A: S = (-Q) K^T for scale < 0
+            const uint32_t idesc_s = C::kIdescS | (negate_scores ? (1u << 13) : 0u);
             bool ok = mbar_wait(&bars->q_full, 0, kSiteQ, abort);
             auto issue_pv = [&](int m) -> bool {
                 const int st = m % C::kStages;
@@ -207,7 +209,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                     const uint32_t koff = (kk >> 2) * C::kChunkBytes + (kk & 3) * 32;
                     const uint64_t adesc = sdesc_sw128(q_addr + koff, 16, 1024);
                     const uint64_t bdesc = sdesc_sw128(k_addr + koff, 16, 1024);
-                    mma_ss(tS, adesc, bdesc, C::kIdescS, kk > 0 ? 1u : 0u);
+                    mma_ss(tS, adesc, bdesc, idesc_s, kk > 0 ? 1u : 0u);
                 }
                 mma_commit(&bars->s_full);
                 if (n > 0 && !issue_pv(n - 1)) {
@@ -246,21 +248,27 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars->s_free);
 
-            // scores to log2 units, masking
+            // Row max of the raw scores over the keys this row may see.  scale_log2 is
+            // >= 0 (a negative scale is applied by negating Q in the MMA), so the max
+            // of the scaled scores is scale_log2 times the raw max.
             const bool diag = causal && j == qt;
             const bool tail = !causal && (j + 1) * kTile > T;
-            const int key0 = j * kTile;
-            float u[kTile];
+            const bool masked_tile = diag || tail;
+            const int key_lim = diag ? (int)row : (tail ? T - 1 - j * kTile : kTile - 1);
+            float s[kTile];
 #pragma unroll
             for (int c = 0; c < kTile; ++c) {
-                float x = __uint_as_float(sraw[c]) * scale_log2;
-                if (diag && c > (int)row) x = -INFINITY;
-                if (tail && key0 + c >= T) x = -INFINITY;
-                u[c] = x;
+                s[c] = __uint_as_float(sraw[c]);
+                if (masked_tile && c > key_lim) s[c] = -INFINITY;
             }
-            float mt = -INFINITY;
+            float mx[8];
 #pragma unroll
-            for (int c = 0; c < kTile; ++c) mt = fmaxf(mt, u[c]);
+            for (int e = 0; e < 8; ++e) mx[e] = s[e];
+#pragma unroll
+            for (int c = 8; c < kTile; ++c) mx[c & 7] = fmaxf(mx[c & 7], s[c]);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) mx[e] = fmaxf(mx[e], mx[e + 4]);
+            const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * scale_log2;
 
             float alpha = 1.f;
             bool need = false;
@@ -293,19 +301,27 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 tmem_wait_st();
             }
 
-            // P = exp2(u - m), row sum, pack to bf16 pairs and store to TMEM
+            // P = exp2(s * scale_log2 - m), row sum, pack to bf16 pairs, store to TMEM
             const uint32_t tP = tmem + lane_off + ((n & 1) ? C::kColP1 : C::kColP0);
             const uint32_t tPlo = tmem + lane_off + ((n & 1) ? C::kColPlo1 : C::kColPlo0);
-            float ls0 = 0.f, ls1 = 0.f;
+            const float neg_m = -m_run;
+            float ls[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) ls[e] = 0.f;
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
                 uint32_t pk[32], pl[32];
 #pragma unroll
                 for (int e = 0; e < 32; ++e) {
-                    const float p0 = ex2_approx(u[half * 64 + 2 * e] - m_run);
-                    const float p1 = ex2_approx(u[half * 64 + 2 * e + 1] - m_run);
-                    ls0 += p0;
-                    ls1 += p1;
+                    const int c = half * 64 + 2 * e;
+                    float p0 = ex2_approx(fmaf(s[c], scale_log2, neg_m));
+                    float p1 = ex2_approx(fmaf(s[c + 1], scale_log2, neg_m));
+                    if (masked_tile) {  // also covers scale 0, where -inf * 0 is NaN
+                        p0 = c > key_lim ? 0.f : p0;
+                        p1 = c + 1 > key_lim ? 0.f : p1;
+                    }
+                    ls[(2 * e) & 7] += p0;
+                    ls[(2 * e + 1) & 7] += p1;
                     pk[e] = pack_bf16x2(p0, p1);
                     if (PRECISE)
                         pl[e] = pack_bf16x2(p0 - bf16_lo_to_float(pk[e]),
@@ -314,6 +330,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 tmem_st32(tP + half * 32, pk);
                 if (PRECISE) tmem_st32(tPlo + half * 32, pl);
             }
+            const float ls0 = (ls[0] + ls[1]) + (ls[2] + ls[3]);
+            const float ls1 = (ls[4] + ls[5]) + (ls[6] + ls[7]);
             l_run += ls0 + ls1;
             tmem_wait_st();
             tc_fence_before();
@@ -397,7 +415,8 @@ cudaError_t launch_fwd_dp(const CUtensorMap& tq, const CUtensorMap& tk, const CU
     const int n_qtiles = (T + kTile - 1) / kTile;
     dim3 grid(BH, n_qtiles);
     attn_fwd_kernel<D, PRECISE><<<grid, kFwdThreads, C::kSmemBytes, stream>>>(
-        tq, tk, tv, to, o, lse, T, n_qtiles, scale * kLog2e, causal, o_f32);
+        tq, tk, tv, to, o, lse, T, n_qtiles, fabsf(scale) * kLog2e, scale < 0.f ? 1 : 0, causal,
+        o_f32);
     return cudaGetLastError();
 }
 
@@ -422,6 +441,10 @@ cudaError_t launch_attn_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const 
                                 stream);
     return launch_fwd_d<128>(tq, tk, tv, to, o, lse, BH, T, scale, causal, o_f32, precise,
                              stream);
+}
+
+cudaError_t read_and_clear_device_error_fwd(unsigned int* value) {
+    return read_and_clear_unit_error(value);
 }
 
 }  // namespace forge

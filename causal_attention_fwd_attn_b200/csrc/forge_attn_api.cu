@@ -14,19 +14,13 @@
 
 namespace forge {
 
-__device__ unsigned int g_device_error = 0;
-
 cudaError_t read_and_clear_device_error(unsigned int* value, cudaStream_t stream) {
     cudaError_t e = cudaStreamSynchronize(stream);
     if (e != cudaSuccess) return e;
     unsigned int v = 0;
-    e = cudaMemcpyFromSymbol(&v, g_device_error, sizeof(v));
-    if (e != cudaSuccess) return e;
-    if (v != 0) {
-        const unsigned int zero = 0;
-        e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero));
-        if (e != cudaSuccess) return e;
-    }
+    if ((e = read_and_clear_device_error_fwd(&v)) != cudaSuccess) return e;
+    if ((e = read_and_clear_device_error_bwd(&v)) != cudaSuccess) return e;
+    if ((e = read_and_clear_device_error_probe(&v)) != cudaSuccess) return e;
     *value = v;
     return cudaSuccess;
 }
@@ -65,6 +59,23 @@ int make_map_bf16(CUtensorMap* map, const void* base, long long inner, long long
     return r == CUDA_SUCCESS ? FORGE_ATTN_OK : FORGE_ATTN_ERR_CUDA;
 }
 
+// fp32 tensor [planes][rows][inner] in {32, 128, 1} boxes with 128-byte swizzle (the
+// dQ accumulator, written by TMA reduce-add).
+int make_map_f32(CUtensorMap* map, const void* base, long long inner, long long rows,
+                 long long planes) {
+    auto fn = encode_fn();
+    if (!fn) return FORGE_ATTN_ERR_CUDA;
+    cuuint64_t dims[3] = {(cuuint64_t)inner, (cuuint64_t)rows, (cuuint64_t)planes};
+    cuuint64_t strides[2] = {(cuuint64_t)(inner * 4), (cuuint64_t)(inner * rows * 4)};
+    cuuint32_t box[3] = {32, 128, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), dims,
+                    strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? FORGE_ATTN_OK : FORGE_ATTN_ERR_CUDA;
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 int check_shape(int B, int H, int T, int d) {
@@ -88,6 +99,12 @@ int check_common(int B, int H, int T, int d, float scale, int causal) {
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? FORGE_ATTN_OK : FORGE_ATTN_ERR_CUDA; }
 
 size_t round_up_256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Bytes of the padded row statistics (LSE * log2 e and D, 2 x B*H x t_pad fp32).
+size_t rowstats_bytes(int B, int H, int T) {
+    const size_t t_pad = (size_t)((T + 127) / 128) * 128;
+    return round_up_256(2 * (size_t)B * H * t_pad * sizeof(float));
+}
 
 }  // namespace
 }  // namespace forge
@@ -127,6 +144,7 @@ int forge_attn_fwd_ex(const void* q, const void* k, const void* v, void* o, floa
     if ((s = make_map_bf16(&tk, k, d, T, BH)) != FORGE_ATTN_OK) return s;
     if ((s = make_map_bf16(&tv, v, d, T, BH)) != FORGE_ATTN_OK) return s;
     // the output map is only used for bf16 output
+    // the output map is only used for bf16 output
     if ((s = make_map_bf16(&to, o_f32 ? q : o, d, T, BH)) != FORGE_ATTN_OK) return s;
     return cuda_status(launch_attn_fwd(tq, tk, tv, to, o, lse, (int)BH, T, d, scale, causal,
                                        o_f32, (flags & FORGE_ATTN_PRECISE) != 0,
@@ -141,43 +159,43 @@ int forge_attn_fwd(const void* q, const void* k, const void* v, void* o, float* 
 size_t forge_attn_bwd_workspace_size(int B, int H, int T, int d) {
     if (check_shape(B, H, T, d) != FORGE_ATTN_OK) return 0;
     const size_t rows = (size_t)B * H * T;
-    return round_up_256(rows * sizeof(float)) + round_up_256(rows * d * sizeof(float));
+    return rowstats_bytes(B, H, T) + round_up_256(rows * d * sizeof(float));
 }
 
-int forge_attn_bwd_preprocess(const void* o, const void* dO, float* delta, float* dq_accum,
-                              int B, int H, int T, int d, int flags, void* stream) {
-    if (!o || !dO || !delta) return FORGE_ATTN_ERR_INVALID_ARG;
+int forge_attn_bwd_preprocess(const void* o, const void* dO, const float* lse, float* rowstats,
+                              float* dq_accum, int B, int H, int T, int d, int flags,
+                              void* stream) {
+    if (!o || !dO || !lse || !rowstats) return FORGE_ATTN_ERR_INVALID_ARG;
     int s = check_shape(B, H, T, d);
     if (s != FORGE_ATTN_OK) return s;
     if (flags & ~FORGE_ATTN_O_IN_F32) return FORGE_ATTN_ERR_INVALID_ARG;
-    if (!aligned16(o) || !aligned16(dO) || (reinterpret_cast<uintptr_t>(delta) & 3u) ||
-        (dq_accum && !aligned16(dq_accum)))
+    if (!aligned16(o) || !aligned16(dO) || (reinterpret_cast<uintptr_t>(lse) & 3u) ||
+        !aligned16(rowstats) || (dq_accum && !aligned16(dq_accum)))
         return FORGE_ATTN_ERR_MISALIGNED;
-    return cuda_status(launch_bwd_preprocess(o, dO, delta, dq_accum, B * H, T, d,
+    return cuda_status(launch_bwd_preprocess(o, dO, lse, rowstats, dq_accum, B * H, T, d,
                                              (flags & FORGE_ATTN_O_IN_F32) != 0,
                                              static_cast<cudaStream_t>(stream)));
 }
 
 int forge_attn_bwd_dkdv(const void* q, const void* k, const void* v, const void* dO,
-                        const float* lse, const float* delta, float* dq_accum, void* dk,
-                        void* dv, int B, int H, int T, int d, float scale, int causal,
-                        int flags, void* stream) {
-    if (!q || !k || !v || !dO || !lse || !delta || !dq_accum || !dk || !dv)
+                        const float* rowstats, float* dq_accum, void* dk, void* dv, int B, int H,
+                        int T, int d, float scale, int causal, int flags, void* stream) {
+    if (!q || !k || !v || !dO || !rowstats || !dq_accum || !dk || !dv)
         return FORGE_ATTN_ERR_INVALID_ARG;
     int s = check_common(B, H, T, d, scale, causal);
     if (s != FORGE_ATTN_OK) return s;
     if (flags & ~(FORGE_ATTN_OUT_F32 | FORGE_ATTN_PRECISE)) return FORGE_ATTN_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dO) || !aligned16(dk) ||
-        !aligned16(dv) || !aligned16(dq_accum) || (reinterpret_cast<uintptr_t>(lse) & 3u) ||
-        (reinterpret_cast<uintptr_t>(delta) & 3u))
+        !aligned16(dv) || !aligned16(dq_accum) || !aligned16(rowstats))
         return FORGE_ATTN_ERR_MISALIGNED;
     const long long BH = (long long)B * H;
-    CUtensorMap tq, tk, tv, tdo;
+    CUtensorMap tq, tk, tv, tdo, tdq;
     if ((s = make_map_bf16(&tq, q, d, T, BH)) != FORGE_ATTN_OK) return s;
     if ((s = make_map_bf16(&tk, k, d, T, BH)) != FORGE_ATTN_OK) return s;
     if ((s = make_map_bf16(&tv, v, d, T, BH)) != FORGE_ATTN_OK) return s;
     if ((s = make_map_bf16(&tdo, dO, d, T, BH)) != FORGE_ATTN_OK) return s;
-    return cuda_status(launch_bwd_dkdv(tq, tk, tv, tdo, lse, delta, dq_accum, dk, dv, (int)BH, T,
+    if ((s = make_map_f32(&tdq, dq_accum, d, T, BH)) != FORGE_ATTN_OK) return s;
+    return cuda_status(launch_bwd_dkdv(tq, tk, tv, tdo, tdq, rowstats, dq_accum, dk, dv, (int)BH, T,
                                        d, scale, causal, (flags & FORGE_ATTN_OUT_F32) != 0,
                                        (flags & FORGE_ATTN_PRECISE) != 0,
                                        static_cast<cudaStream_t>(stream)));
@@ -211,15 +229,14 @@ int forge_attn_bwd_ex(const void* q, const void* k, const void* v, const void* o
         !aligned16(dq) || !aligned16(dk) || !aligned16(dv) ||
         (reinterpret_cast<uintptr_t>(lse) & 3u))
         return FORGE_ATTN_ERR_MISALIGNED;
-    const size_t rows = (size_t)B * H * T;
-    float* delta = static_cast<float*>(workspace);
+    float* rowstats = static_cast<float*>(workspace);
     float* acc = grad_f32 ? static_cast<float*>(dq)
-                     : reinterpret_cast<float*>(static_cast<char*>(workspace) +
-                                                round_up_256(rows * sizeof(float)));
-    if ((s = forge_attn_bwd_preprocess(o, dO, delta, acc, B, H, T, d,
+                          : reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                                     rowstats_bytes(B, H, T));
+    if ((s = forge_attn_bwd_preprocess(o, dO, lse, rowstats, acc, B, H, T, d,
                                        flags & FORGE_ATTN_O_IN_F32, stream)) != FORGE_ATTN_OK)
         return s;
-    if ((s = forge_attn_bwd_dkdv(q, k, v, dO, lse, delta, acc, dk, dv, B, H, T, d, scale, causal,
+    if ((s = forge_attn_bwd_dkdv(q, k, v, dO, rowstats, acc, dk, dv, B, H, T, d, scale, causal,
                                  flags & (FORGE_ATTN_OUT_F32 | FORGE_ATTN_PRECISE), stream)) !=
         FORGE_ATTN_OK)
         return s;

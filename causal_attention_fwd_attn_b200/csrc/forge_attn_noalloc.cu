@@ -1,7 +1,7 @@
 // forge_attn_noalloc.cu -- the backward for callers that cannot allocate device
 // memory.
 //
-// forge_attn_bwd needs a workspace (the D vector and the fp32 dQ accumulator) that
+// forge_attn_bwd needs a workspace (the row statistics and the fp32 dQ accumulator) that
 // the caller allocates.  Some callers cannot: code that runs after a fixed memory
 // budget has been handed out at start-up (a serving process or an embedded runtime
 // that forbids allocation once running), code whose allocator is not reachable
@@ -13,7 +13,8 @@
 // The array is allocated when the library's device code is loaded onto a GPU and
 // is held on every GPU that loads the library until the process exits.  All calls
 // on a device share it and it keeps the last call's contents; the D pre-pass
-// rewrites D and clears the dQ accumulator at the start of every call, so nothing
+// rewrites the row statistics and clears the dQ accumulator at the start of every
+// call, so nothing
 // leaks from one call into the next.  Two calls whose kernels overlap on the GPU
 // (different streams, no ordering between them) race on the array.
 #include <cmath>
@@ -77,13 +78,15 @@ extern "C" int forge_attn_bwd_noalloc(const void* q, const void* k, const void* 
     if (need > (size_t)FORGE_ATTN_NOALLOC_SCRATCH_BYTES) return FORGE_ATTN_ERR_WORKSPACE;
     void* scratch = nullptr;
     if (scratch_address(&scratch) != cudaSuccess) return FORGE_ATTN_ERR_CUDA;
-    const size_t rows = (size_t)B * H * T;
-    float* delta = static_cast<float*>(scratch);
+    // same layout as the workspace of forge_attn_bwd: padded row statistics, then the
+    // fp32 dQ accumulator
+    const size_t t_pad = (size_t)((T + 127) / 128) * 128;
+    float* rowstats = static_cast<float*>(scratch);
     float* acc = reinterpret_cast<float*>(static_cast<char*>(scratch) +
-                                          round_up_256(rows * sizeof(float)));
-    int s = forge_attn_bwd_preprocess(o, dO, delta, acc, B, H, T, d, 0, stream);
+                                          round_up_256(2 * (size_t)B * H * t_pad * sizeof(float)));
+    int s = forge_attn_bwd_preprocess(o, dO, lse, rowstats, acc, B, H, T, d, 0, stream);
     if (s != FORGE_ATTN_OK) return s;
-    s = forge_attn_bwd_dkdv(q, k, v, dO, lse, delta, acc, dk, dv, B, H, T, d, scale, causal, 0,
+    s = forge_attn_bwd_dkdv(q, k, v, dO, rowstats, acc, dk, dv, B, H, T, d, scale, causal, 0,
                             stream);
     if (s != FORGE_ATTN_OK) return s;
     return forge_attn_bwd_dq_convert(acc, dq, B, H, T, d, stream);

@@ -18,11 +18,14 @@ cudaError_t launch_attn_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const 
                             const CUtensorMap& to, void* o, float* lse, int BH, int T, int d,
                             float scale, int causal, int o_f32, int precise, cudaStream_t stream);
 
-cudaError_t launch_bwd_preprocess(const void* o, const void* dO, float* delta, float* dq_accum,
-                                  int BH, int T, int d, int o_f32, cudaStream_t stream);
+// Row statistics of the backward: fp32 [2][B*H][t_pad], t_pad = 128 * ceil(T / 128).
+cudaError_t launch_bwd_preprocess(const void* o, const void* dO, const float* lse,
+                                  float* rowstats, float* dq_accum, int BH, int T, int d,
+                                  int o_f32, cudaStream_t stream);
 
+// tdq: the fp32 dQ accumulator [B*H][T][d] in {32, 128, 1} boxes, 128-byte swizzle.
 cudaError_t launch_bwd_dkdv(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                            const CUtensorMap& tdo, const float* lse, const float* delta,
+                            const CUtensorMap& tdo, const CUtensorMap& tdq, const float* rowstats,
                             float* dq_accum, void* dk, void* dv, int BH, int T, int d,
                             float scale, int causal, int grad_f32, int precise,
                             cudaStream_t stream);
@@ -35,7 +38,10 @@ cudaError_t launch_probe_mma(const CUtensorMap& ta, const CUtensorMap& tb, const
 
 cudaError_t launch_probe_wait_timeout(unsigned long long limit_ns, cudaStream_t stream);
 
-// Device error word accessors (defined next to the word itself).
-cudaError_t read_and_clear_device_error(unsigned int* value, cudaStream_t stream);
+// Device error words, one per translation unit with kernels: each reader ORs its
+// word into *value and clears it (the stream must have been synchronised).
+cudaError_t read_and_clear_device_error_fwd(unsigned int* value);
+cudaError_t read_and_clear_device_error_bwd(unsigned int* value);
+cudaError_t read_and_clear_device_error_probe(unsigned int* value);
 
 }  // namespace forge

@@ -8,6 +8,7 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_runtime.h>
 #include <stdint.h>
 
 namespace forge {
@@ -15,9 +16,26 @@ namespace forge {
 // ----------------------------------------------------------------------------
 // Device-side error word.  Every spin-wait in the library is bounded; a wait
 // that runs out records (site, block) here and the kernel winds down instead of
-// hanging.  forge_attn_check_device_error() reads and clears it.
+// hanging.  Each translation unit that launches kernels has its own word (the
+// library is built without relocatable device code, which keeps ptxas's
+// per-warpgroup register budgets); forge_attn_check_device_error() reads and
+// clears all of them through each unit's read_and_clear_device_error_<unit>().
 // ----------------------------------------------------------------------------
-extern __device__ unsigned int g_device_error;
+static __device__ unsigned int g_device_error = 0;
+
+// Host side: read this unit's word and clear it (after the caller synchronised).
+static inline cudaError_t read_and_clear_unit_error(unsigned int* value) {
+    unsigned int v = 0;
+    cudaError_t e = cudaMemcpyFromSymbol(&v, g_device_error, sizeof(v));
+    if (e != cudaSuccess) return e;
+    if (v != 0) {
+        const unsigned int zero = 0;
+        e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero));
+        if (e != cudaSuccess) return e;
+    }
+    *value |= v;
+    return cudaSuccess;
+}
 
 // Wait limit for one mbarrier wait, in nanoseconds of %globaltimer.  Every wait in
 // these kernels is for a TMA copy or a tensor-core MMA of the same CTA, which
@@ -120,6 +138,28 @@ __device__ __forceinline__ void tma_load_3d(void* smem_dst, const void* map, uin
         "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes "
         "[%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(smem_dst)),
         "l"(map), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
+        : "memory");
+}
+
+// 1-D bulk copy global -> shared (16-byte aligned, size a multiple of 16), completion
+// counted on `bar` in bytes.
+__device__ __forceinline__ void bulk_load(void* smem_dst, const void* src, uint32_t bytes,
+                                          uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_u32(smem_dst)),
+        "l"(src), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// 3-D tiled reduce-add shared -> global (element type from the tensor map; rows
+// outside the tensor are clipped).
+__device__ __forceinline__ void tma_reduce_add_3d(const void* map, const void* smem_src, int c0,
+                                                  int c1, int c2) {
+    asm volatile(
+        "cp.reduce.async.bulk.tensor.3d.global.shared::cta.add.bulk_group [%0, {%2, %3, %4}], "
+        "[%1];" ::"l"(map),
+        "r"(smem_u32(smem_src)), "r"(c0), "r"(c1), "r"(c2)
         : "memory");
 }
 
@@ -249,6 +289,18 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
         "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
         "r"(r[15])
         : "memory");
+}
+
+// Warpgroup register reallocation: every warp of a warpgroup executes the same
+// instruction.  The block's total is fixed at launch (threads x registers);
+// decreases must free what increases take.
+template <uint32_t N>
+__device__ __forceinline__ void regs_dec() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void regs_inc() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
 }
 
 // ------------------------------------------------------------- descriptors --

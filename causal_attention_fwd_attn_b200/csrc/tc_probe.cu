@@ -168,4 +168,8 @@ cudaError_t launch_probe_wait_timeout(unsigned long long limit_ns, cudaStream_t 
     return cudaGetLastError();
 }
 
+cudaError_t read_and_clear_device_error_probe(unsigned int* value) {
+    return read_and_clear_unit_error(value);
+}
+
 }  // namespace forge

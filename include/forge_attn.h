@@ -20,7 +20,7 @@
  *               library never allocates or frees device memory.
  *   Layout      q, k, v, o, dO, dq, dk, dv are contiguous row-major [B][H][T][d]
  *               (d fastest).  lse and the backward's D are fp32 [B][H][T].
- *               Elements are bf16 bit patterns unless a dtype argument says fp32.
+ *               Elements are bf16 bit patterns unless an option bit says fp32.
  *   Alignment   Every tensor base must be 16-byte aligned (a TMA requirement);
  *               the workspace must be 256-byte aligned.
  *   Aliasing    Outputs must not overlap inputs or each other.
@@ -38,8 +38,8 @@
  *               bounded: a wait that runs out is reported by
  *               forge_attn_check_device_error().
  *   Determinism The forward is deterministic.  The backward accumulates dQ with
- *               fp32 atomic adds, so dQ may differ in the last bits run to run;
- *               dK and dV are deterministic.
+ *               unordered fp32 reductions, so dQ may differ in the last bits run to
+ *               run; dK and dV are deterministic.
  */
 #ifndef FORGE_ATTN_H
 #define FORGE_ATTN_H
@@ -95,9 +95,10 @@ int forge_attn_fwd_ex(const void* q, const void* k, const void* v, void* o, floa
                       int H, int T, int d, float scale, int causal, int flags, void* stream);
 
 /*
- * Bytes of device workspace forge_attn_bwd needs: the D vector (fp32 [B][H][T])
- * and the fp32 dQ accumulator ([B][H][T][d]), each at a 256-byte aligned offset.
- * Returns 0 for arguments forge_attn_bwd would reject.
+ * Bytes of device workspace forge_attn_bwd needs: the row statistics (fp32
+ * [2][B*H][t_pad], t_pad = 128 * ceil(T / 128): LSE * log2(e), then D) and the fp32
+ * dQ accumulator ([B][H][T][d]), each at a 256-byte aligned offset.  Returns 0 for
+ * arguments forge_attn_bwd would reject.
  */
 size_t forge_attn_bwd_workspace_size(int B, int H, int T, int d);
 
@@ -108,9 +109,9 @@ size_t forge_attn_bwd_workspace_size(int B, int H, int T, int d);
  * forge_attn_bwd_workspace_size() bytes, 256-byte aligned; its contents on entry
  * do not matter and on return are unspecified.
  * `o` is bf16 here (fp32 with forge_attn_bwd_ex and FORGE_ATTN_O_IN_F32).
- * Launch sequence on `stream`: D pre-pass (also zeroes the dQ accumulator),
- * the dK/dV kernel over key tiles (dQ partials added with fp32 atomics), and
- * the dQ conversion.
+ * Launch sequence on `stream`: the pre-pass (row statistics; also zeroes the dQ
+ * accumulator), the dK/dV kernel over key tiles (dQ partials added into the fp32
+ * accumulator by TMA reduce-add or fp32 vector reductions), and the dQ conversion.
  */
 int forge_attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO,
                    const float* lse, void* dq, void* dk, void* dv, void* workspace,
@@ -129,27 +130,30 @@ int forge_attn_bwd_ex(const void* q, const void* k, const void* v, const void* o
  * The three backward stages as separate calls, for callers that schedule or time
  * them one by one.  forge_attn_bwd_ex is exactly these three in order.
  *
- * forge_attn_bwd_preprocess: delta[i] = sum_k dO[i][k] * o[i][k] (fp32 [B][H][T]),
- *   and dq_accum (fp32 [B][H][T][d]) set to zero unless it is NULL.  flags:
- *   FORGE_ATTN_O_IN_F32 (o is fp32).
- * forge_attn_bwd_dkdv: recomputes P per key tile, writes dk and dv, and adds
- *   scale * dS K into dq_accum with fp32 atomics.  flags: FORGE_ATTN_OUT_F32
- *   (dk, dv fp32), FORGE_ATTN_PRECISE.
+ * forge_attn_bwd_preprocess: the row statistics rowstats (fp32 [2][B*H][t_pad],
+ *   t_pad = 128 * ceil(T / 128), 16-byte aligned): rowstats[0][bh][t] = lse * log2(e)
+ *   and rowstats[1][bh][t] = D = sum_k dO[t][k] * o[t][k], with +inf and 0 in the
+ *   padding rows t >= T; and dq_accum (fp32 [B][H][T][d]) set to zero unless it is
+ *   NULL.  flags: FORGE_ATTN_O_IN_F32 (o is fp32).
+ * forge_attn_bwd_dkdv: recomputes P per key tile from the row statistics, writes dk
+ *   and dv, and adds scale * dS K into dq_accum (TMA reduce-add or fp32 vector
+ *   reductions).  flags: FORGE_ATTN_OUT_F32 (dk, dv fp32), FORGE_ATTN_PRECISE.
  * forge_attn_bwd_dq_convert: dq = bf16(dq_accum).  Only needed for bf16 dq.
  */
-int forge_attn_bwd_preprocess(const void* o, const void* dO, float* delta, float* dq_accum,
-                              int B, int H, int T, int d, int flags, void* stream);
+int forge_attn_bwd_preprocess(const void* o, const void* dO, const float* lse, float* rowstats,
+                              float* dq_accum, int B, int H, int T, int d, int flags,
+                              void* stream);
 int forge_attn_bwd_dkdv(const void* q, const void* k, const void* v, const void* dO,
-                        const float* lse, const float* delta, float* dq_accum, void* dk,
-                        void* dv, int B, int H, int T, int d, float scale, int causal,
-                        int flags, void* stream);
+                        const float* rowstats, float* dq_accum, void* dk, void* dv, int B, int H,
+                        int T, int d, float scale, int causal, int flags, void* stream);
 int forge_attn_bwd_dq_convert(const float* dq_accum, void* dq, int B, int H, int T, int d,
                               void* stream);
 
 /*
  * Bytes of the fixed device array that forge_attn_bwd_noalloc uses in place of a
- * workspace: 64 MiB, enough for B*H*T*(d+1) up to about 16.7 million (for example
- * B=4 H=16 T=2048 d=64, or B=1 H=16 T=4096 d=64).
+ * workspace: 64 MiB, enough whenever forge_attn_bwd_workspace_size() <= 64 MiB,
+ * i.e. B*H*(T*d + 2*t_pad) floats up to about 16.7 million (for example B=4 H=16
+ * T=2048 d=64, or B=1 H=16 T=4096 d=64).
  */
 #define FORGE_ATTN_NOALLOC_SCRATCH_BYTES (64u << 20)
 
@@ -159,7 +163,8 @@ int forge_attn_bwd_dq_convert(const float* dq_accum, void* dq, int B, int H, int
  * but no allocator, a latency-critical loop that must not call the allocator).
  * The paper has no counterpart; this is a property of this library, not of the
  * method.  Same arguments, results and launch sequence as forge_attn_bwd, minus the
- * workspace: D and the fp32 dQ accumulator live in a file-scope __device__ array of
+ * workspace: the row statistics and the fp32 dQ accumulator live in a file-scope
+ * __device__ array of
  * FORGE_ATTN_NOALLOC_SCRATCH_BYTES that every GPU which loads the library holds
  * until the process exits.  No cudaMalloc, cudaFree or allocating library call is
  * made.
@@ -169,7 +174,7 @@ int forge_attn_bwd_dq_convert(const float* dq_accum, void* dq, int B, int H, int
  *     device, with that device current); make that first call before any stream
  *     capture begins.
  *   - All calls on a device share the array, which keeps the last call's contents;
- *     each call rewrites D and clears the accumulator first.  Calls whose kernels
+ *     each call rewrites the row statistics and clears the accumulator first.  Calls whose kernels
  *     can overlap on the GPU (unordered streams) race on the array and must not be
  *     issued.
  */

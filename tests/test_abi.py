@@ -44,15 +44,20 @@ def test_version_and_status_strings(lib):
     assert "unknown" in _lib.status_string(99)
 
 
+def _up256(x):
+    return (x + 255) // 256 * 256
+
+
 def test_workspace_size(lib):
+    # padded row statistics (2 x B*H x 128*ceil(T/128) fp32), then the fp32 dQ accumulator
     n = _lib.forge_attn_bwd_workspace_size(1, 2, 128, 64)
-    rows = 2 * 128
-    assert n == ((rows * 4 + 255) // 256) * 256 + ((rows * 64 * 4 + 255) // 256) * 256
+    assert n == _up256(2 * 2 * 128 * 4) + _up256(2 * 128 * 64 * 4)
     assert _lib.forge_attn_bwd_workspace_size(1, 1, 1, 96) == 0
     assert _lib.forge_attn_bwd_workspace_size(0, 1, 1, 64) == 0
-    # ragged T: both parts stay 256-byte aligned
+    # ragged T: the statistics are padded to whole tiles, both parts 256-byte aligned
     n = _lib.forge_attn_bwd_workspace_size(1, 1, 7, 64)
-    assert n == 256 + ((7 * 64 * 4 + 255) // 256) * 256
+    assert n == _up256(2 * 128 * 4) + _up256(7 * 64 * 4)
+    assert _lib.rowstats_bytes(3, 5, 200) == _up256(2 * 15 * 256 * 4)
 
 
 P = 4096  # a 16-byte aligned fake address; never dereferenced (rejected first)
@@ -105,13 +110,15 @@ def test_bwd_rejects_bad_arguments(lib):
 
 
 def test_stage_entry_points_reject_bad_arguments(lib):
-    assert _lib.forge_attn_bwd_preprocess(0, P, P, P, 1, 1, 8, 64, 0, None) == \
+    assert _lib.forge_attn_bwd_preprocess(0, P, P, P, P, 1, 1, 8, 64, 0, None) == \
         _lib.ERR_INVALID_ARG
-    assert _lib.forge_attn_bwd_preprocess(P, P, P, P + 4, 1, 1, 8, 64, 0, None) == \
+    assert _lib.forge_attn_bwd_preprocess(P, P, P, P, P + 4, 1, 1, 8, 64, 0, None) == \
         _lib.ERR_MISALIGNED
-    assert _lib.forge_attn_bwd_preprocess(P, P, P, P, 1, 1, 8, 64, _lib.PRECISE, None) == \
+    assert _lib.forge_attn_bwd_preprocess(P, P, P, P + 8, P, 1, 1, 8, 64, 0, None) == \
+        _lib.ERR_MISALIGNED  # row statistics must be 16-byte aligned
+    assert _lib.forge_attn_bwd_preprocess(P, P, P, P, P, 1, 1, 8, 64, _lib.PRECISE, None) == \
         _lib.ERR_INVALID_ARG
-    assert _lib.forge_attn_bwd_dkdv(P, P, P, P, P, P, 0, P, P, 1, 1, 8, 64, 0.1, 1, 0, None) == \
+    assert _lib.forge_attn_bwd_dkdv(P, P, P, P, P, 0, P, P, 1, 1, 8, 64, 0.1, 1, 0, None) == \
         _lib.ERR_INVALID_ARG
     assert _lib.forge_attn_bwd_dq_convert(P, P, 1, 1, 8, 48, None) == _lib.ERR_UNSUPPORTED
     assert _lib.forge_probe_mma(P, P, P, 96, 64, 0, None) == _lib.ERR_INVALID_ARG
