@@ -24,9 +24,8 @@ import json
 import math
 import os
 import statistics
-import subprocess
 import sys
-import tempfile
+import threading
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -84,61 +83,90 @@ def find_workload(name):
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle-reason samples during the timed region."""
+    """SM clock, power and clock-event reasons sampled every few milliseconds by an NVML
+    thread while the timed region runs.
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    mark_begin()/mark_end() bracket the timed region on the host; only samples taken
+    between them are reported."""
 
-    def __init__(self, gpu_index):
-        self.gpu = gpu_index
-        self.proc = None
-        self.path = None
+    REASON_BITS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40,
+                   "sw_thermal_slowdown": 0x20, "sw_power_cap": 0x4,
+                   "hw_power_brake_slowdown": 0x80}
+
+    def __init__(self, device_index, period_s=0.004):
+        self.dev = device_index
+        self.period = period_s
+        self.samples = []  # (host time, sm MHz, power W, reasons bitmask)
+        self.handle = None
+        self.nvml = None
+        self.sm_max = None
+        self.thread = None
+        self.stop_flag = False
+        self.window = [None, None]
+        self.error = None
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            self.handle = self._handle(pynvml, device_index)
+            self.sm_max = pynvml.nvmlDeviceGetMaxClockInfo(self.handle, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # noqa: BLE001 - any NVML failure means "no samples"
+            self.error = f"nvml unavailable: {type(e).__name__}"
+            self.nvml = None
+
+    @staticmethod
+    def _handle(pynvml, device_index):
+        p = torch.cuda.get_device_properties(device_index)
+        bus = f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0"
+        return pynvml.nvmlDeviceGetHandleByPciBusId(bus.encode())
+
+    def _read(self):
+        n = self.nvml
+        sm = n.nvmlDeviceGetClockInfo(self.handle, n.NVML_CLOCK_SM)
+        pw = n.nvmlDeviceGetPowerUsage(self.handle) / 1000.0
+        rs = n.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
+        return sm, pw, rs
+
+    def _loop(self):
+        while not self.stop_flag:
+            try:
+                sm, pw, rs = self._read()
+                self.samples.append((time.perf_counter(), sm, pw, rs))
+            except Exception as e:  # noqa: BLE001
+                self.error = f"nvml read failed: {type(e).__name__}"
+                return
+            time.sleep(self.period)
 
     def start(self):
-        fd, self.path = tempfile.mkstemp(suffix=".csv")
-        os.close(fd)
-        try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
-                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
-        except (FileNotFoundError, OSError):
-            self.proc = None
+        if self.nvml is None:
+            return
+        self.thread = threading.Thread(target=self._loop, daemon=True)
+        self.thread.start()
+
+    def mark_begin(self):
+        self.window[0] = time.perf_counter()
+
+    def mark_end(self):
+        self.window[1] = time.perf_counter()
 
     def stop(self):
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        rows = []
-        with open(self.path) as f:
-            for line in f:
-                parts = [p.strip() for p in line.split(",")]
-                if len(parts) >= 9:
-                    rows.append(parts)
-        os.unlink(self.path)
+        if self.thread is not None:
+            self.stop_flag = True
+            self.thread.join(timeout=5)
+        lo, hi = self.window
+        rows = [s for s in self.samples
+                if (lo is None or s[0] >= lo) and (hi is None or s[0] <= hi)]
         if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
-        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
-        smax = max(float(r[2]) for r in rows if r[2].replace(".", "").isdigit())
-        loaded = [r for r in rows if _num(r[3]) and float(r[3]) > 200] or rows
-        sm_loaded = [float(r[1]) for r in loaded if r[1].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
-        return {"sm_mhz": statistics.median(sm_loaded or sm), "sm_max_mhz": smax,
-                "reasons": reasons, "samples": len(rows)}
-
-
-def _num(x):
-    try:
-        float(x)
-        return True
-    except ValueError:
-        return False
+            return {"sm_mhz": None, "sm_max_mhz": self.sm_max,
+                    "reasons": [self.error or "no samples in the timed region"], "samples": 0}
+        reasons = sorted({name for s in rows for name, bit in self.REASON_BITS.items()
+                          if s[3] & bit})
+        return {"sm_mhz": statistics.median(s[1] for s in rows), "sm_max_mhz": self.sm_max,
+                "sm_min_mhz": min(s[1] for s in rows),
+                "power_w_median": round(statistics.median(s[2] for s in rows), 1),
+                "reasons": reasons, "samples": len(rows), "source": "nvml",
+                "period_ms": round(1000 * self.period, 1)}
 
 
 # ------------------------------------------------------------------- ours ----
@@ -199,18 +227,18 @@ def run_ours(args, rank, world, local_rank):
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    vis = [v for v in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if v]
-    clocks = ClockSampler(vis[local_rank] if local_rank < len(vis) else str(local_rank))
+    clocks = ClockSampler(local_rank)
+    clocks.start()
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
-    clocks.start()
-    time.sleep(0.3)  # let the sampler start before the timed region
+    clocks.mark_begin()
     t0.record(stream)
     for i in range(args.steps):
         step(sets[(args.warmup + i) % n_sets], evs[i])
     t1.record(stream)
     torch.cuda.synchronize()
+    clocks.mark_end()
     if world > 1:
         torch.distributed.barrier()
     clk = clocks.stop()
@@ -424,8 +452,8 @@ def main():
     ap = argparse.ArgumentParser(description=__doc__,
                                  formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-baseline-seconds", type=float, default=12.0,

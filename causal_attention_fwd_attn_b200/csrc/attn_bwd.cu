@@ -8,9 +8,9 @@
 // score matrices S^T = K Q^T and dP^T = V dO^T by exchanging operand roles
 // rather than moving data (same section).  Here:
 //
-//   attn_bwd_preprocess  D[i] = sum_k dO[i][k] O[i][k] (fp32), LSE[i] * log2(e), both
+//   attn_bwd_preprocess  D[i] = sum_k dO[i][k] O[i][k] (fp32), -LSE[i] * log2(e), both
 //                        padded per head to a whole number of 128-row tiles (D = 0,
-//                        LSE = +inf past T, so those queries get P = 0), and the fp32
+//                        -LSE = -inf past T, so those queries get P ~ 0), and the fp32
 //                        dQ accumulator cleared.  Memory-bound.
 //   attn_bwd_dkdv        one CTA per (head, 128-key tile j), looping over the query
 //                        tiles i that see it (i >= j under the causal mask):
@@ -29,34 +29,48 @@
 //                        replace the paper's second pass over the scores.
 //   attn_bwd_dq_convert  dQ = bf16(accumulator).
 //
-// dkdv warp roles (320 threads):
-//   warp 0      producer (one thread): K_j, V_j once; Q_i, dO_i by TMA into staged
-//               rings; the LSE_i and D_i vectors (128 floats each) by 1-D bulk copies
-//               from the padded row statistics, counted on Q_i's barrier.
-//   warp 1      MMA issuer (one thread).
-//   warps 2..9  compute: warp w owns TMEM lanes 32*(w%4).. (key rows of the tile)
-//               and half h = (w-2)/4 of the 128 query columns.  Each thread writes
-//               its 64 P^T and dS^T values bf16 into 128-byte-swizzled shared
-//               memory (the A operand of dV/dK, and the MN-major A operand of dQ),
-//               drains its half of dQ_i's columns for query row 32*(w%4)+lane,
-//               and stores its half of the dK/dV columns at the end.
+// dkdv warp roles (512 threads, four warpgroups; setmaxnreg moves registers from the
+// drain and control warpgroups to the two compute warpgroups):
+//   warps 0..3   dQ drain: warp w owns TMEM lanes 32w.. (query rows of dQ_i) and all d
+//                columns; it moves dQ_i out of tensor memory, scales it and adds it to
+//                the fp32 accumulator (TMA reduce-add from shared memory, or
+//                red.global.add.v4.f32), off the compute warps' path.
+//   warps 4..11  compute: warp w owns TMEM lanes 32*(w%4).. (key rows of the tile) and
+//                half h = (w-4)/4 of the 128 query columns.  Each thread forms its 64
+//                P^T values and writes them bf16 either into tensor memory (d = 64:
+//                the A operand of dV) or into 128-byte-swizzled shared memory, then
+//                its 64 dS^T values into shared memory (the A operand of dK, and the
+//                MN-major A operand of dQ), and stores its half of the dK/dV columns
+//                at the end.
+//   warp 12      producer (one thread): K_j, V_j once; Q_i, dO_i by TMA into staged
+//                rings; the LSE_i and D_i vectors (128 floats each) by 1-D bulk copies
+//                from the padded row statistics, counted on Q_i's barrier.
+//   warp 13      MMA issuer (one thread); allocates tensor memory.
+//   warps 14,15  idle (they complete the control warpgroup for setmaxnreg).
 // Tensor memory: dV [0,d) | dK [d,2d) | S^T [2d,2d+128) | dP^T [2d+128,2d+256) |
-//   dQ_i [2d+256, 3d+256) for d = 64; for d = 128 dQ_i reuses the dP^T columns once
-//   dS^T has been formed (512 columns hold no more).
+//   dQ_i [2d+256, 3d+256) and P^T as bf16 pairs [3d+256, 3d+320) for d = 64; for
+//   d = 128 dQ_i reuses the dP^T columns once dS^T has been formed (512 columns hold
+//   no more) and P^T stays in shared memory.
 #include "forge_internal.h"
 #include "sm100_ptx.cuh"
 
 namespace forge {
 namespace {
 
-constexpr int kBwdThreads = 320;
+// Which pairs of P^T's exponentials go to the FMA-pipe polynomial (exp2_poly2)
+// instead of the MUFU unit: 1 of every 4.  Precise mode keeps all on the MUFU unit.
+__device__ __forceinline__ constexpr bool use_poly_pair(int e) { return (e & 3) == 3; }
+
+constexpr int kBwdThreads = 512;
 constexpr int kComputeWarps = 8;
+constexpr int kDrainWarps = 4;
+constexpr uint32_t kWarpCompute0 = 4, kWarpProducer = 12, kWarpMma = 13;
 constexpr float kLog2e = 1.4426950408889634f;
 
 enum : uint32_t {
     kSiteKV = 1, kSiteQFull, kSiteDOFull, kSiteQEmpty, kSiteDOEmpty, kSiteSFull,
     kSiteSFree, kSiteDPFull, kSitePFull, kSitePFree, kSiteDSFull, kSiteDSFree, kSiteDQFull,
-    kSiteDQFree, kSiteAccDone, kSiteAlign
+    kSiteDQFree, kSiteAccDone, kSiteAlign, kSiteStageFree, kSiteStageFull
 };
 
 template <int D, bool PRECISE>
@@ -66,6 +80,9 @@ struct BwdCfg {
     static constexpr int kTileBytes = kChunks * kChunkBytes;
     // dQ through shared memory and a TMA reduce where there is room (d = 64 default)
     static constexpr bool kTmaDQ = (D == 64 && !PRECISE);
+    // P^T goes back into tensor memory (bf16 pairs) as the A operand of dV where
+    // columns are left for it (d = 64 default); otherwise into shared memory.
+    static constexpr bool kPInTmem = (D == 64 && !PRECISE);
     static constexpr int kStagesQ = kTmaDQ ? 3 : 2;
     // Precise mode at d = 128 needs the room of one dO stage for the lo buffer.
     static constexpr int kStagesDO = (D == 128 && PRECISE) ? 1 : 2;
@@ -85,17 +102,28 @@ struct BwdCfg {
     static constexpr int kOffQ = kOffV + kTileBytes;
     static constexpr int kOffDO = kOffQ + kStagesQ * kTileBytes;
     static constexpr int kOffP = kOffDO + kStagesDO * kTileBytes;
-    static constexpr int kOffDS = kSeparatePdS ? kOffP + kSplit * kScoreBytes : kOffP;
+    static constexpr int kPBytes = kPInTmem ? 0 : kSplit * kScoreBytes;
+    static constexpr int kOffDS = kSeparatePdS ? kOffP + kPBytes : kOffP;
     static constexpr int kOffDQS = kOffDS + kSplit * kScoreBytes;
-    static constexpr int kOffLse = kOffDQS + (kTmaDQ ? 2 * kDQStageBytes : 0);
+    static constexpr int kDQSlices = kTmaDQ ? D / 32 : 0;  // 32-column staging slices
+    static constexpr int kOffLse = kOffDQS + kDQSlices * kDQStageBytes;
     static constexpr int kOffDelta = kOffLse + kStagesQ * kTile * 4;
     static constexpr int kOffBar = kOffDelta + kStagesQ * kTile * 4;
     static constexpr int kSmemBytes = kOffBar + 256;
     static_assert(kSmemBytes <= 232448, "shared memory budget");
     static constexpr uint32_t kColDV = 0, kColDK = D, kColS = 2 * D, kColDP = 2 * D + 128;
     static constexpr uint32_t kColDQ = kSeparateDQ ? 2 * D + 256 : kColDP;
+    static constexpr uint32_t kColP = 3 * D + 256;
     static constexpr uint32_t kTmemCols = 512;
     static_assert(kColDQ + D <= kTmemCols, "tensor memory budget");
+    static_assert(!kPInTmem || (kSeparateDQ && kColP + 64 <= kTmemCols), "tensor memory budget");
+    // registers per thread after setmaxnreg (the launch gives 512 x 128): the precise
+    // d = 128 MMA issuer needs more, its drain (64 columns at a time) less
+    static constexpr uint32_t kRegsDrain = (D == 128 && PRECISE) ? 80 : 96;
+    static constexpr uint32_t kRegsCompute = 168;
+    static constexpr uint32_t kRegsCtl = (D == 128 && PRECISE) ? 96 : 80;
+    static_assert(128 * kRegsDrain + 256 * kRegsCompute + 128 * kRegsCtl <= 65536,
+                  "register split exceeds the block's launch allocation");
     static constexpr uint32_t kIdescScore = idesc_bf16_f32(128, 128, false, false);
     static constexpr uint32_t kIdescGrad = idesc_bf16_f32(128, D, false, true);  // dV, dK
     static constexpr uint32_t kIdescDQ = idesc_bf16_f32(128, D, true, true);     // dQ
@@ -108,10 +136,12 @@ struct BwdBarriers {
     uint64_t q_empty[3];
     uint64_t do_empty[2];
     uint64_t s_full, s_free, dp_full, p_full, p_free, ds_full, ds_free, dq_full, dq_free;
+    uint64_t stage_free, stage_full;  // dQ staging in shared memory (drain warps)
     uint64_t acc_done, mma_final;
     uint32_t tmem_base;
     int abort;
 };
+static_assert(sizeof(BwdBarriers) <= 256, "barrier block");
 
 // Eight fp32 values as bf16 into a 16-byte chunk at base + off; in precise mode the
 // remainders x - bf16(x), rounded to bf16, go to the same place in the lo buffer
@@ -189,14 +219,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         mbar_init(&bars->ds_full, kComputeWarps);
         mbar_init(&bars->ds_free, 1);
         mbar_init(&bars->dq_full, 1);
-        mbar_init(&bars->dq_free, kComputeWarps);
+        mbar_init(&bars->dq_free, kDrainWarps);
+        mbar_init(&bars->stage_free, 1);
+        mbar_init(&bars->stage_full, kDrainWarps);
         mbar_init(&bars->acc_done, 1);
         mbar_init(&bars->mma_final, 1);
         bars->abort = (smem_u32(smem) & 1023u) ? 1 : 0;
         if (bars->abort) record_timeout(kSiteAlign);
         fence_mbar_init();
     }
-    if (warp == 1) {
+    if (warp == kWarpMma) {
         tmem_alloc(&bars->tmem_base, C::kTmemCols);
         tmem_relinquish();
     }
@@ -205,9 +237,261 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     tc_fence_after();
     const uint32_t tmem = bars->tmem_base;
 
-    if (warp == 0) {
-        // ------------------------------------------------------------ producer
-        if (lane == 0) {
+    if (warp < kWarpCompute0) {
+        // ---------------------------------------------------------- dQ drain
+        regs_dec<C::kRegsDrain>();
+        const uint32_t row = (warp << 5) + lane;  // query row of the tile
+        const uint32_t lane_off = (warp << 5) << 16;
+        const bool leader = warp == 0 && lane == 0;
+        for (int m = 0; m < n_iter; ++m) {
+            if (!warp_wait(&bars->dq_full, m & 1, kSiteDQFull, abort)) break;
+            tc_fence_after();
+            const int i = i_begin + m;
+            if constexpr (C::kTmaDQ) {
+                uint32_t r[D];
+#pragma unroll
+                for (int c = 0; c < D / 32; ++c)
+                    tmem_ld32(tmem + lane_off + C::kColDQ + c * 32, r + c * 32);
+                tmem_wait_ld();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars->dq_free);
+                // the staging slices must have been read by the previous reduce (bounded
+                // mbarrier waits rather than bar.sync, so an abort cannot strand a warp)
+                if (leader) {
+                    tma_store_wait_all_read();
+                    mbar_arrive(&bars->stage_free);
+                }
+                if (!warp_wait(&bars->stage_free, m & 1, kSiteStageFree, abort)) break;
+#pragma unroll
+                for (int sl = 0; sl < C::kDQSlices; ++sl) {
+                    uint8_t* stage = smem + C::kOffDQS + sl * C::kDQStageBytes;
+#pragma unroll
+                    for (int ch = 0; ch < 8; ++ch) {
+                        const uint32_t* x = r + sl * 32 + 4 * ch;
+                        *reinterpret_cast<float4*>(stage + sw128_offset(row, ch)) =
+                            make_float4(__uint_as_float(x[0]) * scale, __uint_as_float(x[1]) * scale,
+                                        __uint_as_float(x[2]) * scale, __uint_as_float(x[3]) * scale);
+                    }
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars->stage_full);
+                if (warp == 0) {
+                    if (!warp_wait(&bars->stage_full, m & 1, kSiteStageFull, abort)) break;
+                    if (leader) {
+#pragma unroll
+                        for (int sl = 0; sl < C::kDQSlices; ++sl)
+                            tma_reduce_add_3d(&tmap_dq, smem + C::kOffDQS + sl * C::kDQStageBytes,
+                                              32 * sl, i * kTile, bh);
+                        tma_store_commit();
+                    }
+                }
+            } else {
+                // 64 columns at a time; the columns are released after the last load
+                const int q = i * kTile + (int)row;
+                float* dst = dq_accum + ((size_t)bh * T + q) * D;
+#pragma unroll
+                for (int c = 0; c < D / 64; ++c) {
+                    uint32_t r[64];
+                    tmem_ld32(tmem + lane_off + C::kColDQ + c * 64, r);
+                    tmem_ld32(tmem + lane_off + C::kColDQ + c * 64 + 32, r + 32);
+                    tmem_wait_ld();
+                    if (c == D / 64 - 1) {
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&bars->dq_free);
+                    }
+                    if (q < T) {
+#pragma unroll
+                        for (int e = 0; e < 16; ++e)
+                            red_add_v4(dst + c * 64 + 4 * e, __uint_as_float(r[4 * e]) * scale,
+                                       __uint_as_float(r[4 * e + 1]) * scale,
+                                       __uint_as_float(r[4 * e + 2]) * scale,
+                                       __uint_as_float(r[4 * e + 3]) * scale);
+                    }
+                }
+            }
+        }
+        if (C::kTmaDQ && leader) tma_store_wait_all();  // reduces done before the CTA exits
+    } else if (warp < kWarpProducer) {
+        // ----------------------------------------------------------- compute
+        regs_inc<C::kRegsCompute>();
+        const uint32_t quarter = warp & 3;
+        const uint32_t half = (warp - kWarpCompute0) >> 2;  // which 64 query columns
+        const uint32_t row = (quarter << 5) + lane;          // key row
+        const uint32_t lane_off = (quarter << 5) << 16;
+        uint8_t* p_smem = smem + C::kOffP + half * C::kChunkBytes;
+        uint8_t* ds_smem = smem + C::kOffDS + half * C::kChunkBytes;
+        const int c0 = half * 64;                            // first query column owned
+        bool ok = !*abort;
+
+        for (int n = 0; ok && n < n_iter; ++n) {
+            const int sq = n % C::kStagesQ;
+            const int i = i_begin + n;
+            const bool diag = causal && (i == kt);
+            // ---- P^T for 64 query columns
+            if (!warp_wait(&bars->s_full, n & 1, kSiteSFull, abort)) { ok = false; break; }
+            tc_fence_after();
+            uint32_t sraw[64];
+            tmem_ld32(tmem + lane_off + C::kColS + c0, sraw);
+            tmem_ld32(tmem + lane_off + C::kColS + c0 + 32, sraw + 32);
+            tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->s_free);
+            // LSE_i and D_i arrived with Q_i
+            if (!warp_wait(&bars->q_full[sq], (n / C::kStagesQ) & 1, kSiteQFull, abort)) {
+                ok = false;
+                break;
+            }
+            // P^T = exp2(S^T * scale * log2(e) - LSE * log2(e)), two queries at a time
+            const float4* nlse4 = reinterpret_cast<const float4*>(s_lse + sq * kTile + c0);
+            const float2 sl2 = make_float2(scale_log2, scale_log2);
+            float p[64];
+#pragma unroll
+            for (int c4 = 0; c4 < 16; ++c4) {
+                const float4 l = nlse4[c4];
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int c = 4 * c4 + 2 * h;
+                    const float2 x = ffma2(
+                        make_float2(__uint_as_float(sraw[c]), __uint_as_float(sraw[c + 1])), sl2,
+                        h == 0 ? make_float2(l.x, l.y) : make_float2(l.z, l.w));
+                    float2 e2;
+                    if (!PRECISE && use_poly_pair(c >> 1)) {
+                        e2 = exp2_poly2(x);
+                    } else {
+                        e2.x = ex2_approx(x.x);
+                        e2.y = ex2_approx(x.y);
+                    }
+                    p[c] = e2.x;
+                    p[c + 1] = e2.y;
+                }
+            }
+            if (diag) {  // a query that precedes the key row
+#pragma unroll
+                for (int c = 0; c < 64; ++c)
+                    if (c0 + c < (int)row) p[c] = 0.f;
+            }
+            // the P^T buffer must no longer be read by the previous iteration's MMAs
+            if (n > 0) {
+                uint64_t* fb = C::kSeparatePdS ? &bars->p_free : &bars->ds_free;
+                if (!warp_wait(fb, (n - 1) & 1, kSitePFree, abort)) { ok = false; break; }
+            }
+            if constexpr (C::kPInTmem) {
+                uint32_t pk[32];
+#pragma unroll
+                for (int e = 0; e < 32; ++e) pk[e] = pack_bf16x2(p[2 * e], p[2 * e + 1]);
+                tc_fence_after();
+                tmem_st32(tmem + lane_off + C::kColP + half * 32, pk);
+                tmem_wait_st();
+                tc_fence_before();
+            } else {
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch)  // 8 chunks of 8 queries
+                    store_split8<PRECISE>(p_smem, C::kScoreBytes, sw128_offset(row, ch),
+                                          p + ch * 8);
+                fence_proxy_async_smem();
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->p_full);
+
+            // ---- dS^T = P^T o (dP^T - D), 32 queries at a time
+            if (!warp_wait(&bars->dp_full, n & 1, kSiteDPFull, abort)) { ok = false; break; }
+            {
+                // dS^T buffer: free once dK/dQ of the previous iteration (separate
+                // buffers) or dV of this one (shared buffer) have read it
+                bool w = true;
+                if (C::kSeparatePdS) {
+                    if (n > 0) w = warp_wait(&bars->ds_free, (n - 1) & 1, kSiteDSFree, abort);
+                } else {
+                    w = warp_wait(&bars->p_free, n & 1, kSitePFree, abort);
+                }
+                if (!w) { ok = false; break; }
+            }
+            tc_fence_after();
+            const float4* d4 = reinterpret_cast<const float4*>(s_delta + sq * kTile + c0);
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+                uint32_t dp[32];
+                tmem_ld32(tmem + lane_off + C::kColDP + c0 + c * 32, dp);
+                tmem_wait_ld();
+#pragma unroll
+                for (int ch = 0; ch < 4; ++ch) {  // 4 chunks of 8 queries
+                    const float4 da = d4[c * 8 + ch * 2], db = d4[c * 8 + ch * 2 + 1];
+                    const float2 dv2[4] = {make_float2(da.x, da.y), make_float2(da.z, da.w),
+                                           make_float2(db.x, db.y), make_float2(db.z, db.w)};
+                    float ds[8];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int qc = c * 32 + ch * 8 + 2 * e;
+                        const float2 g = fmul2(
+                            make_float2(p[qc], p[qc + 1]),
+                            fsub2(make_float2(__uint_as_float(dp[ch * 8 + 2 * e]),
+                                              __uint_as_float(dp[ch * 8 + 2 * e + 1])),
+                                  dv2[e]));
+                        ds[2 * e] = g.x;
+                        ds[2 * e + 1] = g.y;
+                    }
+                    store_split8<PRECISE>(ds_smem, C::kScoreBytes, sw128_offset(row, c * 4 + ch),
+                                          ds);
+                }
+            }
+            tc_fence_before();
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->ds_full);
+        }
+
+        // ------------------------------------------------ dK / dV epilogue
+        if (ok && warp_wait(&bars->acc_done, 0, kSiteAccDone, abort)) {
+            tc_fence_after();
+            const int key = kt * kTile + (int)row;
+            const size_t base = ((size_t)bh * T + key) * D + half * (D / 2);
+#pragma unroll
+            for (int which = 0; which < 2; ++which) {
+                const uint32_t col = (which == 0 ? C::kColDV : C::kColDK) + half * (D / 2);
+                const float mul = which == 0 ? 1.f : scale;
+                void* out = which == 0 ? dv_out : dk_out;
+#pragma unroll
+                for (int c = 0; c < D / 64; ++c) {
+                    uint32_t r[32];
+                    tmem_ld32(tmem + lane_off + col + c * 32, r);
+                    tmem_wait_ld();
+                    if (key < T) {
+                        if (grad_f32) {
+                            float* o = reinterpret_cast<float*>(out) + base + c * 32;
+#pragma unroll
+                            for (int e = 0; e < 8; ++e)
+                                reinterpret_cast<float4*>(o)[e] = make_float4(
+                                    __uint_as_float(r[4 * e]) * mul,
+                                    __uint_as_float(r[4 * e + 1]) * mul,
+                                    __uint_as_float(r[4 * e + 2]) * mul,
+                                    __uint_as_float(r[4 * e + 3]) * mul);
+                        } else {
+                            uint4* o = reinterpret_cast<uint4*>(
+                                reinterpret_cast<__nv_bfloat16*>(out) + base + c * 32);
+#pragma unroll
+                            for (int e = 0; e < 4; ++e)
+                                o[e] = make_uint4(
+                                    pack_bf16x2(__uint_as_float(r[8 * e]) * mul,
+                                                __uint_as_float(r[8 * e + 1]) * mul),
+                                    pack_bf16x2(__uint_as_float(r[8 * e + 2]) * mul,
+                                                __uint_as_float(r[8 * e + 3]) * mul),
+                                    pack_bf16x2(__uint_as_float(r[8 * e + 4]) * mul,
+                                                __uint_as_float(r[8 * e + 5]) * mul),
+                                    pack_bf16x2(__uint_as_float(r[8 * e + 6]) * mul,
+                                                __uint_as_float(r[8 * e + 7]) * mul));
+                        }
+                    }
+                }
+            }
+        }
+    } else {
+        regs_dec<C::kRegsCtl>();
+        if (warp == kWarpProducer && lane == 0) {
+            // -------------------------------------------------------- producer
             int last_q[3] = {-1, -1, -1}, last_do[2] = {-1, -1};
             bool kv_issued = false;
             if (!*abort) {
@@ -259,27 +543,28 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 for (int s = 0; s < 2; ++s)
                     if (last_do[s] >= 0) mbar_wait_drain(&bars->do_full[s], last_do[s] & 1);
             }
-        }
-    } else if (warp == 1) {
-        // --------------------------------------------------------- MMA issuer
-        if (lane == 0 && !*abort) {
+        } else if (warp == kWarpMma) {
+            // ------------------------------------------------------ MMA issuer
+            // The whole warp runs this loop; one elected lane issues each MMA.
             const uint32_t tS = tmem + C::kColS;
             const uint32_t tDP = tmem + C::kColDP;
             const uint32_t tDQ = tmem + C::kColDQ;
             const uint32_t tDV = tmem + C::kColDV;
             const uint32_t tDK = tmem + C::kColDK;
+            const uint32_t tP = tmem + C::kColP;
             const uint32_t k_addr = smem_u32(smem + C::kOffK);
             const uint32_t v_addr = smem_u32(smem + C::kOffV);
             const uint32_t p_addr = smem_u32(smem + C::kOffP);
             const uint32_t ds_addr = smem_u32(smem + C::kOffDS);
-            bool ok = mbar_wait(&bars->kv_full, 0, kSiteKV, abort);
+            bool ok = __all_sync(0xffffffffu, !*abort) &&
+                      warp_wait(&bars->kv_full, 0, kSiteKV, abort);
 
             // S^T = K Q^T  or  dP^T = V dO^T: M = 128 keys, N = 128 queries, K = d
             auto score_mma = [&](uint32_t d_tmem, uint32_t a_addr, uint32_t b_addr) {
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * C::kChunkBytes + (kk & 3) * 32;
-                    mma_ss(d_tmem, sdesc_sw128(a_addr + off, 16, 1024),
+                    mma_ss_warp(d_tmem, sdesc_sw128(a_addr + off, 16, 1024),
                            sdesc_sw128(b_addr + off, 16, 1024), C::kIdescScore, kk > 0 ? 1u : 0u);
                 }
             };
@@ -288,16 +573,23 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
                 for (int kk = 0; kk < kTile / 16; ++kk) {
                     const uint32_t aoff = (kk >> 2) * C::kChunkBytes + (kk & 3) * 32;
-                    mma_ss(d_tmem, sdesc_sw128(a_addr + aoff, 16, 1024),
+                    mma_ss_warp(d_tmem, sdesc_sw128(a_addr + aoff, 16, 1024),
                            sdesc_sw128(b_addr + kk * 2048, C::kChunkBytes, 1024), C::kIdescGrad,
                            (acc || kk > 0) ? 1u : 0u);
                 }
+            };
+            // dV += P^T dO with P^T in tensor memory (16 queries = 8 columns per step)
+            auto dv_mma_tmem = [&](uint32_t b_addr, bool acc) {
+#pragma unroll
+                for (int kk = 0; kk < kTile / 16; ++kk)
+                    mma_ts_warp(tDV, tP + kk * 8, sdesc_sw128(b_addr + kk * 2048, C::kChunkBytes, 1024),
+                           C::kIdescGrad, (acc || kk > 0) ? 1u : 0u);
             };
             // dQ_i = dS K: M = 128 queries (dS^T read MN-major), N = d, K = 128 keys
             auto dq_mma = [&](uint32_t a_addr, bool acc) {
 #pragma unroll
                 for (int kk = 0; kk < kTile / 16; ++kk)
-                    mma_ss(tDQ, sdesc_sw128(a_addr + kk * 2048, C::kChunkBytes, 1024),
+                    mma_ss_warp(tDQ, sdesc_sw128(a_addr + kk * 2048, C::kChunkBytes, 1024),
                            sdesc_sw128(k_addr + kk * 2048, C::kChunkBytes, 1024), C::kIdescDQ,
                            (acc || kk > 0) ? 1u : 0u);
             };
@@ -309,279 +601,88 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             };
 
             // prologue: S_0, dP_0
-            if (ok) ok = mbar_wait(&bars->q_full[0], 0, kSiteQFull, abort);
+            if (ok) ok = warp_wait(&bars->q_full[0], 0, kSiteQFull, abort);
             if (ok) {
                 tc_fence_after();
                 score_mma(tS, k_addr, q_stage(0));
-                mma_commit(&bars->s_full);
+                mma_commit_warp(&bars->s_full);
             }
-            if (ok) ok = mbar_wait(&bars->do_full[0], 0, kSiteDOFull, abort);
+            if (ok) ok = warp_wait(&bars->do_full[0], 0, kSiteDOFull, abort);
             if (ok) {
                 tc_fence_after();
                 score_mma(tDP, v_addr, do_stage(0));
-                mma_commit(&bars->dp_full);
+                mma_commit_warp(&bars->dp_full);
             }
             for (int n = 0; ok && n < n_iter; ++n) {
                 // S_{n+1} as soon as the compute warps hold S_n in registers
                 if (n + 1 < n_iter) {
-                    if (!mbar_wait(&bars->s_free, n & 1, kSiteSFree, abort)) { ok = false; break; }
-                    if (!mbar_wait(&bars->q_full[(n + 1) % C::kStagesQ],
+                    if (!warp_wait(&bars->s_free, n & 1, kSiteSFree, abort)) { ok = false; break; }
+                    if (!warp_wait(&bars->q_full[(n + 1) % C::kStagesQ],
                                    ((n + 1) / C::kStagesQ) & 1, kSiteQFull, abort)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
                     score_mma(tS, k_addr, q_stage(n + 1));
-                    mma_commit(&bars->s_full);
+                    mma_commit_warp(&bars->s_full);
                 }
                 // dV += P^T dO_n
-                if (!mbar_wait(&bars->p_full, n & 1, kSitePFull, abort)) { ok = false; break; }
+                if (!warp_wait(&bars->p_full, n & 1, kSitePFull, abort)) { ok = false; break; }
                 tc_fence_after();
-                grad_mma(tDV, p_addr, do_stage(n), n > 0);
-                if (PRECISE) grad_mma(tDV, p_addr + C::kScoreBytes, do_stage(n), true);
-                mma_commit(&bars->p_free);
-                mma_commit(&bars->do_empty[n % C::kStagesDO]);
+                if constexpr (C::kPInTmem) {
+                    dv_mma_tmem(do_stage(n), n > 0);
+                } else {
+                    grad_mma(tDV, p_addr, do_stage(n), n > 0);
+                    if (PRECISE) grad_mma(tDV, p_addr + C::kScoreBytes, do_stage(n), true);
+                }
+                mma_commit_warp(&bars->p_free);
+                mma_commit_warp(&bars->do_empty[n % C::kStagesDO]);
                 // dK += dS^T Q_n ; dQ_n = dS K
-                if (!mbar_wait(&bars->ds_full, n & 1, kSiteDSFull, abort)) { ok = false; break; }
+                if (!warp_wait(&bars->ds_full, n & 1, kSiteDSFull, abort)) { ok = false; break; }
                 tc_fence_after();
                 grad_mma(tDK, ds_addr, q_stage(n), n > 0);
                 if (PRECISE) grad_mma(tDK, ds_addr + C::kScoreBytes, q_stage(n), true);
                 // separate dQ columns: free once dQ_{n-1} is drained; shared with dP^T:
                 // dP_n has been read (ds_full)
                 if (C::kSeparateDQ && n > 0 &&
-                    !mbar_wait(&bars->dq_free, (n - 1) & 1, kSiteDQFree, abort)) {
+                    !warp_wait(&bars->dq_free, (n - 1) & 1, kSiteDQFree, abort)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
                 dq_mma(ds_addr, false);
                 if (PRECISE) dq_mma(ds_addr + C::kScoreBytes, true);
-                mma_commit(&bars->dq_full);
-                mma_commit(&bars->ds_free);
-                mma_commit(&bars->q_empty[n % C::kStagesQ]);
+                mma_commit_warp(&bars->dq_full);
+                mma_commit_warp(&bars->ds_free);
+                mma_commit_warp(&bars->q_empty[n % C::kStagesQ]);
                 // dP_{n+1}: its columns are free once dS_n is formed (separate dQ) or
                 // once dQ_n has left tensor memory (shared columns)
                 if (n + 1 < n_iter) {
                     if (!C::kSeparateDQ &&
-                        !mbar_wait(&bars->dq_free, n & 1, kSiteDQFree, abort)) {
+                        !warp_wait(&bars->dq_free, n & 1, kSiteDQFree, abort)) {
                         ok = false;
                         break;
                     }
-                    if (!mbar_wait(&bars->do_full[(n + 1) % C::kStagesDO],
+                    if (!warp_wait(&bars->do_full[(n + 1) % C::kStagesDO],
                                    ((n + 1) / C::kStagesDO) & 1, kSiteDOFull, abort)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
                     score_mma(tDP, v_addr, do_stage(n + 1));
-                    mma_commit(&bars->dp_full);
+                    mma_commit_warp(&bars->dp_full);
                 }
             }
-            if (ok) mma_commit(&bars->acc_done);
-            mma_commit(&bars->mma_final);
+            if (ok) mma_commit_warp(&bars->acc_done);
+            mma_commit_warp(&bars->mma_final);
             mbar_wait_drain(&bars->mma_final, 0);
-        }
-    } else {
-        // ----------------------------------------------------------- compute
-        const uint32_t quarter = warp & 3;
-        const uint32_t half = (warp - 2) >> 2;          // which 64 query columns
-        const uint32_t row = (quarter << 5) + lane;      // key row (and dQ query row)
-        const uint32_t lane_off = (quarter << 5) << 16;
-        uint8_t* p_smem = smem + C::kOffP + half * C::kChunkBytes;
-        uint8_t* ds_smem = smem + C::kOffDS + half * C::kChunkBytes;
-        uint8_t* dq_stage = smem + C::kOffDQS + half * C::kDQStageBytes;
-        const bool leader = lane == 0 && quarter == 2;   // warps 2 and 6: one per half
-        const int c0 = half * 64;                        // first query column owned
-        bool ok = !*abort;
-
-        // dQ_m: this thread's query row, its half of the d columns, times scale,
-        // into the fp32 accumulator
-        auto drain_dq = [&](int m) -> bool {
-            if (!warp_wait(&bars->dq_full, m & 1, kSiteDQFull, abort)) return false;
-            tc_fence_after();
-            uint32_t r[D / 2];
-#pragma unroll
-            for (int c = 0; c < D / 64; ++c)
-                tmem_ld32(tmem + lane_off + C::kColDQ + half * (D / 2) + c * 32, r + c * 32);
-            tmem_wait_ld();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars->dq_free);
-            const int i = i_begin + m;
-            if constexpr (C::kTmaDQ) {
-                // staging must have been read by this half's previous reduce
-                if (leader) tma_store_wait_all_read();
-                named_bar_sync(2 + half, 128);
-#pragma unroll
-                for (int ch = 0; ch < 8; ++ch)
-                    *reinterpret_cast<float4*>(dq_stage + sw128_offset(row, ch)) = make_float4(
-                        __uint_as_float(r[4 * ch]) * scale, __uint_as_float(r[4 * ch + 1]) * scale,
-                        __uint_as_float(r[4 * ch + 2]) * scale,
-                        __uint_as_float(r[4 * ch + 3]) * scale);
-                fence_proxy_async_smem();
-                named_bar_sync(2 + half, 128);
-                if (leader) {
-                    tma_reduce_add_3d(&tmap_dq, dq_stage, 32 * half, i * kTile, bh);
-                    tma_store_commit();
-                }
-            } else {
-                const int q = i * kTile + (int)row;
-                if (q < T) {
-                    float* dst = dq_accum + ((size_t)bh * T + q) * D + half * (D / 2);
-#pragma unroll
-                    for (int e = 0; e < D / 8; ++e)
-                        red_add_v4(dst + 4 * e, __uint_as_float(r[4 * e]) * scale,
-                                   __uint_as_float(r[4 * e + 1]) * scale,
-                                   __uint_as_float(r[4 * e + 2]) * scale,
-                                   __uint_as_float(r[4 * e + 3]) * scale);
-                }
-            }
-            return true;
-        };
-
-        for (int n = 0; ok && n < n_iter; ++n) {
-            const int sq = n % C::kStagesQ;
-            const int i = i_begin + n;
-            const bool diag = causal && (i == kt);
-            // ---- P^T for 64 query columns
-            if (!warp_wait(&bars->s_full, n & 1, kSiteSFull, abort)) { ok = false; break; }
-            tc_fence_after();
-            uint32_t sraw[64];
-            tmem_ld32(tmem + lane_off + C::kColS + c0, sraw);
-            tmem_ld32(tmem + lane_off + C::kColS + c0 + 32, sraw + 32);
-            tmem_wait_ld();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars->s_free);
-            // LSE_i and D_i arrived with Q_i
-            if (!warp_wait(&bars->q_full[sq], (n / C::kStagesQ) & 1, kSiteQFull, abort)) {
-                ok = false;
-                break;
-            }
-            const float4* lse4 = reinterpret_cast<const float4*>(s_lse + sq * kTile + c0);
-            float p[64];
-#pragma unroll
-            for (int c4 = 0; c4 < 16; ++c4) {
-                const float4 l = lse4[c4];
-                const float lv[4] = {l.x, l.y, l.z, l.w};
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int c = 4 * c4 + e;
-                    float x = ex2_approx(fmaf(__uint_as_float(sraw[c]), scale_log2, -lv[e]));
-                    if (diag && c0 + c < (int)row) x = 0.f;  // query precedes the key row
-                    p[c] = x;
-                }
-            }
-            // the P^T buffer must no longer be read by the previous iteration's MMAs
-            if (n > 0) {
-                uint64_t* fb = C::kSeparatePdS ? &bars->p_free : &bars->ds_free;
-                if (!warp_wait(fb, (n - 1) & 1, kSitePFree, abort)) { ok = false; break; }
-            }
-#pragma unroll
-            for (int ch = 0; ch < 8; ++ch)  // 8 chunks of 8 queries
-                store_split8<PRECISE>(p_smem, C::kScoreBytes, sw128_offset(row, ch), p + ch * 8);
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars->p_full);
-
-            // ---- with its own columns, dQ_{n-1} drains while dP_n / dV_n run
-            if (C::kSeparateDQ && n > 0 && !drain_dq(n - 1)) { ok = false; break; }
-
-            // ---- dS^T = P^T o (dP^T - D), 32 queries at a time
-            if (!warp_wait(&bars->dp_full, n & 1, kSiteDPFull, abort)) { ok = false; break; }
-            {
-                // dS^T buffer: free once dK/dQ of the previous iteration (separate
-                // buffers) or dV of this one (shared buffer) have read it
-                bool w = true;
-                if (C::kSeparatePdS) {
-                    if (n > 0) w = warp_wait(&bars->ds_free, (n - 1) & 1, kSiteDSFree, abort);
-                } else {
-                    w = warp_wait(&bars->p_free, n & 1, kSitePFree, abort);
-                }
-                if (!w) { ok = false; break; }
-            }
-            tc_fence_after();
-            const float4* d4 = reinterpret_cast<const float4*>(s_delta + sq * kTile + c0);
-#pragma unroll
-            for (int c = 0; c < 2; ++c) {
-                uint32_t dp[32];
-                tmem_ld32(tmem + lane_off + C::kColDP + c0 + c * 32, dp);
-                tmem_wait_ld();
-#pragma unroll
-                for (int ch = 0; ch < 4; ++ch) {  // 4 chunks of 8 queries
-                    const float4 da = d4[c * 8 + ch * 2], db = d4[c * 8 + ch * 2 + 1];
-                    const float dv8[8] = {da.x, da.y, da.z, da.w, db.x, db.y, db.z, db.w};
-                    float ds[8];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const int qc = c * 32 + ch * 8 + e;
-                        ds[e] = p[qc] * (__uint_as_float(dp[ch * 8 + e]) - dv8[e]);
-                    }
-                    store_split8<PRECISE>(ds_smem, C::kScoreBytes, sw128_offset(row, c * 4 + ch),
-                                          ds);
-                }
-            }
-            tc_fence_before();
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars->ds_full);
-
-            // ---- sharing its columns with dP^T, dQ_n drains before dP_{n+1}
-            if (!C::kSeparateDQ && !drain_dq(n)) { ok = false; break; }
-        }
-        if (ok && C::kSeparateDQ && !drain_dq(n_iter - 1)) ok = false;
-        if (C::kTmaDQ && leader) tma_store_wait_all();  // reduces done before the CTA exits
-
-        // ------------------------------------------------ dK / dV epilogue
-        if (ok && warp_wait(&bars->acc_done, 0, kSiteAccDone, abort)) {
-            tc_fence_after();
-            const int key = kt * kTile + (int)row;
-            const size_t base = ((size_t)bh * T + key) * D + half * (D / 2);
-#pragma unroll
-            for (int which = 0; which < 2; ++which) {
-                const uint32_t col = (which == 0 ? C::kColDV : C::kColDK) + half * (D / 2);
-                const float mul = which == 0 ? 1.f : scale;
-                void* out = which == 0 ? dv_out : dk_out;
-#pragma unroll
-                for (int c = 0; c < D / 64; ++c) {
-                    uint32_t r[32];
-                    tmem_ld32(tmem + lane_off + col + c * 32, r);
-                    tmem_wait_ld();
-                    if (key < T) {
-                        if (grad_f32) {
-                            float* o = reinterpret_cast<float*>(out) + base + c * 32;
-#pragma unroll
-                            for (int e = 0; e < 8; ++e)
-                                reinterpret_cast<float4*>(o)[e] = make_float4(
-                                    __uint_as_float(r[4 * e]) * mul,
-                                    __uint_as_float(r[4 * e + 1]) * mul,
-                                    __uint_as_float(r[4 * e + 2]) * mul,
-                                    __uint_as_float(r[4 * e + 3]) * mul);
-                        } else {
-                            uint4* o = reinterpret_cast<uint4*>(
-                                reinterpret_cast<__nv_bfloat16*>(out) + base + c * 32);
-#pragma unroll
-                            for (int e = 0; e < 4; ++e)
-                                o[e] = make_uint4(
-                                    pack_bf16x2(__uint_as_float(r[8 * e]) * mul,
-                                                __uint_as_float(r[8 * e + 1]) * mul),
-                                    pack_bf16x2(__uint_as_float(r[8 * e + 2]) * mul,
-                                                __uint_as_float(r[8 * e + 3]) * mul),
-                                    pack_bf16x2(__uint_as_float(r[8 * e + 4]) * mul,
-                                                __uint_as_float(r[8 * e + 5]) * mul),
-                                    pack_bf16x2(__uint_as_float(r[8 * e + 6]) * mul,
-                                                __uint_as_float(r[8 * e + 7]) * mul));
-                        }
-                    }
-                }
-            }
         }
     }
 
     // ------------------------------------------------------------- teardown
     tc_fence_before();
     __syncthreads();
-    if (warp == 1) {
+    if (warp == kWarpMma) {
         __syncwarp();
         tc_fence_after();
         tmem_dealloc(tmem, C::kTmemCols);
@@ -589,8 +690,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 }
 
 // Row statistics of the backward, padded per head to t_pad = 128 * ceil(T / 128) rows:
-// rowstats[0][bh][t] = LSE * log2(e) and rowstats[1][bh][t] = D = rowsum(dO o O)
-// (fp32; +inf and 0 past T), and the dQ accumulator cleared.  O is bf16 or fp32
+// rowstats[0][bh][t] = -LSE * log2(e) (negated: it is the addend of the exponent) and
+// rowstats[1][bh][t] = D = rowsum(dO o O) (fp32; -inf and 0 past T), and the dQ
+// accumulator cleared.  O is bf16 or fp32
 // (TO); dO is bf16.  A group of D/8 consecutive threads covers one row, 8 elements
 // each, so every load of a warp is one contiguous span.
 template <int D, typename TO>
@@ -641,7 +743,7 @@ __global__ void __launch_bounds__(256) attn_bwd_preprocess_kernel(
 #pragma unroll
     for (int off = kGroup / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
     if (pr < padded_rows && part == 0) {
-        rowstats[pr] = valid ? lse[r] * kLog2e : INFINITY;
+        rowstats[pr] = valid ? -lse[r] * kLog2e : -INFINITY;
         rowstats[padded_rows + pr] = valid ? acc : 0.f;
     }
 }

@@ -37,6 +37,11 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
+// Which pairs of a row's exponentials go to the FMA-pipe polynomial (exp2_poly2)
+// instead of the MUFU unit: 3 of every 8, which balances the two units' time per
+// tile.  Precise mode keeps every exponential on the MUFU unit.
+__device__ __forceinline__ constexpr bool use_poly_pair(int e) { return (e & 7) >= 5; }
+
 // wait sites (for the device error word)
 enum : uint32_t {
     kSiteQ = 1, kSiteKFull, kSiteVFull, kSiteKVEmpty, kSiteSFull, kSiteSFree, kSitePFull,
@@ -78,6 +83,11 @@ struct FwdBarriers {
     uint32_t tmem_base;
     int abort;
 };
+
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, uint32_t site,
+                                          volatile int* abort) {
+    return __all_sync(0xffffffffu, mbar_wait(bar, parity, site, abort));
+}
 
 template <int D, bool PRECISE>
 __global__ void __launch_bounds__(kFwdThreads, 1)
@@ -165,17 +175,18 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         }
     } else if (warp == 1) {
         // --------------------------------------------------------- MMA issuer
-        if (lane == 0) {
+        // The whole warp runs this loop; one elected lane issues each MMA.
+        {
             const uint32_t tS = tmem + C::kColS;
             const uint32_t tO = tmem + C::kColO;
             const uint32_t q_addr = smem_u32(smem + C::kOffQ);
             // bit 13 of the instruction descriptor negates A: S = (-Q) K^T for scale < 0
             const uint32_t idesc_s = C::kIdescS | (negate_scores ? (1u << 13) : 0u);
-            bool ok = mbar_wait(&bars->q_full, 0, kSiteQ, abort);
+            bool ok = warp_wait(&bars->q_full, 0, kSiteQ, abort);
             auto issue_pv = [&](int m) -> bool {
                 const int st = m % C::kStages;
-                if (!mbar_wait(&bars->p_full, m & 1, kSitePFull, abort)) return false;
-                if (!mbar_wait(&bars->v_full[st], (m / C::kStages) & 1, kSiteVFull, abort))
+                if (!warp_wait(&bars->p_full, m & 1, kSitePFull, abort)) return false;
+                if (!warp_wait(&bars->v_full[st], (m / C::kStages) & 1, kSiteVFull, abort))
                     return false;
                 tc_fence_after();
                 const uint32_t tP = tmem + ((m & 1) ? C::kColP1 : C::kColP0);
@@ -185,20 +196,20 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 for (int kk = 0; kk < kTile / 16; ++kk) {
                     // B = V tile, MN-major: 16 keys = 2 x 8-row groups of 1024 bytes
                     const uint64_t bdesc = sdesc_sw128(v_addr + kk * 2048, C::kChunkBytes, 1024);
-                    mma_ts(tO, tP + kk * 8, bdesc, C::kIdescPV, (m > 0 || kk > 0) ? 1u : 0u);
-                    if (PRECISE) mma_ts(tO, tPlo + kk * 8, bdesc, C::kIdescPV, 1u);
+                    mma_ts_warp(tO, tP + kk * 8, bdesc, C::kIdescPV, (m > 0 || kk > 0) ? 1u : 0u);
+                    if (PRECISE) mma_ts_warp(tO, tPlo + kk * 8, bdesc, C::kIdescPV, 1u);
                 }
-                mma_commit(&bars->pv_done);
-                mma_commit(&bars->kv_empty[st]);
+                mma_commit_warp(&bars->pv_done);
+                mma_commit_warp(&bars->kv_empty[st]);
                 return true;
             };
             for (int n = 0; ok && n < n_tiles; ++n) {
                 const int st = n % C::kStages;
-                if (!mbar_wait(&bars->k_full[st], (n / C::kStages) & 1, kSiteKFull, abort)) {
+                if (!warp_wait(&bars->k_full[st], (n / C::kStages) & 1, kSiteKFull, abort)) {
                     ok = false;
                     break;
                 }
-                if (n > 0 && !mbar_wait(&bars->s_free, (n - 1) & 1, kSiteSFree, abort)) {
+                if (n > 0 && !warp_wait(&bars->s_free, (n - 1) & 1, kSiteSFree, abort)) {
                     ok = false;
                     break;
                 }
@@ -209,18 +220,18 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                     const uint32_t koff = (kk >> 2) * C::kChunkBytes + (kk & 3) * 32;
                     const uint64_t adesc = sdesc_sw128(q_addr + koff, 16, 1024);
                     const uint64_t bdesc = sdesc_sw128(k_addr + koff, 16, 1024);
-                    mma_ss(tS, adesc, bdesc, idesc_s, kk > 0 ? 1u : 0u);
+                    mma_ss_warp(tS, adesc, bdesc, idesc_s, kk > 0 ? 1u : 0u);
                 }
-                mma_commit(&bars->s_full);
+                mma_commit_warp(&bars->s_full);
                 if (n > 0 && !issue_pv(n - 1)) {
                     ok = false;
                     break;
                 }
             }
             if (ok) ok = issue_pv(n_tiles - 1);
-            if (ok) mma_commit(&bars->o_done);
+            if (ok) mma_commit_warp(&bars->o_done);
             // every MMA this thread issued must retire before tensor memory is freed
-            mma_commit(&bars->mma_final);
+            mma_commit_warp(&bars->mma_final);
             mbar_wait_drain(&bars->mma_final, 0);
         }
     } else {
@@ -257,18 +268,22 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             const int key_lim = diag ? (int)row : (tail ? T - 1 - j * kTile : kTile - 1);
             float s[kTile];
 #pragma unroll
-            for (int c = 0; c < kTile; ++c) {
-                s[c] = __uint_as_float(sraw[c]);
-                if (masked_tile && c > key_lim) s[c] = -INFINITY;
+            for (int c = 0; c < kTile; ++c) s[c] = __uint_as_float(sraw[c]);
+            if (masked_tile) {  // the same for every thread of the CTA
+#pragma unroll
+                for (int c = 0; c < kTile; ++c)
+                    if (c > key_lim) s[c] = -INFINITY;
             }
-            float mx[8];
+            // four independent chains of three-input max
+            float mx[4];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) mx[e] = s[e];
+            for (int e = 0; e < 4; ++e) mx[e] = fmaxf(s[2 * e], s[2 * e + 1]);
 #pragma unroll
-            for (int c = 8; c < kTile; ++c) mx[c & 7] = fmaxf(mx[c & 7], s[c]);
+            for (int c = 8; c < kTile; c += 8) {
 #pragma unroll
-            for (int e = 0; e < 4; ++e) mx[e] = fmaxf(mx[e], mx[e + 4]);
-            const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * scale_log2;
+                for (int e = 0; e < 4; ++e) mx[e] = fmax3(mx[e], s[c + 2 * e], s[c + 2 * e + 1]);
+            }
+            const float mt = fmax3(mx[0], mx[1], fmaxf(mx[2], mx[3])) * scale_log2;
 
             float alpha = 1.f;
             bool need = false;
@@ -305,34 +320,41 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             const uint32_t tP = tmem + lane_off + ((n & 1) ? C::kColP1 : C::kColP0);
             const uint32_t tPlo = tmem + lane_off + ((n & 1) ? C::kColPlo1 : C::kColPlo0);
             const float neg_m = -m_run;
-            float ls[8];
+            const float2 sl2 = make_float2(scale_log2, scale_log2);
+            const float2 nm2 = make_float2(neg_m, neg_m);
+            float2 ls[4];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) ls[e] = 0.f;
+            for (int e = 0; e < 4; ++e) ls[e] = make_float2(0.f, 0.f);
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
                 uint32_t pk[32], pl[32];
 #pragma unroll
                 for (int e = 0; e < 32; ++e) {
                     const int c = half * 64 + 2 * e;
-                    float p0 = ex2_approx(fmaf(s[c], scale_log2, neg_m));
-                    float p1 = ex2_approx(fmaf(s[c + 1], scale_log2, neg_m));
-                    if (masked_tile) {  // also covers scale 0, where -inf * 0 is NaN
-                        p0 = c > key_lim ? 0.f : p0;
-                        p1 = c + 1 > key_lim ? 0.f : p1;
+                    const float2 x = ffma2(make_float2(s[c], s[c + 1]), sl2, nm2);
+                    float2 p;
+                    if (!PRECISE && use_poly_pair(e)) {
+                        p = exp2_poly2(x);
+                    } else {
+                        p.x = ex2_approx(x.x);
+                        p.y = ex2_approx(x.y);
                     }
-                    ls[(2 * e) & 7] += p0;
-                    ls[(2 * e + 1) & 7] += p1;
-                    pk[e] = pack_bf16x2(p0, p1);
+                    if (masked_tile) {  // also covers scale 0, where -inf * 0 is NaN
+                        p.x = c > key_lim ? 0.f : p.x;
+                        p.y = c + 1 > key_lim ? 0.f : p.y;
+                    }
+                    ls[e & 3] = fadd2(ls[e & 3], p);
+                    pk[e] = pack_bf16x2(p.x, p.y);
                     if (PRECISE)
-                        pl[e] = pack_bf16x2(p0 - bf16_lo_to_float(pk[e]),
-                                            p1 - bf16_hi_to_float(pk[e]));
+                        pl[e] = pack_bf16x2(p.x - bf16_lo_to_float(pk[e]),
+                                            p.y - bf16_hi_to_float(pk[e]));
                 }
                 tmem_st32(tP + half * 32, pk);
                 if (PRECISE) tmem_st32(tPlo + half * 32, pl);
             }
-            const float ls0 = (ls[0] + ls[1]) + (ls[2] + ls[3]);
-            const float ls1 = (ls[4] + ls[5]) + (ls[6] + ls[7]);
-            l_run += ls0 + ls1;
+            const float2 ls01 = fadd2(ls[0], ls[1]), ls23 = fadd2(ls[2], ls[3]);
+            const float2 lsum = fadd2(ls01, ls23);
+            l_run += lsum.x + lsum.y;
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();

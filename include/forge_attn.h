@@ -96,7 +96,7 @@ int forge_attn_fwd_ex(const void* q, const void* k, const void* v, void* o, floa
 
 /*
  * Bytes of device workspace forge_attn_bwd needs: the row statistics (fp32
- * [2][B*H][t_pad], t_pad = 128 * ceil(T / 128): LSE * log2(e), then D) and the fp32
+ * [2][B*H][t_pad], t_pad = 128 * ceil(T / 128): -LSE * log2(e), then D) and the fp32
  * dQ accumulator ([B][H][T][d]), each at a 256-byte aligned offset.  Returns 0 for
  * arguments forge_attn_bwd would reject.
  */
@@ -131,8 +131,8 @@ int forge_attn_bwd_ex(const void* q, const void* k, const void* v, const void* o
  * them one by one.  forge_attn_bwd_ex is exactly these three in order.
  *
  * forge_attn_bwd_preprocess: the row statistics rowstats (fp32 [2][B*H][t_pad],
- *   t_pad = 128 * ceil(T / 128), 16-byte aligned): rowstats[0][bh][t] = lse * log2(e)
- *   and rowstats[1][bh][t] = D = sum_k dO[t][k] * o[t][k], with +inf and 0 in the
+ *   t_pad = 128 * ceil(T / 128), 16-byte aligned): rowstats[0][bh][t] = -lse * log2(e)
+ *   and rowstats[1][bh][t] = D = sum_k dO[t][k] * o[t][k], with -inf and 0 in the
  *   padding rows t >= T; and dq_accum (fp32 [B][H][T][d]) set to zero unless it is
  *   NULL.  flags: FORGE_ATTN_O_IN_F32 (o is fp32).
  * forge_attn_bwd_dkdv: recomputes P per key tile from the row statistics, writes dk
