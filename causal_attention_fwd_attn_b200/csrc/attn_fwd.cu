@@ -38,9 +38,10 @@ constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
 // Which pairs of a row's exponentials go to the FMA-pipe polynomial (exp2_poly2)
-// instead of the MUFU unit: 3 of every 8, which balances the two units' time per
-// tile.  Precise mode keeps every exponential on the MUFU unit.
-__device__ __forceinline__ constexpr bool use_poly_pair(int e) { return (e & 7) >= 5; }
+// instead of the MUFU unit.  None: with one softmax warp per SM sub-partition this
+// kernel is latency-bound rather than MUFU-bound, and the polynomial's extra
+// instructions measured slower at every share tried (3/8 to 6/8).
+__device__ __forceinline__ constexpr bool use_poly_pair(int) { return false; }
 
 // wait sites (for the device error word)
 enum : uint32_t {
@@ -274,16 +275,17 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 for (int c = 0; c < kTile; ++c)
                     if (c > key_lim) s[c] = -INFINITY;
             }
-            // four independent chains of three-input max
-            float mx[4];
+            // eight independent chains of three-input max (16 values each), then 8 -> 1
+            float mx[8];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) mx[e] = fmaxf(s[2 * e], s[2 * e + 1]);
+            for (int e = 0; e < 8; ++e) {
+                mx[e] = fmaxf(s[16 * e], s[16 * e + 1]);
 #pragma unroll
-            for (int c = 8; c < kTile; c += 8) {
-#pragma unroll
-                for (int e = 0; e < 4; ++e) mx[e] = fmax3(mx[e], s[c + 2 * e], s[c + 2 * e + 1]);
+                for (int c = 2; c < 16; c += 2) mx[e] = fmax3(mx[e], s[16 * e + c], s[16 * e + c + 1]);
             }
-            const float mt = fmax3(mx[0], mx[1], fmaxf(mx[2], mx[3])) * scale_log2;
+            const float mt =
+                fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7])) *
+                scale_log2;
 
             float alpha = 1.f;
             bool need = false;
