@@ -80,19 +80,18 @@ struct BwdCfg {
     static constexpr int kTileBytes = kChunks * kChunkBytes;
     // dQ through shared memory and a TMA reduce where there is room (d = 64 default)
     static constexpr bool kTmaDQ = (D == 64 && !PRECISE);
-    // P^T goes back into tensor memory (bf16 pairs) as the A operand of dV where
-    // columns are left for it (d = 64 default); otherwise into shared memory.
-    static constexpr bool kPInTmem = (D == 64 && !PRECISE);
+    // P^T goes back into tensor memory (bf16 pairs) as the A operand of dV: into
+    // columns of its own where 64 are left (d = 64 default), otherwise over the S^T
+    // columns it was computed from (each 64-query half into the first 32 (hi) and
+    // last 32 (lo, precise mode) of its own 64 columns), so the next S^T waits for dV.
+    static constexpr bool kPAliasS = !(D == 64 && !PRECISE);
     static constexpr int kStagesQ = kTmaDQ ? 3 : 2;
     // Precise mode at d = 128 needs the room of one dO stage for the lo buffer.
     static constexpr int kStagesDO = (D == 128 && PRECISE) ? 1 : 2;
-    // P^T and dS^T: [128 keys][128 queries] bf16 = two 64-query chunks; in precise
-    // mode each is a hi buffer followed by a lo buffer.
+    // dS^T: [128 keys][128 queries] bf16 = two 64-query chunks; in precise mode a hi
+    // buffer followed by a lo buffer.
     static constexpr int kScoreBytes = 2 * kChunkBytes;
     static constexpr int kSplit = PRECISE ? 2 : 1;
-    // With d = 128 shared memory only holds one set of score buffers, used for P^T
-    // and then for dS^T.
-    static constexpr bool kSeparatePdS = (D == 64);
     // With d = 64 dQ_i has tensor-memory columns of its own.
     static constexpr bool kSeparateDQ = (D == 64);
     // dQ staging for the TMA reduce: per column half, [128 rows][32 fp32] swizzled
@@ -101,9 +100,7 @@ struct BwdCfg {
     static constexpr int kOffV = kOffK + kTileBytes;
     static constexpr int kOffQ = kOffV + kTileBytes;
     static constexpr int kOffDO = kOffQ + kStagesQ * kTileBytes;
-    static constexpr int kOffP = kOffDO + kStagesDO * kTileBytes;
-    static constexpr int kPBytes = kPInTmem ? 0 : kSplit * kScoreBytes;
-    static constexpr int kOffDS = kSeparatePdS ? kOffP + kPBytes : kOffP;
+    static constexpr int kOffDS = kOffDO + kStagesDO * kTileBytes;
     static constexpr int kOffDQS = kOffDS + kSplit * kScoreBytes;
     static constexpr int kDQSlices = kTmaDQ ? D / 32 : 0;  // 32-column staging slices
     static constexpr int kOffLse = kOffDQS + kDQSlices * kDQStageBytes;
@@ -113,10 +110,14 @@ struct BwdCfg {
     static_assert(kSmemBytes <= 232448, "shared memory budget");
     static constexpr uint32_t kColDV = 0, kColDK = D, kColS = 2 * D, kColDP = 2 * D + 128;
     static constexpr uint32_t kColDQ = kSeparateDQ ? 2 * D + 256 : kColDP;
-    static constexpr uint32_t kColP = 3 * D + 256;
+    static constexpr uint32_t kColP = kPAliasS ? kColS : 3 * D + 256;
     static constexpr uint32_t kTmemCols = 512;
     static_assert(kColDQ + D <= kTmemCols, "tensor memory budget");
-    static_assert(!kPInTmem || (kSeparateDQ && kColP + 64 <= kTmemCols), "tensor memory budget");
+    static_assert(kPAliasS || (kSeparateDQ && kColP + 64 <= kTmemCols), "tensor memory budget");
+    // tensor-memory column of P^T's 16-query group kk (0..7), hi part
+    static __device__ __forceinline__ constexpr uint32_t p_col(int kk) {
+        return kPAliasS ? kColS + (kk >> 2) * 64 + (kk & 3) * 8 : kColP + kk * 8;
+    }
     // registers per thread after setmaxnreg (the launch gives 512 x 128): the precise
     // d = 128 MMA issuer needs more, its drain (64 columns at a time) less
     static constexpr uint32_t kRegsDrain = (D == 128 && PRECISE) ? 80 : 96;
@@ -321,7 +322,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const uint32_t half = (warp - kWarpCompute0) >> 2;  // which 64 query columns
         const uint32_t row = (quarter << 5) + lane;          // key row
         const uint32_t lane_off = (quarter << 5) << 16;
-        uint8_t* p_smem = smem + C::kOffP + half * C::kChunkBytes;
         uint8_t* ds_smem = smem + C::kOffDS + half * C::kChunkBytes;
         const int c0 = half * 64;                            // first query column owned
         bool ok = !*abort;
@@ -337,9 +337,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             tmem_ld32(tmem + lane_off + C::kColS + c0, sraw);
             tmem_ld32(tmem + lane_off + C::kColS + c0 + 32, sraw + 32);
             tmem_wait_ld();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars->s_free);
+            if constexpr (!C::kPAliasS) {
+                // S^T is in registers: its columns may take the next product
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars->s_free);
+            }
             // LSE_i and D_i arrived with Q_i
             if (!warp_wait(&bars->q_full[sq], (n / C::kStagesQ) & 1, kSiteQFull, abort)) {
                 ok = false;
@@ -374,41 +377,43 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 for (int c = 0; c < 64; ++c)
                     if (c0 + c < (int)row) p[c] = 0.f;
             }
-            // the P^T buffer must no longer be read by the previous iteration's MMAs
-            if (n > 0) {
-                uint64_t* fb = C::kSeparatePdS ? &bars->p_free : &bars->ds_free;
-                if (!warp_wait(fb, (n - 1) & 1, kSitePFree, abort)) { ok = false; break; }
+            // P^T into tensor memory.  Own columns: they must no longer be read by the
+            // previous iteration's dV.  Over S^T: this thread has read its S^T columns,
+            // and S_n was issued after dV_{n-1}.
+            if (!C::kPAliasS && n > 0 &&
+                !warp_wait(&bars->p_free, (n - 1) & 1, kSitePFree, abort)) {
+                ok = false;
+                break;
             }
-            if constexpr (C::kPInTmem) {
+            {
                 uint32_t pk[32];
 #pragma unroll
                 for (int e = 0; e < 32; ++e) pk[e] = pack_bf16x2(p[2 * e], p[2 * e + 1]);
+                const uint32_t tp = tmem + lane_off + C::p_col(4 * (int)half);
                 tc_fence_after();
-                tmem_st32(tmem + lane_off + C::kColP + half * 32, pk);
+                if constexpr (PRECISE) {
+                    uint32_t pl[32];  // remainders p - bf16(p), the lo terms
+#pragma unroll
+                    for (int e = 0; e < 32; ++e)
+                        pl[e] = pack_bf16x2(p[2 * e] - bf16_lo_to_float(pk[e]),
+                                            p[2 * e + 1] - bf16_hi_to_float(pk[e]));
+                    tmem_st32(tp, pk);
+                    tmem_st32(tp + 32, pl);
+                } else {
+                    tmem_st32(tp, pk);
+                }
                 tmem_wait_st();
                 tc_fence_before();
-            } else {
-#pragma unroll
-                for (int ch = 0; ch < 8; ++ch)  // 8 chunks of 8 queries
-                    store_split8<PRECISE>(p_smem, C::kScoreBytes, sw128_offset(row, ch),
-                                          p + ch * 8);
-                fence_proxy_async_smem();
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars->p_full);
 
             // ---- dS^T = P^T o (dP^T - D), 32 queries at a time
             if (!warp_wait(&bars->dp_full, n & 1, kSiteDPFull, abort)) { ok = false; break; }
-            {
-                // dS^T buffer: free once dK/dQ of the previous iteration (separate
-                // buffers) or dV of this one (shared buffer) have read it
-                bool w = true;
-                if (C::kSeparatePdS) {
-                    if (n > 0) w = warp_wait(&bars->ds_free, (n - 1) & 1, kSiteDSFree, abort);
-                } else {
-                    w = warp_wait(&bars->p_free, n & 1, kSitePFree, abort);
-                }
-                if (!w) { ok = false; break; }
+            // dS^T buffer: free once dK and dQ of the previous iteration have read it
+            if (n > 0 && !warp_wait(&bars->ds_free, (n - 1) & 1, kSiteDSFree, abort)) {
+                ok = false;
+                break;
             }
             tc_fence_after();
             const float4* d4 = reinterpret_cast<const float4*>(s_delta + sq * kTile + c0);
@@ -551,10 +556,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             const uint32_t tDQ = tmem + C::kColDQ;
             const uint32_t tDV = tmem + C::kColDV;
             const uint32_t tDK = tmem + C::kColDK;
-            const uint32_t tP = tmem + C::kColP;
             const uint32_t k_addr = smem_u32(smem + C::kOffK);
             const uint32_t v_addr = smem_u32(smem + C::kOffV);
-            const uint32_t p_addr = smem_u32(smem + C::kOffP);
             const uint32_t ds_addr = smem_u32(smem + C::kOffDS);
             bool ok = __all_sync(0xffffffffu, !*abort) &&
                       warp_wait(&bars->kv_full, 0, kSiteKV, abort);
@@ -578,12 +581,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                            (acc || kk > 0) ? 1u : 0u);
                 }
             };
-            // dV += P^T dO with P^T in tensor memory (16 queries = 8 columns per step)
-            auto dv_mma_tmem = [&](uint32_t b_addr, bool acc) {
+            // dV += P^T dO with P^T in tensor memory (16 queries = 8 columns per step;
+            // precise mode adds the lo terms, 32 columns further)
+            auto dv_mma = [&](uint32_t b_addr, bool acc) {
 #pragma unroll
-                for (int kk = 0; kk < kTile / 16; ++kk)
-                    mma_ts_warp(tDV, tP + kk * 8, sdesc_sw128(b_addr + kk * 2048, C::kChunkBytes, 1024),
-                           C::kIdescGrad, (acc || kk > 0) ? 1u : 0u);
+                for (int kk = 0; kk < kTile / 16; ++kk) {
+                    const uint64_t bdesc = sdesc_sw128(b_addr + kk * 2048, C::kChunkBytes, 1024);
+                    mma_ts_warp(tDV, tmem + C::p_col(kk), bdesc, C::kIdescGrad,
+                                (acc || kk > 0) ? 1u : 0u);
+                    if (PRECISE) mma_ts_warp(tDV, tmem + C::p_col(kk) + 32, bdesc, C::kIdescGrad, 1u);
+                }
             };
             // dQ_i = dS K: M = 128 queries (dS^T read MN-major), N = d, K = 128 keys
             auto dq_mma = [&](uint32_t a_addr, bool acc) {
@@ -613,30 +620,34 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 score_mma(tDP, v_addr, do_stage(0));
                 mma_commit_warp(&bars->dp_full);
             }
+            auto issue_s_next = [&](int n) -> bool {
+                if (!warp_wait(&bars->q_full[(n + 1) % C::kStagesQ], ((n + 1) / C::kStagesQ) & 1,
+                               kSiteQFull, abort))
+                    return false;
+                tc_fence_after();
+                score_mma(tS, k_addr, q_stage(n + 1));
+                mma_commit_warp(&bars->s_full);
+                return true;
+            };
             for (int n = 0; ok && n < n_iter; ++n) {
-                // S_{n+1} as soon as the compute warps hold S_n in registers
-                if (n + 1 < n_iter) {
+                // own P^T columns: S_{n+1} as soon as the compute warps hold S_n in
+                // registers
+                if (!C::kPAliasS && n + 1 < n_iter) {
                     if (!warp_wait(&bars->s_free, n & 1, kSiteSFree, abort)) { ok = false; break; }
-                    if (!warp_wait(&bars->q_full[(n + 1) % C::kStagesQ],
-                                   ((n + 1) / C::kStagesQ) & 1, kSiteQFull, abort)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    score_mma(tS, k_addr, q_stage(n + 1));
-                    mma_commit_warp(&bars->s_full);
+                    if (!issue_s_next(n)) { ok = false; break; }
                 }
                 // dV += P^T dO_n
                 if (!warp_wait(&bars->p_full, n & 1, kSitePFull, abort)) { ok = false; break; }
                 tc_fence_after();
-                if constexpr (C::kPInTmem) {
-                    dv_mma_tmem(do_stage(n), n > 0);
-                } else {
-                    grad_mma(tDV, p_addr, do_stage(n), n > 0);
-                    if (PRECISE) grad_mma(tDV, p_addr + C::kScoreBytes, do_stage(n), true);
-                }
+                dv_mma(do_stage(n), n > 0);
                 mma_commit_warp(&bars->p_free);
                 mma_commit_warp(&bars->do_empty[n % C::kStagesDO]);
+                // P^T over S^T: S_{n+1} once dV_n, which reads P^T there, has completed
+                // (waiting for the commit rather than relying on issue order)
+                if (C::kPAliasS && n + 1 < n_iter) {
+                    if (!warp_wait(&bars->p_free, n & 1, kSitePFree, abort)) { ok = false; break; }
+                    if (!issue_s_next(n)) { ok = false; break; }
+                }
                 // dK += dS^T Q_n ; dQ_n = dS K
                 if (!warp_wait(&bars->ds_full, n & 1, kSiteDSFull, abort)) { ok = false; break; }
                 tc_fence_after();
