@@ -54,8 +54,9 @@ def measured_peaks():
 
 
 def kernel_source_sha():
+    """Hash of the dK/dV kernel's sources (the kernel whose traffic is recorded)."""
     h = hashlib.sha256()
-    for name in ("attn_bwd.cu", "attn_fwd.cu", "sm100_ptx.cuh"):
+    for name in ("attn_bwd.cu", "sm100_ptx.cuh"):
         with open(os.path.join(ROOT, "causal_attention_fwd_attn_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
