@@ -62,6 +62,18 @@ namespace {
 __device__ __forceinline__ constexpr bool use_poly_pair(int e) { return (e & 3) == 3; }
 
 constexpr int kBwdThreads = 512;
+// registers per thread at launch: __launch_bounds__(512, 1) gives each thread 128
+constexpr uint32_t kLaunchRegs = 65536 / kBwdThreads;
+
+// Moves this warpgroup's register budget to N: setmaxnreg.inc above the launch
+// count, .dec below it (a .dec to a larger count, or an .inc to a smaller one, is
+// not a valid instruction).
+template <uint32_t N>
+__device__ __forceinline__ void set_warpgroup_regs() {
+    static_assert(N % 8 == 0 && N >= 24 && N <= 256, "setmaxnreg range");
+    if constexpr (N > kLaunchRegs) regs_inc<N>();
+    else if constexpr (N < kLaunchRegs) regs_dec<N>();
+}
 constexpr int kComputeWarps = 8;
 constexpr int kDrainWarps = 4;
 constexpr uint32_t kWarpCompute0 = 4, kWarpProducer = 12, kWarpMma = 13;
@@ -70,7 +82,7 @@ constexpr float kLog2e = 1.4426950408889634f;
 enum : uint32_t {
     kSiteKV = 1, kSiteQFull, kSiteDOFull, kSiteQEmpty, kSiteDOEmpty, kSiteSFull,
     kSiteSFree, kSiteDPFull, kSitePFull, kSitePFree, kSiteDSFull, kSiteDSFree, kSiteDQFull,
-    kSiteDQFree, kSiteAccDone, kSiteAlign, kSiteStageFree, kSiteStageFull
+    kSiteDQFree, kSiteAccDone, kSiteAlign, kSiteStageFree, kSiteStageFull, kSiteStageDone
 };
 
 template <int D, bool PRECISE>
@@ -78,32 +90,45 @@ struct BwdCfg {
     static constexpr int kChunks = D / 64;
     static constexpr int kChunkBytes = kTile * 128;        // 128 rows x 128 bytes
     static constexpr int kTileBytes = kChunks * kChunkBytes;
-    // dQ through shared memory and a TMA reduce where there is room (d = 64 default)
-    static constexpr bool kTmaDQ = (D == 64 && !PRECISE);
+    // dQ_n leaves tensor memory through 128-byte-swizzled fp32 staging in shared
+    // memory, 32-column slices at a time, and a TMA reduce-add.  Default mode: a
+    // staging buffer of its own (two slices; two rounds per step at d = 128).
+    // Precise mode has no room for it and stages through the dS^T buffer, which
+    // dQ_n's products have finished reading once dQ_n is complete (the compute warps
+    // then wait for the drain before writing the next dS^T).
+    static constexpr bool kStageOwn = !PRECISE;
     // P^T goes back into tensor memory (bf16 pairs) as the A operand of dV: into
     // columns of its own where 64 are left (d = 64 default), otherwise over the S^T
     // columns it was computed from (each 64-query half into the first 32 (hi) and
     // last 32 (lo, precise mode) of its own 64 columns), so the next S^T waits for dV.
     static constexpr bool kPAliasS = !(D == 64 && !PRECISE);
-    static constexpr int kStagesQ = kTmaDQ ? 3 : 2;
-    // Precise mode at d = 128 needs the room of one dO stage for the lo buffer.
-    static constexpr int kStagesDO = (D == 128 && PRECISE) ? 1 : 2;
+    static constexpr int kStagesQ = (D == 64 && !PRECISE) ? 3 : 2;
+    // d = 128 holds one dO stage: dO_{n+1} has from dV_n to dP_{n+1} (issued after
+    // dQ_n is drained) to arrive.
+    static constexpr int kStagesDO = D == 128 ? 1 : 2;
     // dS^T: [128 keys][128 queries] bf16 = two 64-query chunks; in precise mode a hi
     // buffer followed by a lo buffer.
     static constexpr int kScoreBytes = 2 * kChunkBytes;
     static constexpr int kSplit = PRECISE ? 2 : 1;
     // With d = 64 dQ_i has tensor-memory columns of its own.
     static constexpr bool kSeparateDQ = (D == 64);
-    // dQ staging for the TMA reduce: per column half, [128 rows][32 fp32] swizzled
-    static constexpr int kDQStageBytes = kTile * 32 * 4;
+    static constexpr int kDQStageBytes = kTile * 32 * 4;  // one slice: [128 rows][32 fp32]
+    static constexpr int kStageSlicesDS = kSplit * kScoreBytes / kDQStageBytes;
+    static constexpr int kStageSlices =  // per round
+        kStageOwn ? 2 : (kStageSlicesDS < D / 32 ? kStageSlicesDS : D / 32);
+    static constexpr int kDrainRounds = (D / 32) / kStageSlices;
+    static_assert(kDrainRounds * kStageSlices == D / 32, "dQ staging slices");
+    // slices moved out of tensor memory per load group: the last group's load frees
+    // the columns, before any wait for the staging
+    static constexpr int kLoadGroup = kStageOwn ? 2 : (kDrainRounds > 1 ? 2 : 1);
     static constexpr int kOffK = 0;
     static constexpr int kOffV = kOffK + kTileBytes;
     static constexpr int kOffQ = kOffV + kTileBytes;
     static constexpr int kOffDO = kOffQ + kStagesQ * kTileBytes;
     static constexpr int kOffDS = kOffDO + kStagesDO * kTileBytes;
     static constexpr int kOffDQS = kOffDS + kSplit * kScoreBytes;
-    static constexpr int kDQSlices = kTmaDQ ? D / 32 : 0;  // 32-column staging slices
-    static constexpr int kOffLse = kOffDQS + kDQSlices * kDQStageBytes;
+    static constexpr int kOffStage = kStageOwn ? kOffDQS : kOffDS;
+    static constexpr int kOffLse = kOffDQS + (kStageOwn ? kStageSlices * kDQStageBytes : 0);
     static constexpr int kOffDelta = kOffLse + kStagesQ * kTile * 4;
     static constexpr int kOffBar = kOffDelta + kStagesQ * kTile * 4;
     static constexpr int kSmemBytes = kOffBar + 256;
@@ -119,11 +144,12 @@ struct BwdCfg {
         return kPAliasS ? kColS + (kk >> 2) * 64 + (kk & 3) * 8 : kColP + kk * 8;
     }
     // registers per thread after setmaxnreg (the launch gives 512 x 128): the precise
-    // d = 128 MMA issuer needs more, its drain (64 columns at a time) less
+    // d = 128 MMA issuer needs more, its drain (one slice at a time) less
     static constexpr uint32_t kRegsDrain = (D == 128 && PRECISE) ? 80 : 96;
     static constexpr uint32_t kRegsCompute = 168;
     static constexpr uint32_t kRegsCtl = (D == 128 && PRECISE) ? 96 : 80;
-    static_assert(128 * kRegsDrain + 256 * kRegsCompute + 128 * kRegsCtl <= 65536,
+    static_assert(128 * kRegsDrain + 256 * kRegsCompute + 128 * kRegsCtl <=
+                      kBwdThreads * kLaunchRegs,
                   "register split exceeds the block's launch allocation");
     static constexpr uint32_t kIdescScore = idesc_bf16_f32(128, 128, false, false);
     static constexpr uint32_t kIdescGrad = idesc_bf16_f32(128, D, false, true);  // dV, dK
@@ -138,6 +164,7 @@ struct BwdBarriers {
     uint64_t do_empty[2];
     uint64_t s_full, s_free, dp_full, p_full, p_free, ds_full, ds_free, dq_full, dq_free;
     uint64_t stage_free, stage_full;  // dQ staging in shared memory (drain warps)
+    uint64_t stage_done;              // staging in the dS^T buffer is over (per step)
     uint64_t acc_done, mma_final;
     uint32_t tmem_base;
     int abort;
@@ -223,6 +250,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         mbar_init(&bars->dq_free, kDrainWarps);
         mbar_init(&bars->stage_free, 1);
         mbar_init(&bars->stage_full, kDrainWarps);
+        mbar_init(&bars->stage_done, 1);
         mbar_init(&bars->acc_done, 1);
         mbar_init(&bars->mma_final, 1);
         bars->abort = (smem_u32(smem) & 1023u) ? 1 : 0;
@@ -240,84 +268,92 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
     if (warp < kWarpCompute0) {
         // ---------------------------------------------------------- dQ drain
-        regs_dec<C::kRegsDrain>();
+        set_warpgroup_regs<C::kRegsDrain>();
         const uint32_t row = (warp << 5) + lane;  // query row of the tile
         const uint32_t lane_off = (warp << 5) << 16;
         const bool leader = warp == 0 && lane == 0;
+        int n_sfree = 0, n_sfull = 0;  // completed phases of the staging barriers
         for (int m = 0; m < n_iter; ++m) {
             if (!warp_wait(&bars->dq_full, m & 1, kSiteDQFull, abort)) break;
             tc_fence_after();
             const int i = i_begin + m;
-            if constexpr (C::kTmaDQ) {
-                uint32_t r[D];
+            bool fine = true;
+            constexpr int kG = C::kLoadGroup;
+            constexpr int kGroups = D / 32 / kG;
+            constexpr int kGroupsPerRound = C::kStageSlices / kG;
 #pragma unroll
-                for (int c = 0; c < D / 32; ++c)
-                    tmem_ld32(tmem + lane_off + C::kColDQ + c * 32, r + c * 32);
+            for (int pr = 0; pr < kGroups; ++pr) {
+                const int rd = pr / kGroupsPerRound, sl0 = kG * (pr % kGroupsPerRound);
+                uint32_t r[32 * kG];
+#pragma unroll
+                for (int h = 0; h < kG; ++h)
+                    tmem_ld32(tmem + lane_off + C::kColDQ + 32 * (kG * pr + h), r + 32 * h);
                 tmem_wait_ld();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&bars->dq_free);
-                // the staging slices must have been read by the previous reduce (bounded
-                // mbarrier waits rather than bar.sync, so an abort cannot strand a warp)
+                if (pr == kGroups - 1) {  // every column of dQ_n has been read
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&bars->dq_free);
+                }
+                // a round's staging must have been read by the previous round's reduce
+                // (the dS^T buffer is free at the first round of a step by construction);
+                // bounded mbarrier waits rather than bar.sync, so an abort strands no warp
+                if (sl0 == 0 && (C::kStageOwn || rd > 0)) {
+                    if (leader) {
+                        tma_store_wait_all_read();
+                        mbar_arrive(&bars->stage_free);
+                    }
+                    if (!warp_wait(&bars->stage_free, n_sfree & 1, kSiteStageFree, abort)) {
+                        fine = false;
+                        break;
+                    }
+                    ++n_sfree;
+                }
+#pragma unroll
+                for (int h = 0; h < kG; ++h) {
+                    uint8_t* stage = smem + C::kOffStage + (sl0 + h) * C::kDQStageBytes;
+#pragma unroll
+                    for (int ch = 0; ch < 8; ++ch)
+                        *reinterpret_cast<float4*>(stage + sw128_offset(row, ch)) = make_float4(
+                            __uint_as_float(r[32 * h + 4 * ch]) * scale,
+                            __uint_as_float(r[32 * h + 4 * ch + 1]) * scale,
+                            __uint_as_float(r[32 * h + 4 * ch + 2]) * scale,
+                            __uint_as_float(r[32 * h + 4 * ch + 3]) * scale);
+                }
+                if (sl0 + kG == C::kStageSlices) {  // the round's slices are staged
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&bars->stage_full);
+                    if (warp == 0) {
+                        if (!warp_wait(&bars->stage_full, n_sfull & 1, kSiteStageFull, abort)) {
+                            fine = false;
+                            break;
+                        }
+                        if (leader) {
+#pragma unroll
+                            for (int sl = 0; sl < C::kStageSlices; ++sl)
+                                tma_reduce_add_3d(&tmap_dq,
+                                                  smem + C::kOffStage + sl * C::kDQStageBytes,
+                                                  (rd * C::kStageSlices + sl) * 32, i * kTile, bh);
+                            tma_store_commit();
+                        }
+                    }
+                    ++n_sfull;
+                }
+            }
+            if (!fine) break;
+            if constexpr (!C::kStageOwn) {
+                // the dS^T buffer goes back to the compute warps once the reduces have
+                // read it
                 if (leader) {
                     tma_store_wait_all_read();
-                    mbar_arrive(&bars->stage_free);
-                }
-                if (!warp_wait(&bars->stage_free, m & 1, kSiteStageFree, abort)) break;
-#pragma unroll
-                for (int sl = 0; sl < C::kDQSlices; ++sl) {
-                    uint8_t* stage = smem + C::kOffDQS + sl * C::kDQStageBytes;
-#pragma unroll
-                    for (int ch = 0; ch < 8; ++ch) {
-                        const uint32_t* x = r + sl * 32 + 4 * ch;
-                        *reinterpret_cast<float4*>(stage + sw128_offset(row, ch)) =
-                            make_float4(__uint_as_float(x[0]) * scale, __uint_as_float(x[1]) * scale,
-                                        __uint_as_float(x[2]) * scale, __uint_as_float(x[3]) * scale);
-                    }
-                }
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&bars->stage_full);
-                if (warp == 0) {
-                    if (!warp_wait(&bars->stage_full, m & 1, kSiteStageFull, abort)) break;
-                    if (leader) {
-#pragma unroll
-                        for (int sl = 0; sl < C::kDQSlices; ++sl)
-                            tma_reduce_add_3d(&tmap_dq, smem + C::kOffDQS + sl * C::kDQStageBytes,
-                                              32 * sl, i * kTile, bh);
-                        tma_store_commit();
-                    }
-                }
-            } else {
-                // 64 columns at a time; the columns are released after the last load
-                const int q = i * kTile + (int)row;
-                float* dst = dq_accum + ((size_t)bh * T + q) * D;
-#pragma unroll
-                for (int c = 0; c < D / 64; ++c) {
-                    uint32_t r[64];
-                    tmem_ld32(tmem + lane_off + C::kColDQ + c * 64, r);
-                    tmem_ld32(tmem + lane_off + C::kColDQ + c * 64 + 32, r + 32);
-                    tmem_wait_ld();
-                    if (c == D / 64 - 1) {
-                        tc_fence_before();
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(&bars->dq_free);
-                    }
-                    if (q < T) {
-#pragma unroll
-                        for (int e = 0; e < 16; ++e)
-                            red_add_v4(dst + c * 64 + 4 * e, __uint_as_float(r[4 * e]) * scale,
-                                       __uint_as_float(r[4 * e + 1]) * scale,
-                                       __uint_as_float(r[4 * e + 2]) * scale,
-                                       __uint_as_float(r[4 * e + 3]) * scale);
-                    }
+                    mbar_arrive(&bars->stage_done);
                 }
             }
         }
-        if (C::kTmaDQ && leader) tma_store_wait_all();  // reduces done before the CTA exits
+        if (leader) tma_store_wait_all();  // reduces done before the CTA exits
     } else if (warp < kWarpProducer) {
         // ----------------------------------------------------------- compute
-        regs_inc<C::kRegsCompute>();
+        set_warpgroup_regs<C::kRegsCompute>();
         const uint32_t quarter = warp & 3;
         const uint32_t half = (warp - kWarpCompute0) >> 2;  // which 64 query columns
         const uint32_t row = (quarter << 5) + lane;          // key row
@@ -411,7 +447,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             // ---- dS^T = P^T o (dP^T - D), 32 queries at a time
             if (!warp_wait(&bars->dp_full, n & 1, kSiteDPFull, abort)) { ok = false; break; }
             // dS^T buffer: free once dK and dQ of the previous iteration have read it
-            if (n > 0 && !warp_wait(&bars->ds_free, (n - 1) & 1, kSiteDSFree, abort)) {
+            // and, where it stages dQ, once the drain is done with it
+            constexpr bool kStaged = !C::kStageOwn;
+            if (n > 0 && !warp_wait(kStaged ? &bars->stage_done : &bars->ds_free, (n - 1) & 1,
+                                    kStaged ? kSiteStageDone : kSiteDSFree, abort)) {
                 ok = false;
                 break;
             }
@@ -494,7 +533,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             }
         }
     } else {
-        regs_dec<C::kRegsCtl>();
+        set_warpgroup_regs<C::kRegsCtl>();
         if (warp == kWarpProducer && lane == 0) {
             // -------------------------------------------------------- producer
             int last_q[3] = {-1, -1, -1}, last_do[2] = {-1, -1};
