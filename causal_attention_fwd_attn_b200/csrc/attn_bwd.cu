@@ -12,45 +12,46 @@
 //                        padded per head to a whole number of 128-row tiles (D = 0,
 //                        -LSE = -inf past T, so those queries get P ~ 0), and the fp32
 //                        dQ accumulator cleared.  Memory-bound.
-//   attn_bwd_dkdv        one CTA per (head, 128-key tile j), looping over the query
-//                        tiles i that see it (i >= j under the causal mask):
+//   attn_bwd_dkdv        persistent CTAs (one per SM) walking (head, 128-key tile j)
+//                        items heaviest first; per item, a loop over the query tiles i
+//                        that see the key tile (i >= j under the causal mask):
 //                          S^T  = K_j Q_i^T           (tcgen05, TMEM)
 //                          dP^T = V_j dO_i^T          (tcgen05, TMEM)
 //                          P^T  = exp2(S^T*scale*log2e - LSE_i*log2e)   (threads)
 //                          dS^T = P^T o (dP^T - D_i)                     (threads)
 //                          dV  += P^T dO_i ;  dK += dS^T Q_i             (tcgen05, TMEM)
 //                          dQ_i = dS K_j  (tcgen05 with dS^T read MN-major), then
-//                                 scale * dQ_i added to the fp32 accumulator: staged
-//                                 in shared memory and added by TMA reduce-add
-//                                 (d = 64), or with red.global.add.v4.f32 (d = 128 and
-//                                 precise mode, whose shared memory is full).
+//                                 scale * dQ_i staged in shared memory and added to
+//                                 the fp32 accumulator by TMA reduce-add.
 //                        The dQ stage of the paper is fused here: its partial sums
 //                        come out of the same recomputation, and reductions in L2
-//                        replace the paper's second pass over the scores.
+//                        replace the paper's second pass over the scores.  The steps
+//                        of consecutive items form one pipeline: the next item's first
+//                        products are issued while this item's dK/dV leave TMEM.
 //   attn_bwd_dq_convert  dQ = bf16(accumulator).
 //
-// dkdv warp roles (512 threads, four warpgroups; setmaxnreg moves registers from the
-// drain and control warpgroups to the two compute warpgroups):
-//   warps 0..3   dQ drain: warp w owns TMEM lanes 32w.. (query rows of dQ_i) and all d
-//                columns; it moves dQ_i out of tensor memory, scales it and adds it to
-//                the fp32 accumulator (TMA reduce-add from shared memory, or
-//                red.global.add.v4.f32), off the compute warps' path.
+// dkdv warp roles (512 threads, four warpgroups; setmaxnreg moves registers between
+// them):
+//   warps 0..3   dQ drain and epilogue: warp w owns TMEM lanes 32w.. (query rows of
+//                dQ_i, key rows of dK/dV) and all d columns; it moves dQ_i out of
+//                tensor memory into fp32 staging and TMA reduce-adds it into the
+//                accumulator, and at the end of an item stores dK and dV, off the
+//                compute warps' path.
 //   warps 4..11  compute: warp w owns TMEM lanes 32*(w%4).. (key rows of the tile) and
 //                half h = (w-4)/4 of the 128 query columns.  Each thread forms its 64
-//                P^T values and writes them bf16 either into tensor memory (d = 64:
-//                the A operand of dV) or into 128-byte-swizzled shared memory, then
-//                its 64 dS^T values into shared memory (the A operand of dK, and the
-//                MN-major A operand of dQ), and stores its half of the dK/dV columns
-//                at the end.
-//   warp 12      producer (one thread): K_j, V_j once; Q_i, dO_i by TMA into staged
-//                rings; the LSE_i and D_i vectors (128 floats each) by 1-D bulk copies
-//                from the padded row statistics, counted on Q_i's barrier.
-//   warp 13      MMA issuer (one thread); allocates tensor memory.
+//                P^T values and writes them bf16 into tensor memory (the A operand of
+//                dV), then its 64 dS^T values into shared memory (the A operand of
+//                dK, and the MN-major A operand of dQ).
+//   warp 12      producer (one thread): K_j, V_j per item; Q_i, dO_i by TMA into
+//                staged rings; the LSE_i and D_i vectors (128 floats each) by 1-D bulk
+//                copies from the padded row statistics, counted on Q_i's barrier.
+//   warp 13      MMA issuer (converged warp, one elected lane issues); allocates
+//                tensor memory.
 //   warps 14,15  idle (they complete the control warpgroup for setmaxnreg).
 // Tensor memory: dV [0,d) | dK [d,2d) | S^T [2d,2d+128) | dP^T [2d+128,2d+256) |
 //   dQ_i [2d+256, 3d+256) and P^T as bf16 pairs [3d+256, 3d+320) for d = 64; for
-//   d = 128 dQ_i reuses the dP^T columns once dS^T has been formed (512 columns hold
-//   no more) and P^T stays in shared memory.
+//   d = 128 (and precise mode) P^T is written over the S^T columns and dQ_i reuses
+//   the dP^T columns once dS^T has been formed (512 columns hold no more).
 #include "forge_internal.h"
 #include "sm100_ptx.cuh"
 
@@ -82,7 +83,8 @@ constexpr float kLog2e = 1.4426950408889634f;
 enum : uint32_t {
     kSiteKV = 1, kSiteQFull, kSiteDOFull, kSiteQEmpty, kSiteDOEmpty, kSiteSFull,
     kSiteSFree, kSiteDPFull, kSitePFull, kSitePFree, kSiteDSFull, kSiteDSFree, kSiteDQFull,
-    kSiteDQFree, kSiteAccDone, kSiteAlign, kSiteStageFree, kSiteStageFull, kSiteStageDone
+    kSiteDQFree, kSiteAccDone, kSiteAlign, kSiteStageFree, kSiteStageFull, kSiteStageDone, kSiteKVEmpty,
+    kSiteAccFree
 };
 
 template <int D, bool PRECISE>
@@ -121,9 +123,13 @@ struct BwdCfg {
     // slices moved out of tensor memory per load group: the last group's load frees
     // the columns, before any wait for the staging
     static constexpr int kLoadGroup = kStageOwn ? 2 : (kDrainRounds > 1 ? 2 : 1);
+    // K/V buffers.  One: the next item's K_j, V_j load after this item's last dQ,
+    // and its first S^T waits for them.  (Two buffers at d = 64 measured slower: the
+    // extra 32 KB of shared memory cost more than the overlap gained.)
+    static constexpr int kKVBufs = 1;
     static constexpr int kOffK = 0;
-    static constexpr int kOffV = kOffK + kTileBytes;
-    static constexpr int kOffQ = kOffV + kTileBytes;
+    static constexpr int kOffV = kOffK + kKVBufs * kTileBytes;
+    static constexpr int kOffQ = kOffV + kKVBufs * kTileBytes;
     static constexpr int kOffDO = kOffQ + kStagesQ * kTileBytes;
     static constexpr int kOffDS = kOffDO + kStagesDO * kTileBytes;
     static constexpr int kOffDQS = kOffDS + kSplit * kScoreBytes;
@@ -157,7 +163,7 @@ struct BwdCfg {
 };
 
 struct BwdBarriers {
-    uint64_t kv_full;
+    uint64_t kv_full[2], kv_empty[2];  // K_j, V_j per item (one or two buffers)
     uint64_t q_full[3];
     uint64_t do_full[2];
     uint64_t q_empty[3];
@@ -165,7 +171,8 @@ struct BwdBarriers {
     uint64_t s_full, s_free, dp_full, p_full, p_free, ds_full, ds_free, dq_full, dq_free;
     uint64_t stage_free, stage_full;  // dQ staging in shared memory (drain warps)
     uint64_t stage_done;              // staging in the dS^T buffer is over (per step)
-    uint64_t acc_done, mma_final;
+    uint64_t acc_done, acc_free;  // an item's dK, dV complete / read out of tensor memory
+    uint64_t mma_final;
     uint32_t tmem_base;
     int abort;
 };
@@ -196,13 +203,6 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, uint32
     return __all_sync(0xffffffffu, mbar_wait(bar, parity, site, abort));
 }
 
-// Fire-and-forget fp32 vector reduction into global memory (no value returned).
-__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
-    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b),
-                 "f"(c), "f"(d)
-                 : "memory");
-}
-
 template <int D, bool PRECISE>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmap_q,
@@ -212,7 +212,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                          const __grid_constant__ CUtensorMap tmap_dq,
                          const float* __restrict__ rowstats, float* __restrict__ dq_accum,
                          void* __restrict__ dk_out, void* __restrict__ dv_out, int T, int BH,
-                         int n_kvtiles, float scale, float scale_log2, int causal, int grad_f32) {
+                         int n_kvtiles, int n_items, float scale, float scale_log2, int causal,
+                         int grad_f32) {
     using C = BwdCfg<D, PRECISE>;
     extern __shared__ __align__(1024) uint8_t smem[];
     BwdBarriers* bars = reinterpret_cast<BwdBarriers*>(smem + C::kOffBar);
@@ -220,17 +221,31 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     float* s_lse = reinterpret_cast<float*>(smem + C::kOffLse);
     float* s_delta = reinterpret_cast<float*>(smem + C::kOffDelta);
 
-    const int bh = blockIdx.x;
-    const int kt = blockIdx.y;  // key tile: tile 0 sees the most query tiles, so it goes first
     const int n_qtiles = n_kvtiles;
     const int t_pad = n_qtiles * kTile;  // row-statistics stride per head
-    const int i_begin = causal ? kt : 0;
-    const int n_iter = n_qtiles - i_begin;
+    const int n_ctas = (int)gridDim.x;
+    // Persistent CTAs.  The CTA's r-th work item is a (head, key tile) pair; items are
+    // numbered heaviest first (key tile 0 sees the most query tiles) and dealt in a
+    // zigzag over the CTAs, which keeps every CTA's total close to the mean.  Every
+    // role walks the same item sequence; the per-step barriers count steps across
+    // items, so one item's last steps overlap the next item's first.
+    auto item_of = [&](int r, int& bh_out, int& kt_out) -> bool {
+        const int k = r * n_ctas + ((r & 1) ? (n_ctas - 1 - (int)blockIdx.x) : (int)blockIdx.x);
+        if (k >= n_items) return false;
+        kt_out = k / BH;
+        bh_out = k - kt_out * BH;
+        return true;
+    };
+    auto first_qtile = [&](int kt_) { return causal ? kt_ : 0; };
     const uint32_t warp = warp_id();
     const uint32_t lane = lane_id();
 
     if (threadIdx.x == 0) {
-        mbar_init(&bars->kv_full, 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&bars->kv_full[s], 1);
+            mbar_init(&bars->kv_empty[s], 1);
+        }
+        mbar_init(&bars->acc_free, kDrainWarps);
         for (int s = 0; s < 3; ++s) {
             mbar_init(&bars->q_full[s], 1);
             mbar_init(&bars->q_empty[s], 1);
@@ -273,10 +288,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const uint32_t lane_off = (warp << 5) << 16;
         const bool leader = warp == 0 && lane == 0;
         int n_sfree = 0, n_sfull = 0;  // completed phases of the staging barriers
-        for (int m = 0; m < n_iter; ++m) {
-            if (!warp_wait(&bars->dq_full, m & 1, kSiteDQFull, abort)) break;
+        int g = 0;                     // steps drained so far (all items)
+        bool run = true;
+        int bh, kt;
+        for (int item = 0; run && item_of(item, bh, kt); ++item) {
+        for (int i = first_qtile(kt); i < n_qtiles; ++i, ++g) {
+            if (!warp_wait(&bars->dq_full, g & 1, kSiteDQFull, abort)) { run = false; break; }
             tc_fence_after();
-            const int i = i_begin + m;
             bool fine = true;
             constexpr int kG = C::kLoadGroup;
             constexpr int kGroups = D / 32 / kG;
@@ -340,7 +358,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     ++n_sfull;
                 }
             }
-            if (!fine) break;
+            if (!fine) { run = false; break; }
             if constexpr (!C::kStageOwn) {
                 // the dS^T buffer goes back to the compute warps once the reduces have
                 // read it
@@ -350,7 +368,63 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 }
             }
         }
-        if (leader) tma_store_wait_all();  // reduces done before the CTA exits
+        if (!run) break;
+        // ------------------------------------------------ dK / dV epilogue
+        // the item's dV, dK leave tensor memory here, while the compute warps go on
+        // with the next item; its first dV, dK products wait for acc_free
+        if (!warp_wait(&bars->acc_done, item & 1, kSiteAccDone, abort)) break;
+        tc_fence_after();
+        {
+            const int key = kt * kTile + (int)row;
+            const size_t base = ((size_t)bh * T + key) * D;
+#pragma unroll
+            for (int which = 0; which < 2; ++which) {
+                const uint32_t col = which == 0 ? C::kColDV : C::kColDK;
+                const float mul = which == 0 ? 1.f : scale;
+                void* out = which == 0 ? dv_out : dk_out;
+#pragma unroll
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t r[32];
+                    tmem_ld32(tmem + lane_off + col + c * 32, r);
+                    tmem_wait_ld();
+                    if (which == 1 && c == D / 32 - 1) {
+                        // every column of dV and dK has been read
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&bars->acc_free);
+                    }
+                    if (key < T) {
+                        if (grad_f32) {
+                            float4* o =
+                                reinterpret_cast<float4*>(reinterpret_cast<float*>(out) + base + c * 32);
+#pragma unroll
+                            for (int e = 0; e < 8; ++e)
+                                o[e] = make_float4(__uint_as_float(r[4 * e]) * mul,
+                                                   __uint_as_float(r[4 * e + 1]) * mul,
+                                                   __uint_as_float(r[4 * e + 2]) * mul,
+                                                   __uint_as_float(r[4 * e + 3]) * mul);
+                        } else {
+                            uint4* o = reinterpret_cast<uint4*>(
+                                reinterpret_cast<__nv_bfloat16*>(out) + base + c * 32);
+#pragma unroll
+                            for (int e = 0; e < 4; ++e)
+                                o[e] = make_uint4(pack_bf16x2(__uint_as_float(r[8 * e]) * mul,
+                                                              __uint_as_float(r[8 * e + 1]) * mul),
+                                                  pack_bf16x2(__uint_as_float(r[8 * e + 2]) * mul,
+                                                              __uint_as_float(r[8 * e + 3]) * mul),
+                                                  pack_bf16x2(__uint_as_float(r[8 * e + 4]) * mul,
+                                                              __uint_as_float(r[8 * e + 5]) * mul),
+                                                  pack_bf16x2(__uint_as_float(r[8 * e + 6]) * mul,
+                                                              __uint_as_float(r[8 * e + 7]) * mul));
+                        }
+                    }
+                }
+            }
+        }
+        }  // items
+        // the reduces must have read their staging before the CTA's shared memory goes;
+        // their global writes complete before the kernel does
+        if (leader) tma_store_wait_all_read();
     } else if (warp < kWarpProducer) {
         // ----------------------------------------------------------- compute
         set_warpgroup_regs<C::kRegsCompute>();
@@ -361,13 +435,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         uint8_t* ds_smem = smem + C::kOffDS + half * C::kChunkBytes;
         const int c0 = half * 64;                            // first query column owned
         bool ok = !*abort;
-
-        for (int n = 0; ok && n < n_iter; ++n) {
-            const int sq = n % C::kStagesQ;
-            const int i = i_begin + n;
+        int g = 0;  // steps so far (all items)
+        int bh, kt;
+        for (int item = 0; ok && item_of(item, bh, kt); ++item) {
+        for (int i = first_qtile(kt); ok && i < n_qtiles; ++i, ++g) {
+            const int sq = g % C::kStagesQ;
             const bool diag = causal && (i == kt);
             // ---- P^T for 64 query columns
-            if (!warp_wait(&bars->s_full, n & 1, kSiteSFull, abort)) { ok = false; break; }
+            if (!warp_wait(&bars->s_full, g & 1, kSiteSFull, abort)) { ok = false; break; }
             tc_fence_after();
             uint32_t sraw[64];
             tmem_ld32(tmem + lane_off + C::kColS + c0, sraw);
@@ -380,7 +455,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 if (lane == 0) mbar_arrive(&bars->s_free);
             }
             // LSE_i and D_i arrived with Q_i
-            if (!warp_wait(&bars->q_full[sq], (n / C::kStagesQ) & 1, kSiteQFull, abort)) {
+            if (!warp_wait(&bars->q_full[sq], (g / C::kStagesQ) & 1, kSiteQFull, abort)) {
                 ok = false;
                 break;
             }
@@ -416,8 +491,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             // P^T into tensor memory.  Own columns: they must no longer be read by the
             // previous iteration's dV.  Over S^T: this thread has read its S^T columns,
             // and S_n was issued after dV_{n-1}.
-            if (!C::kPAliasS && n > 0 &&
-                !warp_wait(&bars->p_free, (n - 1) & 1, kSitePFree, abort)) {
+            if (!C::kPAliasS && g > 0 &&
+                !warp_wait(&bars->p_free, (g - 1) & 1, kSitePFree, abort)) {
                 ok = false;
                 break;
             }
@@ -445,11 +520,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             if (lane == 0) mbar_arrive(&bars->p_full);
 
             // ---- dS^T = P^T o (dP^T - D), 32 queries at a time
-            if (!warp_wait(&bars->dp_full, n & 1, kSiteDPFull, abort)) { ok = false; break; }
+            if (!warp_wait(&bars->dp_full, g & 1, kSiteDPFull, abort)) { ok = false; break; }
             // dS^T buffer: free once dK and dQ of the previous iteration have read it
             // and, where it stages dQ, once the drain is done with it
             constexpr bool kStaged = !C::kStageOwn;
-            if (n > 0 && !warp_wait(kStaged ? &bars->stage_done : &bars->ds_free, (n - 1) & 1,
+            if (g > 0 && !warp_wait(kStaged ? &bars->stage_done : &bars->ds_free, (g - 1) & 1,
                                     kStaged ? kSiteStageDone : kSiteDSFree, abort)) {
                 ok = false;
                 break;
@@ -470,13 +545,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const int qc = c * 32 + ch * 8 + 2 * e;
-                        const float2 g = fmul2(
+                        const float2 dsv = fmul2(
                             make_float2(p[qc], p[qc + 1]),
                             fsub2(make_float2(__uint_as_float(dp[ch * 8 + 2 * e]),
                                               __uint_as_float(dp[ch * 8 + 2 * e + 1])),
                                   dv2[e]));
-                        ds[2 * e] = g.x;
-                        ds[2 * e + 1] = g.y;
+                        ds[2 * e] = dsv.x;
+                        ds[2 * e + 1] = dsv.y;
                     }
                     store_split8<PRECISE>(ds_smem, C::kScoreBytes, sw128_offset(row, c * 4 + ch),
                                           ds);
@@ -488,100 +563,73 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             if (lane == 0) mbar_arrive(&bars->ds_full);
         }
 
-        // ------------------------------------------------ dK / dV epilogue
-        if (ok && warp_wait(&bars->acc_done, 0, kSiteAccDone, abort)) {
-            tc_fence_after();
-            const int key = kt * kTile + (int)row;
-            const size_t base = ((size_t)bh * T + key) * D + half * (D / 2);
-#pragma unroll
-            for (int which = 0; which < 2; ++which) {
-                const uint32_t col = (which == 0 ? C::kColDV : C::kColDK) + half * (D / 2);
-                const float mul = which == 0 ? 1.f : scale;
-                void* out = which == 0 ? dv_out : dk_out;
-#pragma unroll
-                for (int c = 0; c < D / 64; ++c) {
-                    uint32_t r[32];
-                    tmem_ld32(tmem + lane_off + col + c * 32, r);
-                    tmem_wait_ld();
-                    if (key < T) {
-                        if (grad_f32) {
-                            float* o = reinterpret_cast<float*>(out) + base + c * 32;
-#pragma unroll
-                            for (int e = 0; e < 8; ++e)
-                                reinterpret_cast<float4*>(o)[e] = make_float4(
-                                    __uint_as_float(r[4 * e]) * mul,
-                                    __uint_as_float(r[4 * e + 1]) * mul,
-                                    __uint_as_float(r[4 * e + 2]) * mul,
-                                    __uint_as_float(r[4 * e + 3]) * mul);
-                        } else {
-                            uint4* o = reinterpret_cast<uint4*>(
-                                reinterpret_cast<__nv_bfloat16*>(out) + base + c * 32);
-#pragma unroll
-                            for (int e = 0; e < 4; ++e)
-                                o[e] = make_uint4(
-                                    pack_bf16x2(__uint_as_float(r[8 * e]) * mul,
-                                                __uint_as_float(r[8 * e + 1]) * mul),
-                                    pack_bf16x2(__uint_as_float(r[8 * e + 2]) * mul,
-                                                __uint_as_float(r[8 * e + 3]) * mul),
-                                    pack_bf16x2(__uint_as_float(r[8 * e + 4]) * mul,
-                                                __uint_as_float(r[8 * e + 5]) * mul),
-                                    pack_bf16x2(__uint_as_float(r[8 * e + 6]) * mul,
-                                                __uint_as_float(r[8 * e + 7]) * mul));
-                        }
-                    }
-                }
-            }
-        }
+        }  // items
     } else {
         set_warpgroup_regs<C::kRegsCtl>();
         if (warp == kWarpProducer && lane == 0) {
             // -------------------------------------------------------- producer
-            int last_q[3] = {-1, -1, -1}, last_do[2] = {-1, -1};
-            bool kv_issued = false;
+            int last_q[3] = {-1, -1, -1}, last_do[2] = {-1, -1}, last_kv[2] = {-1, -1};
             if (!*abort) {
                 tma_prefetch_desc(&tmap_q);
                 tma_prefetch_desc(&tmap_k);
                 tma_prefetch_desc(&tmap_v);
                 tma_prefetch_desc(&tmap_do);
-                mbar_arrive_expect_tx(&bars->kv_full, 2 * C::kTileBytes);
-                for (int c = 0; c < C::kChunks; ++c) {
-                    tma_load_3d(smem + C::kOffK + c * C::kChunkBytes, &tmap_k, &bars->kv_full,
-                                64 * c, kt * kTile, bh);
-                    tma_load_3d(smem + C::kOffV + c * C::kChunkBytes, &tmap_v, &bars->kv_full,
-                                64 * c, kt * kTile, bh);
-                }
-                kv_issued = true;
-                const float* lse2_head = rowstats + (size_t)bh * t_pad;
-                const float* delta_head = rowstats + (size_t)BH * t_pad + (size_t)bh * t_pad;
-                for (int n = 0; n < n_iter; ++n) {
-                    const int i = i_begin + n;
-                    // Q_n with the LSE and D vectors of its query tile
-                    const int sq = n % C::kStagesQ, uq = n / C::kStagesQ;
-                    if (uq > 0 && !mbar_wait(&bars->q_empty[sq], (uq - 1) & 1, kSiteQEmpty, abort))
+                int g = 0;  // steps so far (all items)
+                bool run = true;
+                int bh, kt;
+                for (int item = 0; run && item_of(item, bh, kt); ++item) {
+                    // K_j, V_j into the item's buffer once the item before last is done
+                    // with it
+                    const int kb = item % C::kKVBufs, ukv = item / C::kKVBufs;
+                    if (ukv > 0 &&
+                        !mbar_wait(&bars->kv_empty[kb], (ukv - 1) & 1, kSiteKVEmpty, abort))
                         break;
-                    mbar_arrive_expect_tx(&bars->q_full[sq], C::kTileBytes + 2 * kTile * 4);
-                    for (int c = 0; c < C::kChunks; ++c)
-                        tma_load_3d(smem + C::kOffQ + sq * C::kTileBytes + c * C::kChunkBytes,
-                                    &tmap_q, &bars->q_full[sq], 64 * c, i * kTile, bh);
-                    bulk_load(s_lse + sq * kTile, lse2_head + i * kTile, kTile * 4,
-                              &bars->q_full[sq]);
-                    bulk_load(s_delta + sq * kTile, delta_head + i * kTile, kTile * 4,
-                              &bars->q_full[sq]);
-                    last_q[sq] = uq;
-                    // dO_n
-                    const int sd = n % C::kStagesDO, ud = n / C::kStagesDO;
-                    if (ud > 0 &&
-                        !mbar_wait(&bars->do_empty[sd], (ud - 1) & 1, kSiteDOEmpty, abort))
-                        break;
-                    mbar_arrive_expect_tx(&bars->do_full[sd], C::kTileBytes);
-                    for (int c = 0; c < C::kChunks; ++c)
-                        tma_load_3d(smem + C::kOffDO + sd * C::kTileBytes + c * C::kChunkBytes,
-                                    &tmap_do, &bars->do_full[sd], 64 * c, i * kTile, bh);
-                    last_do[sd] = ud;
+                    mbar_arrive_expect_tx(&bars->kv_full[kb], 2 * C::kTileBytes);
+                    for (int c = 0; c < C::kChunks; ++c) {
+                        tma_load_3d(smem + C::kOffK + kb * C::kTileBytes + c * C::kChunkBytes,
+                                    &tmap_k, &bars->kv_full[kb], 64 * c, kt * kTile, bh);
+                        tma_load_3d(smem + C::kOffV + kb * C::kTileBytes + c * C::kChunkBytes,
+                                    &tmap_v, &bars->kv_full[kb], 64 * c, kt * kTile, bh);
+                    }
+                    last_kv[kb] = ukv;
+                    const float* lse2_head = rowstats + (size_t)bh * t_pad;
+                    const float* delta_head = rowstats + (size_t)BH * t_pad + (size_t)bh * t_pad;
+                    for (int i = first_qtile(kt); i < n_qtiles; ++i, ++g) {
+                        // Q_i with the LSE and D vectors of its query tile
+                        const int sq = g % C::kStagesQ, uq = g / C::kStagesQ;
+                        if (uq > 0 &&
+                            !mbar_wait(&bars->q_empty[sq], (uq - 1) & 1, kSiteQEmpty, abort)) {
+                            run = false;
+                            break;
+                        }
+                        mbar_arrive_expect_tx(&bars->q_full[sq], C::kTileBytes + 2 * kTile * 4);
+                        for (int c = 0; c < C::kChunks; ++c)
+                            tma_load_3d(smem + C::kOffQ + sq * C::kTileBytes + c * C::kChunkBytes,
+                                        &tmap_q, &bars->q_full[sq], 64 * c, i * kTile, bh);
+                        bulk_load(s_lse + sq * kTile, lse2_head + i * kTile, kTile * 4,
+                                  &bars->q_full[sq]);
+                        bulk_load(s_delta + sq * kTile, delta_head + i * kTile, kTile * 4,
+                                  &bars->q_full[sq]);
+                        last_q[sq] = uq;
+                        // dO_i
+                        const int sd = g % C::kStagesDO, ud = g / C::kStagesDO;
+                        if (ud > 0 &&
+                            !mbar_wait(&bars->do_empty[sd], (ud - 1) & 1, kSiteDOEmpty, abort)) {
+                            run = false;
+                            break;
+                        }
+                        mbar_arrive_expect_tx(&bars->do_full[sd], C::kTileBytes);
+                        for (int c = 0; c < C::kChunks; ++c)
+                            tma_load_3d(smem + C::kOffDO + sd * C::kTileBytes + c * C::kChunkBytes,
+                                        &tmap_do, &bars->do_full[sd], 64 * c, i * kTile, bh);
+                        last_do[sd] = ud;
+                    }
                 }
             }
             if (*abort) {
-                if (kv_issued) mbar_wait_drain(&bars->kv_full, 0);
+                // let copies already issued land before the CTA's memory is released
+                for (int s = 0; s < 2; ++s)
+                    if (last_kv[s] >= 0) mbar_wait_drain(&bars->kv_full[s], last_kv[s] & 1);
                 for (int s = 0; s < 3; ++s)
                     if (last_q[s] >= 0) mbar_wait_drain(&bars->q_full[s], last_q[s] & 1);
                 for (int s = 0; s < 2; ++s)
@@ -595,11 +643,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             const uint32_t tDQ = tmem + C::kColDQ;
             const uint32_t tDV = tmem + C::kColDV;
             const uint32_t tDK = tmem + C::kColDK;
-            const uint32_t k_addr = smem_u32(smem + C::kOffK);
-            const uint32_t v_addr = smem_u32(smem + C::kOffV);
+            auto k_buf = [&](int b) { return smem_u32(smem + C::kOffK + b * C::kTileBytes); };
+            auto v_buf = [&](int b) { return smem_u32(smem + C::kOffV + b * C::kTileBytes); };
             const uint32_t ds_addr = smem_u32(smem + C::kOffDS);
-            bool ok = __all_sync(0xffffffffu, !*abort) &&
-                      warp_wait(&bars->kv_full, 0, kSiteKV, abort);
+            bool ok = __all_sync(0xffffffffu, !*abort);
 
             // S^T = K Q^T  or  dP^T = V dO^T: M = 128 keys, N = 128 queries, K = d
             auto score_mma = [&](uint32_t d_tmem, uint32_t a_addr, uint32_t b_addr) {
@@ -607,17 +654,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * C::kChunkBytes + (kk & 3) * 32;
                     mma_ss_warp(d_tmem, sdesc_sw128(a_addr + off, 16, 1024),
-                           sdesc_sw128(b_addr + off, 16, 1024), C::kIdescScore, kk > 0 ? 1u : 0u);
+                                sdesc_sw128(b_addr + off, 16, 1024), C::kIdescScore,
+                                kk > 0 ? 1u : 0u);
                 }
             };
-            // dV += P^T dO  or  dK += dS^T Q: M = 128 keys, N = d, K = 128 queries
+            // dK += dS^T Q: M = 128 keys, N = d, K = 128 queries
             auto grad_mma = [&](uint32_t d_tmem, uint32_t a_addr, uint32_t b_addr, bool acc) {
 #pragma unroll
                 for (int kk = 0; kk < kTile / 16; ++kk) {
                     const uint32_t aoff = (kk >> 2) * C::kChunkBytes + (kk & 3) * 32;
                     mma_ss_warp(d_tmem, sdesc_sw128(a_addr + aoff, 16, 1024),
-                           sdesc_sw128(b_addr + kk * 2048, C::kChunkBytes, 1024), C::kIdescGrad,
-                           (acc || kk > 0) ? 1u : 0u);
+                                sdesc_sw128(b_addr + kk * 2048, C::kChunkBytes, 1024),
+                                C::kIdescGrad, (acc || kk > 0) ? 1u : 0u);
                 }
             };
             // dV += P^T dO with P^T in tensor memory (16 queries = 8 columns per step;
@@ -628,102 +676,141 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     const uint64_t bdesc = sdesc_sw128(b_addr + kk * 2048, C::kChunkBytes, 1024);
                     mma_ts_warp(tDV, tmem + C::p_col(kk), bdesc, C::kIdescGrad,
                                 (acc || kk > 0) ? 1u : 0u);
-                    if (PRECISE) mma_ts_warp(tDV, tmem + C::p_col(kk) + 32, bdesc, C::kIdescGrad, 1u);
+                    if (PRECISE)
+                        mma_ts_warp(tDV, tmem + C::p_col(kk) + 32, bdesc, C::kIdescGrad, 1u);
                 }
             };
             // dQ_i = dS K: M = 128 queries (dS^T read MN-major), N = d, K = 128 keys
-            auto dq_mma = [&](uint32_t a_addr, bool acc) {
+            auto dq_mma = [&](uint32_t a_addr, uint32_t k_addr, bool acc) {
 #pragma unroll
                 for (int kk = 0; kk < kTile / 16; ++kk)
                     mma_ss_warp(tDQ, sdesc_sw128(a_addr + kk * 2048, C::kChunkBytes, 1024),
-                           sdesc_sw128(k_addr + kk * 2048, C::kChunkBytes, 1024), C::kIdescDQ,
-                           (acc || kk > 0) ? 1u : 0u);
+                                sdesc_sw128(k_addr + kk * 2048, C::kChunkBytes, 1024),
+                                C::kIdescDQ, (acc || kk > 0) ? 1u : 0u);
             };
-            auto q_stage = [&](int n) {
-                return smem_u32(smem + C::kOffQ + (n % C::kStagesQ) * C::kTileBytes);
+            auto q_stage = [&](int g) {
+                return smem_u32(smem + C::kOffQ + (g % C::kStagesQ) * C::kTileBytes);
             };
-            auto do_stage = [&](int n) {
-                return smem_u32(smem + C::kOffDO + (n % C::kStagesDO) * C::kTileBytes);
+            auto do_stage = [&](int g) {
+                return smem_u32(smem + C::kOffDO + (g % C::kStagesDO) * C::kTileBytes);
             };
 
-            // prologue: S_0, dP_0
-            if (ok) ok = warp_wait(&bars->q_full[0], 0, kSiteQFull, abort);
-            if (ok) {
-                tc_fence_after();
-                score_mma(tS, k_addr, q_stage(0));
-                mma_commit_warp(&bars->s_full);
+            int bh, kt;
+            bool have = ok && item_of(0, bh, kt);
+            // prologue: S and dP^T of the first step
+            if (have) {
+                ok = warp_wait(&bars->kv_full[0], 0, kSiteKV, abort) &&
+                     warp_wait(&bars->q_full[0], 0, kSiteQFull, abort);
+                if (ok) {
+                    tc_fence_after();
+                    score_mma(tS, k_buf(0), q_stage(0));
+                    mma_commit_warp(&bars->s_full);
+                }
+                if (ok) ok = warp_wait(&bars->do_full[0], 0, kSiteDOFull, abort);
+                if (ok) {
+                    tc_fence_after();
+                    score_mma(tDP, v_buf(0), do_stage(0));
+                    mma_commit_warp(&bars->dp_full);
+                }
             }
-            if (ok) ok = warp_wait(&bars->do_full[0], 0, kSiteDOFull, abort);
-            if (ok) {
-                tc_fence_after();
-                score_mma(tDP, v_addr, do_stage(0));
-                mma_commit_warp(&bars->dp_full);
-            }
-            auto issue_s_next = [&](int n) -> bool {
-                if (!warp_wait(&bars->q_full[(n + 1) % C::kStagesQ], ((n + 1) / C::kStagesQ) & 1,
-                               kSiteQFull, abort))
-                    return false;
-                tc_fence_after();
-                score_mma(tS, k_addr, q_stage(n + 1));
-                mma_commit_warp(&bars->s_full);
-                return true;
-            };
-            for (int n = 0; ok && n < n_iter; ++n) {
-                // own P^T columns: S_{n+1} as soon as the compute warps hold S_n in
-                // registers
-                if (!C::kPAliasS && n + 1 < n_iter) {
-                    if (!warp_wait(&bars->s_free, n & 1, kSiteSFree, abort)) { ok = false; break; }
-                    if (!issue_s_next(n)) { ok = false; break; }
-                }
-                // dV += P^T dO_n
-                if (!warp_wait(&bars->p_full, n & 1, kSitePFull, abort)) { ok = false; break; }
-                tc_fence_after();
-                dv_mma(do_stage(n), n > 0);
-                mma_commit_warp(&bars->p_free);
-                mma_commit_warp(&bars->do_empty[n % C::kStagesDO]);
-                // P^T over S^T: S_{n+1} once dV_n, which reads P^T there, has completed
-                // (waiting for the commit rather than relying on issue order)
-                if (C::kPAliasS && n + 1 < n_iter) {
-                    if (!warp_wait(&bars->p_free, n & 1, kSitePFree, abort)) { ok = false; break; }
-                    if (!issue_s_next(n)) { ok = false; break; }
-                }
-                // dK += dS^T Q_n ; dQ_n = dS K
-                if (!warp_wait(&bars->ds_full, n & 1, kSiteDSFull, abort)) { ok = false; break; }
-                tc_fence_after();
-                grad_mma(tDK, ds_addr, q_stage(n), n > 0);
-                if (PRECISE) grad_mma(tDK, ds_addr + C::kScoreBytes, q_stage(n), true);
-                // separate dQ columns: free once dQ_{n-1} is drained; shared with dP^T:
-                // dP_n has been read (ds_full)
-                if (C::kSeparateDQ && n > 0 &&
-                    !warp_wait(&bars->dq_free, (n - 1) & 1, kSiteDQFree, abort)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                dq_mma(ds_addr, false);
-                if (PRECISE) dq_mma(ds_addr + C::kScoreBytes, true);
-                mma_commit_warp(&bars->dq_full);
-                mma_commit_warp(&bars->ds_free);
-                mma_commit_warp(&bars->q_empty[n % C::kStagesQ]);
-                // dP_{n+1}: its columns are free once dS_n is formed (separate dQ) or
-                // once dQ_n has left tensor memory (shared columns)
-                if (n + 1 < n_iter) {
-                    if (!C::kSeparateDQ &&
-                        !warp_wait(&bars->dq_free, n & 1, kSiteDQFree, abort)) {
-                        ok = false;
-                        break;
+            int g = 0;  // steps so far (all items)
+            for (int item = 0; ok && have; ++item) {
+                const int kb = item % C::kKVBufs, nkb = (item + 1) % C::kKVBufs;
+                int nbh, nkt;
+                const bool have_next = item_of(item + 1, nbh, nkt);
+                const int n_it = n_qtiles - first_qtile(kt);
+                for (int n = 0; ok && n < n_it; ++n, ++g) {
+                    const bool last = n + 1 == n_it;
+                    const bool next_step = !last || have_next;  // a step g + 1 exists
+                    const int kb1 = last ? nkb : kb;            // its K/V buffer
+                    // with one K/V buffer the next item's K/V arrive only after this
+                    // item's last dQ has released them: its first S is issued after that
+                    const bool s_late = last && C::kKVBufs == 1;
+                    // S_{g+1}; a new item's first also waits for that item's K/V
+                    auto issue_s = [&]() -> bool {
+                        if (last && !warp_wait(&bars->kv_full[nkb], ((item + 1) / C::kKVBufs) & 1,
+                                               kSiteKV, abort))
+                            return false;
+                        if (!warp_wait(&bars->q_full[(g + 1) % C::kStagesQ],
+                                       ((g + 1) / C::kStagesQ) & 1, kSiteQFull, abort))
+                            return false;
+                        tc_fence_after();
+                        score_mma(tS, k_buf(kb1), q_stage(g + 1));
+                        mma_commit_warp(&bars->s_full);
+                        return true;
+                    };
+                    // the S^T columns are free for S_{g+1}: own P^T columns, once the
+                    // compute warps hold S_g in registers; P^T over S^T, once dV_g (which
+                    // reads P^T there) has completed (its commit, not issue order)
+                    auto s_cols_free = [&]() -> bool {
+                        return C::kPAliasS ? warp_wait(&bars->p_free, g & 1, kSitePFree, abort)
+                                           : warp_wait(&bars->s_free, g & 1, kSiteSFree, abort);
+                    };
+                    if (!C::kPAliasS && next_step && !s_late) {
+                        if (!s_cols_free() || !issue_s()) { ok = false; break; }
                     }
-                    if (!warp_wait(&bars->do_full[(n + 1) % C::kStagesDO],
-                                   ((n + 1) / C::kStagesDO) & 1, kSiteDOFull, abort)) {
+                    // dV += P^T dO_g; an item's first step overwrites dV (and dK), so it
+                    // waits until the previous item's epilogue has read them
+                    if (!warp_wait(&bars->p_full, g & 1, kSitePFull, abort)) { ok = false; break; }
+                    if (n == 0 && item > 0 &&
+                        !warp_wait(&bars->acc_free, (item - 1) & 1, kSiteAccFree, abort)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    score_mma(tDP, v_addr, do_stage(n + 1));
-                    mma_commit_warp(&bars->dp_full);
+                    dv_mma(do_stage(g), n > 0);
+                    mma_commit_warp(&bars->p_free);
+                    mma_commit_warp(&bars->do_empty[g % C::kStagesDO]);  // dP_g, dV_g read it
+                    if (C::kPAliasS && next_step && !s_late) {
+                        if (!s_cols_free() || !issue_s()) { ok = false; break; }
+                    }
+                    // dK += dS^T Q_g ; dQ_g = dS K
+                    if (!warp_wait(&bars->ds_full, g & 1, kSiteDSFull, abort)) { ok = false; break; }
+                    tc_fence_after();
+                    grad_mma(tDK, ds_addr, q_stage(g), n > 0);
+                    if (PRECISE) grad_mma(tDK, ds_addr + C::kScoreBytes, q_stage(g), true);
+                    // separate dQ columns: free once dQ_{g-1} is drained; shared with dP^T:
+                    // dP_g has been read (ds_full)
+                    if (C::kSeparateDQ && g > 0 &&
+                        !warp_wait(&bars->dq_free, (g - 1) & 1, kSiteDQFree, abort)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    dq_mma(ds_addr, k_buf(kb), false);
+                    if (PRECISE) dq_mma(ds_addr + C::kScoreBytes, k_buf(kb), true);
+                    mma_commit_warp(&bars->dq_full);
+                    mma_commit_warp(&bars->ds_free);
+                    mma_commit_warp(&bars->q_empty[g % C::kStagesQ]);
+                    if (last) {
+                        mma_commit_warp(&bars->acc_done);      // the item's dV, dK are complete
+                        mma_commit_warp(&bars->kv_empty[kb]);  // and its K, V read for good
+                    }
+                    if (s_late && next_step) {
+                        if (!s_cols_free() || !issue_s()) { ok = false; break; }
+                    }
+                    // dP_{g+1}: its columns are free once dS_g is formed (separate dQ) or
+                    // once dQ_g has left tensor memory (shared columns)
+                    if (next_step) {
+                        if (!C::kSeparateDQ &&
+                            !warp_wait(&bars->dq_free, g & 1, kSiteDQFree, abort)) {
+                            ok = false;
+                            break;
+                        }
+                        if (!warp_wait(&bars->do_full[(g + 1) % C::kStagesDO],
+                                       ((g + 1) / C::kStagesDO) & 1, kSiteDOFull, abort)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        score_mma(tDP, v_buf(kb1), do_stage(g + 1));
+                        mma_commit_warp(&bars->dp_full);
+                    }
                 }
+                kt = nkt;
+                bh = nbh;
+                have = have_next;
             }
-            if (ok) mma_commit_warp(&bars->acc_done);
             mma_commit_warp(&bars->mma_final);
             mbar_wait_drain(&bars->mma_final, 0);
         }
@@ -810,6 +897,18 @@ __global__ void __launch_bounds__(256) attn_bwd_dq_convert_kernel(const float* _
                                                  pack_bf16x2(b.x, b.y), pack_bf16x2(b.z, b.w));
 }
 
+int sm_count() {
+    static int n = 0;
+    if (n == 0) {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+            n <= 0)
+            n = 148;
+    }
+    return n;
+}
+
 template <int D, bool PRECISE>
 cudaError_t launch_dkdv_dp(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                            const CUtensorMap& tdo, const CUtensorMap& tdq, const float* rowstats,
@@ -825,10 +924,14 @@ cudaError_t launch_dkdv_dp(const CUtensorMap& tq, const CUtensorMap& tk, const C
         configured = true;
     }
     const int n_kvtiles = (T + kTile - 1) / kTile;
-    dim3 grid(BH, n_kvtiles);
+    const long long items = (long long)BH * n_kvtiles;
+    if (items > 0x7fffffff) return cudaErrorInvalidValue;
+    const int n_items = (int)items;
+    // persistent: one CTA per SM (shared memory and tensor memory allow no more)
+    const int grid = n_items < sm_count() ? n_items : sm_count();
     attn_bwd_dkdv_kernel<D, PRECISE><<<grid, kBwdThreads, C::kSmemBytes, stream>>>(
-        tq, tk, tv, tdo, tdq, rowstats, dq_accum, dk, dv, T, BH, n_kvtiles, scale, scale * kLog2e,
-        causal, grad_f32);
+        tq, tk, tv, tdo, tdq, rowstats, dq_accum, dk, dv, T, BH, n_kvtiles, n_items, scale,
+        scale * kLog2e, causal, grad_f32);
     return cudaGetLastError();
 }
 

@@ -409,7 +409,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             for (int c = 0; c < C::kChunks; ++c)
                 tma_store_3d(&tmap_o, stage + c * C::kChunkBytes, 64 * c, qt * kTile, bh);
             tma_store_commit();
-            tma_store_wait_all();
+            tma_store_wait_all_read();  // the store has read the staged O
         }
     }
 
