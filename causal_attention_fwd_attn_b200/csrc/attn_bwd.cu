@@ -764,13 +764,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     if (C::kPAliasS && next_step && !s_late) {
                         if (!s_cols_free() || !issue_s()) { ok = false; break; }
                     }
-                    // dK += dS^T Q_g ; dQ_g = dS K
+                    // dQ_g = dS K and dK += dS^T Q_g.  With a staging buffer of its own, dQ_g
+                    // goes first, so that its drain (and, with shared columns, the next
+                    // dP^T) starts while dK_g runs.  Staged through the dS^T buffer, the
+                    // drain may start only once dK_g has read dS^T too: dK_g goes first.
+                    // Separate dQ columns are free once dQ_{g-1} is drained; shared with
+                    // dP^T, once dP_g has been read (ds_full).
+                    constexpr bool kDQFirst = C::kStageOwn;
                     if (!warp_wait(&bars->ds_full, g & 1, kSiteDSFull, abort)) { ok = false; break; }
                     tc_fence_after();
-                    grad_mma(tDK, ds_addr, q_stage(g), n > 0);
-                    if (PRECISE) grad_mma(tDK, ds_addr + C::kScoreBytes, q_stage(g), true);
-                    // separate dQ columns: free once dQ_{g-1} is drained; shared with dP^T:
-                    // dP_g has been read (ds_full)
+                    if constexpr (!kDQFirst) {
+                        grad_mma(tDK, ds_addr, q_stage(g), n > 0);
+                        if (PRECISE) grad_mma(tDK, ds_addr + C::kScoreBytes, q_stage(g), true);
+                    }
                     if (C::kSeparateDQ && g > 0 &&
                         !warp_wait(&bars->dq_free, (g - 1) & 1, kSiteDQFree, abort)) {
                         ok = false;
@@ -780,6 +786,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     dq_mma(ds_addr, k_buf(kb), false);
                     if (PRECISE) dq_mma(ds_addr + C::kScoreBytes, k_buf(kb), true);
                     mma_commit_warp(&bars->dq_full);
+                    if constexpr (kDQFirst) {
+                        grad_mma(tDK, ds_addr, q_stage(g), n > 0);
+                        if (PRECISE) grad_mma(tDK, ds_addr + C::kScoreBytes, q_stage(g), true);
+                    }
                     mma_commit_warp(&bars->ds_free);
                     mma_commit_warp(&bars->q_empty[g % C::kStagesQ]);
                     if (last) {
