@@ -11,13 +11,20 @@
 // diagonal-matrix trick for the rescale is not needed here: in tensor memory a
 // row of the accumulator is one lane, owned by one thread.
 //
-// Blackwell design (one CTA per query tile, 6 warps):
-//   warp 0      TMA producer: Q once, then K/V tiles into an NS-stage ring.
-//   warp 1      MMA issuer (one thread): S = Q K^T into TMEM, then O += P V with
-//               P read from TMEM (tcgen05.mma with A in tensor memory).
+// Blackwell design (persistent CTAs, one per SM at most, 6 warps).  A work item is
+// one (head, query tile); items are dealt heaviest first, zigzag over the CTAs, and
+// every role walks the same item sequence, so one item's epilogue and the next
+// item's Q load overlap the neighbouring item's products.
+//   warp 0      TMA producer: Q per item (once the item before has finished its
+//               score products), then K/V tiles into an NS-stage ring.
+//   warp 1      MMA issuer (converged warp, one elected lane issues): S = Q K^T into
+//               TMEM, then O += P V with P read from TMEM (tcgen05.mma with A in
+//               tensor memory).  An item's first P V waits until the previous
+//               item's O has been read out.
 //   warps 2..5  softmax: thread r owns query row r (TMEM lane r): loads its S row,
 //               masks, updates the running max/sum, writes P (bf16) back to TMEM,
-//               and in the epilogue normalises O and stores O (TMA) and LSE.
+//               and in the epilogue normalises its O row and writes it and its LSE
+//               to global memory.
 // Tensor memory (512 columns): S [0,128) | P0 [128,192) | P1 [192,256) | O [256, 256+d)
 // | P0 lo [384,448) | P1 lo [448,512) (the lo halves only in precise mode, where P
 // enters P V as two bf16 terms, hi = bf16(p) and lo = bf16(p - hi)).
@@ -46,7 +53,7 @@ __device__ __forceinline__ constexpr bool use_poly_pair(int) { return false; }
 // wait sites (for the device error word)
 enum : uint32_t {
     kSiteQ = 1, kSiteKFull, kSiteVFull, kSiteKVEmpty, kSiteSFull, kSiteSFree, kSitePFull,
-    kSitePV, kSiteODone
+    kSitePV, kSiteODone, kSiteQEmpty, kSiteOFree
 };
 
 template <int D>
@@ -71,7 +78,7 @@ struct FwdCfg {
 };
 
 struct FwdBarriers {
-    uint64_t q_full;
+    uint64_t q_full, q_empty;
     uint64_t k_full[4];
     uint64_t v_full[4];
     uint64_t kv_empty[4];
@@ -79,7 +86,7 @@ struct FwdBarriers {
     uint64_t s_free;
     uint64_t p_full;
     uint64_t pv_done;
-    uint64_t o_done;
+    uint64_t o_done, o_free;  // an item's O complete / read out of tensor memory
     uint64_t mma_final;
     uint32_t tmem_base;
     int abort;
@@ -95,9 +102,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
                     const __grid_constant__ CUtensorMap tmap_k,
                     const __grid_constant__ CUtensorMap tmap_v,
-                    const __grid_constant__ CUtensorMap tmap_o, void* __restrict__ o_f32_out,
-                    float* __restrict__ lse_out, int T, int n_qtiles, float scale_log2,
-                    int negate_scores, int causal, int o_f32) {
+                    void* __restrict__ o_out, float* __restrict__ lse_out, int T, int BH,
+                    int n_qtiles, int n_items, float scale_log2, int negate_scores, int causal,
+                    int o_f32) {
     using C = FwdCfg<D>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -105,15 +112,26 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     FwdBarriers* bars = reinterpret_cast<FwdBarriers*>(smem + C::kOffBar);
     volatile int* abort = &bars->abort;
 
-    const int bh = blockIdx.x;
-    const int qt = n_qtiles - 1 - blockIdx.y;  // heaviest (most key tiles) first
     const int n_kvtiles_total = (T + kTile - 1) / kTile;
-    const int n_tiles = causal ? qt + 1 : n_kvtiles_total;
+    const int n_ctas = (int)gridDim.x;
+    // Persistent CTAs.  The CTA's r-th work item is a (head, query tile) pair; items
+    // are numbered heaviest first (the last query tile sees the most key tiles) and
+    // dealt in a zigzag over the CTAs.  Every role walks the same item sequence; the
+    // per-key-tile barriers count across items.
+    auto item_of = [&](int r, int& bh_out, int& qt_out) -> bool {
+        const int k = r * n_ctas + ((r & 1) ? (n_ctas - 1 - (int)blockIdx.x) : (int)blockIdx.x);
+        if (k >= n_items) return false;
+        qt_out = n_qtiles - 1 - k / BH;
+        bh_out = k % BH;
+        return true;
+    };
+    auto tiles_of = [&](int qt_) { return causal ? qt_ + 1 : n_kvtiles_total; };
     const uint32_t warp = warp_id();
     const uint32_t lane = lane_id();
 
     if (threadIdx.x == 0) {
         mbar_init(&bars->q_full, 1);
+        mbar_init(&bars->q_empty, 1);
         for (int s = 0; s < C::kStages; ++s) {
             mbar_init(&bars->k_full[s], 1);
             mbar_init(&bars->v_full[s], 1);
@@ -124,6 +142,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         mbar_init(&bars->p_full, 4);
         mbar_init(&bars->pv_done, 1);
         mbar_init(&bars->o_done, 1);
+        mbar_init(&bars->o_free, 4);
         mbar_init(&bars->mma_final, 1);
         bars->abort = 0;
         fence_mbar_init();
@@ -143,30 +162,44 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             tma_prefetch_desc(&tmap_q);
             tma_prefetch_desc(&tmap_k);
             tma_prefetch_desc(&tmap_v);
-            mbar_arrive_expect_tx(&bars->q_full, C::kTileBytes);
-            for (int c = 0; c < C::kChunks; ++c)
-                tma_load_3d(smem + C::kOffQ + c * C::kChunkBytes, &tmap_q, &bars->q_full, 64 * c,
-                            qt * kTile, bh);
-            int last_use[4] = {-1, -1, -1, -1};
-            for (int n = 0; n < n_tiles; ++n) {
-                const int st = n % C::kStages;
-                const int use = n / C::kStages;
-                if (use > 0 && !mbar_wait(&bars->kv_empty[st], (use - 1) & 1, kSiteKVEmpty, abort))
+            int last_use[4] = {-1, -1, -1, -1}, last_q = -1;
+            int g = 0;  // key tiles so far (all items)
+            bool run = true;
+            int bh, qt;
+            for (int item = 0; run && item_of(item, bh, qt); ++item) {
+                // Q of the item, once the previous item's last score product has read Q
+                if (item > 0 &&
+                    !mbar_wait(&bars->q_empty, (item - 1) & 1, kSiteQEmpty, abort))
                     break;
-                const int j = causal ? qt - n : n_kvtiles_total - 1 - n;
-                mbar_arrive_expect_tx(&bars->k_full[st], C::kTileBytes);
+                mbar_arrive_expect_tx(&bars->q_full, C::kTileBytes);
                 for (int c = 0; c < C::kChunks; ++c)
-                    tma_load_3d(smem + C::kOffK + st * C::kTileBytes + c * C::kChunkBytes, &tmap_k,
-                                &bars->k_full[st], 64 * c, j * kTile, bh);
-                mbar_arrive_expect_tx(&bars->v_full[st], C::kTileBytes);
-                for (int c = 0; c < C::kChunks; ++c)
-                    tma_load_3d(smem + C::kOffV + st * C::kTileBytes + c * C::kChunkBytes, &tmap_v,
-                                &bars->v_full[st], 64 * c, j * kTile, bh);
-                last_use[st] = use;
+                    tma_load_3d(smem + C::kOffQ + c * C::kChunkBytes, &tmap_q, &bars->q_full,
+                                64 * c, qt * kTile, bh);
+                last_q = item;
+                const int n_tiles = tiles_of(qt);
+                for (int n = 0; n < n_tiles; ++n, ++g) {
+                    const int st = g % C::kStages;
+                    const int use = g / C::kStages;
+                    if (use > 0 &&
+                        !mbar_wait(&bars->kv_empty[st], (use - 1) & 1, kSiteKVEmpty, abort)) {
+                        run = false;
+                        break;
+                    }
+                    const int j = causal ? qt - n : n_kvtiles_total - 1 - n;
+                    mbar_arrive_expect_tx(&bars->k_full[st], C::kTileBytes);
+                    for (int c = 0; c < C::kChunks; ++c)
+                        tma_load_3d(smem + C::kOffK + st * C::kTileBytes + c * C::kChunkBytes,
+                                    &tmap_k, &bars->k_full[st], 64 * c, j * kTile, bh);
+                    mbar_arrive_expect_tx(&bars->v_full[st], C::kTileBytes);
+                    for (int c = 0; c < C::kChunks; ++c)
+                        tma_load_3d(smem + C::kOffV + st * C::kTileBytes + c * C::kChunkBytes,
+                                    &tmap_v, &bars->v_full[st], 64 * c, j * kTile, bh);
+                    last_use[st] = use;
+                }
             }
             if (*abort) {
                 // let copies already issued land before the CTA's memory is released
-                mbar_wait_drain(&bars->q_full, 0);
+                if (last_q >= 0) mbar_wait_drain(&bars->q_full, last_q & 1);
                 for (int s = 0; s < C::kStages; ++s)
                     if (last_use[s] >= 0) {
                         mbar_wait_drain(&bars->k_full[s], last_use[s] & 1);
@@ -183,11 +216,16 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             const uint32_t q_addr = smem_u32(smem + C::kOffQ);
             // bit 13 of the instruction descriptor negates A: S = (-Q) K^T for scale < 0
             const uint32_t idesc_s = C::kIdescS | (negate_scores ? (1u << 13) : 0u);
-            bool ok = warp_wait(&bars->q_full, 0, kSiteQ, abort);
-            auto issue_pv = [&](int m) -> bool {
+            bool ok = true;
+            // O += P(m) V(m); m counts key tiles over all items.  An item's first P V
+            // overwrites O, so it waits until the previous item's epilogue has read O.
+            auto issue_pv = [&](int m, bool first, int item) -> bool {
                 const int st = m % C::kStages;
                 if (!warp_wait(&bars->p_full, m & 1, kSitePFull, abort)) return false;
                 if (!warp_wait(&bars->v_full[st], (m / C::kStages) & 1, kSiteVFull, abort))
+                    return false;
+                if (first && item > 0 &&
+                    !warp_wait(&bars->o_free, (item - 1) & 1, kSiteOFree, abort))
                     return false;
                 tc_fence_after();
                 const uint32_t tP = tmem + ((m & 1) ? C::kColP1 : C::kColP0);
@@ -197,40 +235,52 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 for (int kk = 0; kk < kTile / 16; ++kk) {
                     // B = V tile, MN-major: 16 keys = 2 x 8-row groups of 1024 bytes
                     const uint64_t bdesc = sdesc_sw128(v_addr + kk * 2048, C::kChunkBytes, 1024);
-                    mma_ts_warp(tO, tP + kk * 8, bdesc, C::kIdescPV, (m > 0 || kk > 0) ? 1u : 0u);
+                    mma_ts_warp(tO, tP + kk * 8, bdesc, C::kIdescPV, (!first || kk > 0) ? 1u : 0u);
                     if (PRECISE) mma_ts_warp(tO, tPlo + kk * 8, bdesc, C::kIdescPV, 1u);
                 }
                 mma_commit_warp(&bars->pv_done);
                 mma_commit_warp(&bars->kv_empty[st]);
                 return true;
             };
-            for (int n = 0; ok && n < n_tiles; ++n) {
-                const int st = n % C::kStages;
-                if (!warp_wait(&bars->k_full[st], (n / C::kStages) & 1, kSiteKFull, abort)) {
+            int g = 0;  // key tiles so far (all items)
+            int bh, qt;
+            for (int item = 0; ok && item_of(item, bh, qt); ++item) {
+                if (!warp_wait(&bars->q_full, item & 1, kSiteQ, abort)) {
                     ok = false;
                     break;
                 }
-                if (n > 0 && !warp_wait(&bars->s_free, (n - 1) & 1, kSiteSFree, abort)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                const uint32_t k_addr = smem_u32(smem + C::kOffK + st * C::kTileBytes);
+                const int n_tiles = tiles_of(qt);
+                for (int n = 0; ok && n < n_tiles; ++n, ++g) {
+                    const int st = g % C::kStages;
+                    if (!warp_wait(&bars->k_full[st], (g / C::kStages) & 1, kSiteKFull, abort)) {
+                        ok = false;
+                        break;
+                    }
+                    // the S columns: the softmax has read the previous S (any item)
+                    if (g > 0 && !warp_wait(&bars->s_free, (g - 1) & 1, kSiteSFree, abort)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t k_addr = smem_u32(smem + C::kOffK + st * C::kTileBytes);
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t koff = (kk >> 2) * C::kChunkBytes + (kk & 3) * 32;
-                    const uint64_t adesc = sdesc_sw128(q_addr + koff, 16, 1024);
-                    const uint64_t bdesc = sdesc_sw128(k_addr + koff, 16, 1024);
-                    mma_ss_warp(tS, adesc, bdesc, idesc_s, kk > 0 ? 1u : 0u);
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t koff = (kk >> 2) * C::kChunkBytes + (kk & 3) * 32;
+                        const uint64_t adesc = sdesc_sw128(q_addr + koff, 16, 1024);
+                        const uint64_t bdesc = sdesc_sw128(k_addr + koff, 16, 1024);
+                        mma_ss_warp(tS, adesc, bdesc, idesc_s, kk > 0 ? 1u : 0u);
+                    }
+                    mma_commit_warp(&bars->s_full);
+                    // the item's last score product is the last reader of Q
+                    if (n == n_tiles - 1) mma_commit_warp(&bars->q_empty);
+                    if (n > 0 && !issue_pv(g - 1, n == 1, item)) {
+                        ok = false;
+                        break;
+                    }
                 }
-                mma_commit_warp(&bars->s_full);
-                if (n > 0 && !issue_pv(n - 1)) {
-                    ok = false;
-                    break;
-                }
+                if (ok) ok = issue_pv(g - 1, n_tiles == 1, item);
+                if (ok) mma_commit_warp(&bars->o_done);
             }
-            if (ok) ok = issue_pv(n_tiles - 1);
-            if (ok) mma_commit_warp(&bars->o_done);
             // every MMA this thread issued must retire before tensor memory is freed
             mma_commit_warp(&bars->mma_final);
             mbar_wait_drain(&bars->mma_final, 0);
@@ -241,13 +291,18 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         const uint32_t lane_off = ((warp & 3) << 5) << 16;
         const uint32_t tS = tmem + lane_off + C::kColS;
         const uint32_t tO = tmem + lane_off + C::kColO;
+        bool ok = true;
+        int g0 = 0;  // key tiles before this item (all items)
+        int bh, qt;
+        for (int item = 0; ok && item_of(item, bh, qt); ++item) {
+        const int n_tiles = tiles_of(qt);
         const int grow = qt * kTile + (int)row;  // query index of this row
         float m_run = -INFINITY;                  // running max, log2 units
         float l_run = 0.f;                        // running sum of exp2(u - m_run)
-        bool ok = true;
         for (int n = 0; n < n_tiles; ++n) {
+            const int g = g0 + n;
             const int j = causal ? qt - n : n_kvtiles_total - 1 - n;
-            if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full, n & 1, kSiteSFull, abort))) {
+            if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full, g & 1, kSiteSFull, abort))) {
                 ok = false;
                 break;
             }
@@ -300,7 +355,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             if (n > 0 && __any_sync(0xffffffffu, need)) {
                 // O must include P(n-1) V before it is rescaled
                 if (!__all_sync(0xffffffffu,
-                                mbar_wait(&bars->pv_done, (n - 1) & 1, kSitePV, abort))) {
+                                mbar_wait(&bars->pv_done, (g - 1) & 1, kSitePV, abort))) {
                     ok = false;
                     break;
                 }
@@ -319,8 +374,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             }
 
             // P = exp2(s * scale_log2 - m), row sum, pack to bf16 pairs, store to TMEM
-            const uint32_t tP = tmem + lane_off + ((n & 1) ? C::kColP1 : C::kColP0);
-            const uint32_t tPlo = tmem + lane_off + ((n & 1) ? C::kColPlo1 : C::kColPlo0);
+            const uint32_t tP = tmem + lane_off + ((g & 1) ? C::kColP1 : C::kColP0);
+            const uint32_t tPlo = tmem + lane_off + ((g & 1) ? C::kColPlo1 : C::kColPlo0);
             const float neg_m = -m_run;
             const float2 sl2 = make_float2(scale_log2, scale_log2);
             const float2 nm2 = make_float2(neg_m, neg_m);
@@ -363,53 +418,54 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             if (lane == 0) mbar_arrive(&bars->p_full);
         }
 
+        if (!ok) break;
+        g0 += n_tiles;
+
         // ----------------------------------------------------------- epilogue
-        const bool epi =
-            ok && __all_sync(0xffffffffu, mbar_wait(&bars->o_done, 0, kSiteODone, abort));
-        uint8_t* stage = smem + C::kOffQ;  // Q is no longer read by any MMA
-        if (epi) {
-            tc_fence_after();
-            const float inv_l = 1.f / l_run;
-            if (grow < T) lse_out[(size_t)bh * T + grow] = (m_run + log2f(l_run)) * kLn2;
-            float* orow = reinterpret_cast<float*>(o_f32_out) + ((size_t)bh * T + grow) * D;
+        // O straight from tensor memory to global memory: each thread writes its
+        // own row (d contiguous elements).
+        if (!__all_sync(0xffffffffu, mbar_wait(&bars->o_done, item & 1, kSiteODone, abort))) {
+            ok = false;
+            break;
+        }
+        tc_fence_after();
+        const float inv_l = 1.f / l_run;
+        if (grow < T) lse_out[(size_t)bh * T + grow] = (m_run + log2f(l_run)) * kLn2;
 #pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
-                uint32_t r[32];
-                tmem_ld32(tO + c * 32, r);  // all lanes: the load is warp-collective
-                tmem_wait_ld();
-                if (!o_f32) {
-                    uint32_t pk[16];
-#pragma unroll
-                    for (int e = 0; e < 16; ++e)
-                        pk[e] = pack_bf16x2(__uint_as_float(r[2 * e]) * inv_l,
-                                            __uint_as_float(r[2 * e + 1]) * inv_l);
-                    // 32 columns = 64 bytes = 4 x 16-byte chunks of the row
-                    uint8_t* chunk_base = stage + (c >> 1) * C::kChunkBytes;
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const uint32_t ch = (c & 1) * 4 + e;
-                        *reinterpret_cast<uint4*>(chunk_base + sw128_offset(row, ch)) =
-                            make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
-                    }
-                } else if (grow < T) {
+        for (int c = 0; c < D / 32; ++c) {
+            uint32_t r[32];
+            tmem_ld32(tO + c * 32, r);  // all lanes: the load is warp-collective
+            tmem_wait_ld();
+            if (grow < T) {
+                const size_t base = ((size_t)bh * T + grow) * D + c * 32;
+                if (o_f32) {
+                    float4* dst = reinterpret_cast<float4*>(static_cast<float*>(o_out) + base);
 #pragma unroll
                     for (int e = 0; e < 8; ++e)
-                        *reinterpret_cast<float4*>(orow + c * 32 + 4 * e) =
-                            make_float4(__uint_as_float(r[4 * e]) * inv_l,
-                                        __uint_as_float(r[4 * e + 1]) * inv_l,
-                                        __uint_as_float(r[4 * e + 2]) * inv_l,
-                                        __uint_as_float(r[4 * e + 3]) * inv_l);
+                        dst[e] = make_float4(__uint_as_float(r[4 * e]) * inv_l,
+                                             __uint_as_float(r[4 * e + 1]) * inv_l,
+                                             __uint_as_float(r[4 * e + 2]) * inv_l,
+                                             __uint_as_float(r[4 * e + 3]) * inv_l);
+                } else {
+                    uint4* dst =
+                        reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(o_out) + base);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        dst[e] = make_uint4(pack_bf16x2(__uint_as_float(r[8 * e]) * inv_l,
+                                                        __uint_as_float(r[8 * e + 1]) * inv_l),
+                                            pack_bf16x2(__uint_as_float(r[8 * e + 2]) * inv_l,
+                                                        __uint_as_float(r[8 * e + 3]) * inv_l),
+                                            pack_bf16x2(__uint_as_float(r[8 * e + 4]) * inv_l,
+                                                        __uint_as_float(r[8 * e + 5]) * inv_l),
+                                            pack_bf16x2(__uint_as_float(r[8 * e + 6]) * inv_l,
+                                                        __uint_as_float(r[8 * e + 7]) * inv_l));
                 }
             }
-            if (!o_f32) fence_proxy_async_smem();
         }
-        // every softmax thread reaches this barrier, aborted or not
-        named_bar_sync(1, 128);
-        if (!o_f32 && warp == 2 && lane == 0 && epi && !*abort) {
-            for (int c = 0; c < C::kChunks; ++c)
-                tma_store_3d(&tmap_o, stage + c * C::kChunkBytes, 64 * c, qt * kTile, bh);
-            tma_store_commit();
-            tma_store_wait_all_read();  // the store has read the staged O
+        // the next item's first P V may now overwrite O
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->o_free);
         }
     }
 
@@ -423,10 +479,22 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     }
 }
 
+int sm_count() {
+    static int n = 0;
+    if (n == 0) {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+            n <= 0)
+            n = 148;
+    }
+    return n;
+}
+
 template <int D, bool PRECISE>
 cudaError_t launch_fwd_dp(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                          const CUtensorMap& to, void* o, float* lse, int BH, int T, float scale,
-                          int causal, int o_f32, cudaStream_t stream) {
+                          void* o, float* lse, int BH, int T, float scale, int causal, int o_f32,
+                          cudaStream_t stream) {
     using C = FwdCfg<D>;
     static bool configured = false;
     if (!configured) {
@@ -437,34 +505,31 @@ cudaError_t launch_fwd_dp(const CUtensorMap& tq, const CUtensorMap& tk, const CU
         configured = true;
     }
     const int n_qtiles = (T + kTile - 1) / kTile;
-    dim3 grid(BH, n_qtiles);
+    const int n_items = BH * n_qtiles;
+    const int grid = n_items < sm_count() ? n_items : sm_count();
     attn_fwd_kernel<D, PRECISE><<<grid, kFwdThreads, C::kSmemBytes, stream>>>(
-        tq, tk, tv, to, o, lse, T, n_qtiles, fabsf(scale) * kLog2e, scale < 0.f ? 1 : 0, causal,
-        o_f32);
+        tq, tk, tv, o, lse, T, BH, n_qtiles, n_items, fabsf(scale) * kLog2e,
+        scale < 0.f ? 1 : 0, causal, o_f32);
     return cudaGetLastError();
 }
 
 template <int D>
 cudaError_t launch_fwd_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                         const CUtensorMap& to, void* o, float* lse, int BH, int T, float scale,
-                         int causal, int o_f32, int precise, cudaStream_t stream) {
+                         void* o, float* lse, int BH, int T, float scale, int causal, int o_f32,
+                         int precise, cudaStream_t stream) {
     if (precise)
-        return launch_fwd_dp<D, true>(tq, tk, tv, to, o, lse, BH, T, scale, causal, o_f32,
-                                      stream);
-    return launch_fwd_dp<D, false>(tq, tk, tv, to, o, lse, BH, T, scale, causal, o_f32, stream);
+        return launch_fwd_dp<D, true>(tq, tk, tv, o, lse, BH, T, scale, causal, o_f32, stream);
+    return launch_fwd_dp<D, false>(tq, tk, tv, o, lse, BH, T, scale, causal, o_f32, stream);
 }
 
 }  // namespace
 
 cudaError_t launch_attn_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                            const CUtensorMap& to, void* o, float* lse, int BH, int T, int d,
-                            float scale, int causal, int o_f32, int precise,
-                            cudaStream_t stream) {
+                            void* o, float* lse, int BH, int T, int d, float scale, int causal,
+                            int o_f32, int precise, cudaStream_t stream) {
     if (d == 64)
-        return launch_fwd_d<64>(tq, tk, tv, to, o, lse, BH, T, scale, causal, o_f32, precise,
-                                stream);
-    return launch_fwd_d<128>(tq, tk, tv, to, o, lse, BH, T, scale, causal, o_f32, precise,
-                             stream);
+        return launch_fwd_d<64>(tq, tk, tv, o, lse, BH, T, scale, causal, o_f32, precise, stream);
+    return launch_fwd_d<128>(tq, tk, tv, o, lse, BH, T, scale, causal, o_f32, precise, stream);
 }
 
 cudaError_t read_and_clear_device_error_fwd(unsigned int* value) {

@@ -140,7 +140,7 @@ int forge_attn_fwd_ex(const void* q, const void* k, const void* v, void* o, floa
         (reinterpret_cast<uintptr_t>(lse) & 3u))
         return FORGE_ATTN_ERR_MISALIGNED;
     const long long BH = (long long)B * H;
-    CUtensorMap tq, tk, tv, to;
+    CUtensorMap tq, tk, tv;
     if ((s = make_map_bf16(&tq, q, d, T, BH)) != FORGE_ATTN_OK) return s;
     if ((s = make_map_bf16(&tk, k, d, T, BH)) != FORGE_ATTN_OK) return s;
     if ((s = make_map_bf16(&tv, v, d, T, BH)) != FORGE_ATTN_OK) return s;
@@ -150,9 +150,7 @@ int forge_attn_fwd_ex(const void* q, const void* k, const void* v, void* o, floa
     if (d == 64 && !precise)
         return cuda_status(launch_attn_fwd_pair(tq, tk, tv, o, lse, (int)BH, T, d, scale, causal,
                                                 o_f32, static_cast<cudaStream_t>(stream)));
-    // the output map is only used for bf16 output
-    if ((s = make_map_bf16(&to, o_f32 ? q : o, d, T, BH)) != FORGE_ATTN_OK) return s;
-    return cuda_status(launch_attn_fwd(tq, tk, tv, to, o, lse, (int)BH, T, d, scale, causal,
+    return cuda_status(launch_attn_fwd(tq, tk, tv, o, lse, (int)BH, T, d, scale, causal,
                                        o_f32, (flags & FORGE_ATTN_PRECISE) != 0,
                                        static_cast<cudaStream_t>(stream)));
 }

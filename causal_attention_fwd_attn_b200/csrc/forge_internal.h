@@ -14,9 +14,10 @@ constexpr int kTile = 128;
 
 // Launchers.  Tensor maps describe bf16 [B*H][T][d] tensors with a
 // {64, 128, 1} box and 128-byte swizzle.
+// The one-query-tile persistent forward; o is bf16 or fp32 (o_f32).
 cudaError_t launch_attn_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                            const CUtensorMap& to, void* o, float* lse, int BH, int T, int d,
-                            float scale, int causal, int o_f32, int precise, cudaStream_t stream);
+                            void* o, float* lse, int BH, int T, int d, float scale, int causal,
+                            int o_f32, int precise, cudaStream_t stream);
 
 // The two-query-tile persistent forward (no precise mode); o is bf16 or fp32 (o_f32).
 cudaError_t launch_attn_fwd_pair(const CUtensorMap& tq, const CUtensorMap& tk,
