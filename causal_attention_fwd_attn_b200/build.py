@@ -19,8 +19,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIBRARY = os.path.join(PKG, "libforge_attn.so")
-SOURCES = ["forge_attn_api.cu", "attn_fwd.cu", "attn_fwd_pair.cu", "attn_bwd.cu", "tc_probe.cu",
-           "forge_attn_noalloc.cu"]
+SOURCES = ["forge_attn_api.cu", "attn_fwd.cu", "attn_bwd.cu", "tc_probe.cu", "forge_attn_noalloc.cu"]
 HEADERS = ["sm100_ptx.cuh", "forge_internal.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
@@ -49,7 +48,7 @@ def build(force: bool = False, ptxas_info: bool = False, verbose: bool = False) 
     if not force and not ptxas_info and up_to_date():
         return LIBRARY
     # No relocatable device code: ptxas then honours per-warpgroup register budgets
-    # (setmaxnreg), which the pair forward and the dK/dV kernel rely on.
+    # (setmaxnreg), which the dK/dV kernel relies on.
     cmd = [nvcc_path(), *ARCH, "-O3", "-lineinfo", "-std=c++17", "-shared",
            "-Xcompiler", "-fPIC", "-I", INCLUDE, "-o", LIBRARY + ".tmp"]
     if ptxas_info:

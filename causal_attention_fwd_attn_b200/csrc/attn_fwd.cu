@@ -11,10 +11,11 @@
 // diagonal-matrix trick for the rescale is not needed here: in tensor memory a
 // row of the accumulator is one lane, owned by one thread.
 //
-// Blackwell design (persistent CTAs, one per SM at most, 6 warps).  A work item is
-// one (head, query tile); items are dealt heaviest first, zigzag over the CTAs, and
-// every role walks the same item sequence, so one item's epilogue and the next
-// item's Q load overlap the neighbouring item's products.
+// Blackwell design (persistent CTAs, one per SM at most, 6 warps; used for every head
+// dimension and mode).  A work item is one (head, query tile); items are dealt
+// heaviest first, zigzag over the CTAs, and every role walks the same item sequence,
+// so one item's epilogue and the next item's Q load overlap the neighbouring item's
+// products.
 //   warp 0      TMA producer: Q per item (once the item before has finished its
 //               score products), then K/V tiles into an NS-stage ring.
 //   warp 1      MMA issuer (converged warp, one elected lane issues): S = Q K^T into
@@ -25,12 +26,14 @@
 //               masks, updates the running max/sum, writes P (bf16) back to TMEM,
 //               and in the epilogue normalises its O row and writes it and its LSE
 //               to global memory.
-// Tensor memory (512 columns): S [0,128) | P0 [128,192) | P1 [192,256) | O [256, 256+d)
-// | P0 lo [384,448) | P1 lo [448,512) (the lo halves only in precise mode, where P
-// enters P V as two bf16 terms, hi = bf16(p) and lo = bf16(p - hi)).
-// The MMA warp issues S(n+1) as soon as the softmax has read S(n), so the score
-// product of the next tile overlaps the exponentials of the current one; P is
-// double-buffered so P V of tile n runs while tile n+1's softmax proceeds.
+// Tensor memory (512 columns): S0 [0,128) | S1 [128,256) | O [256, 256+d).  Key tile g
+// uses S buffer g & 1, and its P is written over that S (the softmax thread holds
+// its whole S row in registers by then): hi = bf16(p) in the buffer's first 64
+// columns and, in precise mode, where P enters P V as two bf16 terms, lo =
+// bf16(p - hi) in the next 64.  The score products run two key tiles ahead of the
+// P V products (S0 S1 PV0 S2 PV1 S3 ...): S(g+1) is complete while the softmax is
+// still on tile g, so the softmax never waits for a score product.  S(g+2) reuses
+// the buffer of P(g), so it is issued once P V(g) has completed (its commit).
 // The running max is rescaled lazily: O and the row sum are corrected only when
 // the max grows by more than 2^8 (all values stay finite and exact to rounding).
 #include "forge_internal.h"
@@ -45,9 +48,9 @@ constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
 // Which pairs of a row's exponentials go to the FMA-pipe polynomial (exp2_poly2)
-// instead of the MUFU unit.  None: with one softmax warp per SM sub-partition this
-// kernel is latency-bound rather than MUFU-bound, and the polynomial's extra
-// instructions measured slower at every share tried (3/8 to 6/8).
+// instead of the MUFU unit.  None: every share tried (1/8 to 6/8) measured slower;
+// the MUFU unit runs the 128 exponentials of a row in about 1.2K cycles, close to
+// its 1K-cycle bound, and the polynomial's extra instructions lengthen the rest.
 __device__ __forceinline__ constexpr bool use_poly_pair(int) { return false; }
 
 // wait sites (for the device error word)
@@ -70,8 +73,9 @@ struct FwdCfg {
     // 1 KB of slack for aligning the dynamic shared memory base to 1024 bytes.
     static constexpr int kSmemBytes = kOffBar + kBarBytes + 1024;
     // tensor memory columns
-    static constexpr uint32_t kColS = 0, kColP0 = 128, kColP1 = 192, kColO = 256;
-    static constexpr uint32_t kColPlo0 = 384, kColPlo1 = 448;
+    // two S buffers; tile g uses buffer g & 1, and its P (bf16, 64 columns; the lo
+    // half of precise mode in the next 64) is written over the S it came from
+    static constexpr uint32_t kColS0 = 0, kColBuf = 128, kColPlo = 64, kColO = 256;
     static constexpr uint32_t kTmemCols = 512;
     static constexpr uint32_t kIdescS = idesc_bf16_f32(128, 128, false, false);
     static constexpr uint32_t kIdescPV = idesc_bf16_f32(128, D, false, true);
@@ -82,10 +86,9 @@ struct FwdBarriers {
     uint64_t k_full[4];
     uint64_t v_full[4];
     uint64_t kv_empty[4];
-    uint64_t s_full;
-    uint64_t s_free;
-    uint64_t p_full;
-    uint64_t pv_done;
+    uint64_t s_full[2];  // per S buffer
+    uint64_t p_full[2];  // per S buffer (P is written over S)
+    uint64_t pv_done;    // every P V, in order
     uint64_t o_done, o_free;  // an item's O complete / read out of tensor memory
     uint64_t mma_final;
     uint32_t tmem_base;
@@ -137,9 +140,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             mbar_init(&bars->v_full[s], 1);
             mbar_init(&bars->kv_empty[s], 1);
         }
-        mbar_init(&bars->s_full, 1);
-        mbar_init(&bars->s_free, 4);
-        mbar_init(&bars->p_full, 4);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&bars->s_full[b], 1);
+            mbar_init(&bars->p_full[b], 4);
+        }
         mbar_init(&bars->pv_done, 1);
         mbar_init(&bars->o_done, 1);
         mbar_init(&bars->o_free, 4);
@@ -211,75 +215,101 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         // --------------------------------------------------------- MMA issuer
         // The whole warp runs this loop; one elected lane issues each MMA.
         {
-            const uint32_t tS = tmem + C::kColS;
             const uint32_t tO = tmem + C::kColO;
             const uint32_t q_addr = smem_u32(smem + C::kOffQ);
             // bit 13 of the instruction descriptor negates A: S = (-Q) K^T for scale < 0
             const uint32_t idesc_s = C::kIdescS | (negate_scores ? (1u << 13) : 0u);
-            bool ok = true;
-            // O += P(m) V(m); m counts key tiles over all items.  An item's first P V
-            // overwrites O, so it waits until the previous item's epilogue has read O.
-            auto issue_pv = [&](int m, bool first, int item) -> bool {
-                const int st = m % C::kStages;
-                if (!warp_wait(&bars->p_full, m & 1, kSitePFull, abort)) return false;
-                if (!warp_wait(&bars->v_full[st], (m / C::kStages) & 1, kSiteVFull, abort))
+            // Two cursors walk the CTA's key tiles over all items: the score products
+            // run two tiles ahead of the P V products, in the order
+            //   S(0) S(1) PV(0) S(2) PV(1) S(3) ...
+            // so S(g+1) is in its buffer while the softmax is still on tile g.
+            struct Cursor {
+                int item, n, n_tiles, g;
+                bool valid;
+            };
+            auto start = [&](Cursor& c) {
+                int bh_, qt_;
+                c.item = 0;
+                c.n = 0;
+                c.g = 0;
+                c.valid = item_of(0, bh_, qt_);
+                c.n_tiles = c.valid ? tiles_of(qt_) : 0;
+            };
+            auto advance = [&](Cursor& c) {
+                ++c.g;
+                if (++c.n == c.n_tiles) {
+                    int bh_, qt_;
+                    ++c.item;
+                    c.n = 0;
+                    c.valid = item_of(c.item, bh_, qt_);
+                    c.n_tiles = c.valid ? tiles_of(qt_) : 0;
+                }
+            };
+            // S(g) = Q K(g)^T into buffer g & 1, once P V(g-2) has read the P there
+            auto issue_s = [&](const Cursor& c) -> bool {
+                const int g = c.g;
+                const int st = g % C::kStages;
+                if (c.n == 0 && !warp_wait(&bars->q_full, c.item & 1, kSiteQ, abort)) return false;
+                if (!warp_wait(&bars->k_full[st], (g / C::kStages) & 1, kSiteKFull, abort))
                     return false;
-                if (first && item > 0 &&
-                    !warp_wait(&bars->o_free, (item - 1) & 1, kSiteOFree, abort))
+                if (g >= 2 && !warp_wait(&bars->pv_done, (g - 2) & 1, kSiteSFree, abort))
                     return false;
                 tc_fence_after();
-                const uint32_t tP = tmem + ((m & 1) ? C::kColP1 : C::kColP0);
-                const uint32_t tPlo = tmem + ((m & 1) ? C::kColPlo1 : C::kColPlo0);
+                const uint32_t tS = tmem + C::kColS0 + (g & 1) * C::kColBuf;
+                const uint32_t k_addr = smem_u32(smem + C::kOffK + st * C::kTileBytes);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t koff = (kk >> 2) * C::kChunkBytes + (kk & 3) * 32;
+                    const uint64_t adesc = sdesc_sw128(q_addr + koff, 16, 1024);
+                    const uint64_t bdesc = sdesc_sw128(k_addr + koff, 16, 1024);
+                    mma_ss_warp(tS, adesc, bdesc, idesc_s, kk > 0 ? 1u : 0u);
+                }
+                mma_commit_warp(&bars->s_full[g & 1]);
+                // the item's last score product is the last reader of Q
+                if (c.n == c.n_tiles - 1) mma_commit_warp(&bars->q_empty);
+                return true;
+            };
+            // O += P(g) V(g).  An item's first P V overwrites O, so it waits until the
+            // previous item's epilogue has read O.
+            auto issue_pv = [&](const Cursor& c) -> bool {
+                const int g = c.g;
+                const int st = g % C::kStages;
+                if (!warp_wait(&bars->p_full[g & 1], (g >> 1) & 1, kSitePFull, abort)) return false;
+                if (!warp_wait(&bars->v_full[st], (g / C::kStages) & 1, kSiteVFull, abort))
+                    return false;
+                if (c.n == 0 && c.item > 0 &&
+                    !warp_wait(&bars->o_free, (c.item - 1) & 1, kSiteOFree, abort))
+                    return false;
+                tc_fence_after();
+                const uint32_t tP = tmem + C::kColS0 + (g & 1) * C::kColBuf;
                 const uint32_t v_addr = smem_u32(smem + C::kOffV + st * C::kTileBytes);
 #pragma unroll
                 for (int kk = 0; kk < kTile / 16; ++kk) {
                     // B = V tile, MN-major: 16 keys = 2 x 8-row groups of 1024 bytes
                     const uint64_t bdesc = sdesc_sw128(v_addr + kk * 2048, C::kChunkBytes, 1024);
-                    mma_ts_warp(tO, tP + kk * 8, bdesc, C::kIdescPV, (!first || kk > 0) ? 1u : 0u);
-                    if (PRECISE) mma_ts_warp(tO, tPlo + kk * 8, bdesc, C::kIdescPV, 1u);
+                    mma_ts_warp(tO, tP + kk * 8, bdesc, C::kIdescPV, (c.n > 0 || kk > 0) ? 1u : 0u);
+                    if (PRECISE) mma_ts_warp(tO, tP + C::kColPlo + kk * 8, bdesc, C::kIdescPV, 1u);
                 }
                 mma_commit_warp(&bars->pv_done);
                 mma_commit_warp(&bars->kv_empty[st]);
+                if (c.n == c.n_tiles - 1) mma_commit_warp(&bars->o_done);
                 return true;
             };
-            int g = 0;  // key tiles so far (all items)
-            int bh, qt;
-            for (int item = 0; ok && item_of(item, bh, qt); ++item) {
-                if (!warp_wait(&bars->q_full, item & 1, kSiteQ, abort)) {
-                    ok = false;
-                    break;
+            Cursor cs, cp;
+            start(cs);
+            start(cp);
+            bool ok = true;
+            for (int i = 0; ok && i < 2 && cs.valid; ++i) {
+                ok = issue_s(cs);
+                advance(cs);
+            }
+            while (ok && cp.valid) {
+                ok = issue_pv(cp);
+                advance(cp);
+                if (ok && cs.valid) {
+                    ok = issue_s(cs);
+                    advance(cs);
                 }
-                const int n_tiles = tiles_of(qt);
-                for (int n = 0; ok && n < n_tiles; ++n, ++g) {
-                    const int st = g % C::kStages;
-                    if (!warp_wait(&bars->k_full[st], (g / C::kStages) & 1, kSiteKFull, abort)) {
-                        ok = false;
-                        break;
-                    }
-                    // the S columns: the softmax has read the previous S (any item)
-                    if (g > 0 && !warp_wait(&bars->s_free, (g - 1) & 1, kSiteSFree, abort)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    const uint32_t k_addr = smem_u32(smem + C::kOffK + st * C::kTileBytes);
-#pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint32_t koff = (kk >> 2) * C::kChunkBytes + (kk & 3) * 32;
-                        const uint64_t adesc = sdesc_sw128(q_addr + koff, 16, 1024);
-                        const uint64_t bdesc = sdesc_sw128(k_addr + koff, 16, 1024);
-                        mma_ss_warp(tS, adesc, bdesc, idesc_s, kk > 0 ? 1u : 0u);
-                    }
-                    mma_commit_warp(&bars->s_full);
-                    // the item's last score product is the last reader of Q
-                    if (n == n_tiles - 1) mma_commit_warp(&bars->q_empty);
-                    if (n > 0 && !issue_pv(g - 1, n == 1, item)) {
-                        ok = false;
-                        break;
-                    }
-                }
-                if (ok) ok = issue_pv(g - 1, n_tiles == 1, item);
-                if (ok) mma_commit_warp(&bars->o_done);
             }
             // every MMA this thread issued must retire before tensor memory is freed
             mma_commit_warp(&bars->mma_final);
@@ -289,7 +319,6 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         // ------------------------------------------------------------ softmax
         const uint32_t row = ((warp & 3) << 5) + lane;  // TMEM lane owned by this thread
         const uint32_t lane_off = ((warp & 3) << 5) << 16;
-        const uint32_t tS = tmem + lane_off + C::kColS;
         const uint32_t tO = tmem + lane_off + C::kColO;
         bool ok = true;
         int g0 = 0;  // key tiles before this item (all items)
@@ -302,7 +331,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         for (int n = 0; n < n_tiles; ++n) {
             const int g = g0 + n;
             const int j = causal ? qt - n : n_kvtiles_total - 1 - n;
-            if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full, g & 1, kSiteSFull, abort))) {
+            const uint32_t tS = tmem + lane_off + C::kColS0 + (g & 1) * C::kColBuf;
+            if (!__all_sync(0xffffffffu,
+                            mbar_wait(&bars->s_full[g & 1], (g >> 1) & 1, kSiteSFull, abort))) {
                 ok = false;
                 break;
             }
@@ -311,9 +342,6 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 #pragma unroll
             for (int c = 0; c < kTile / 32; ++c) tmem_ld32(tS + c * 32, sraw + c * 32);
             tmem_wait_ld();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars->s_free);
 
             // Row max of the raw scores over the keys this row may see.  scale_log2 is
             // >= 0 (a negative scale is applied by negating Q in the MMA), so the max
@@ -374,8 +402,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             }
 
             // P = exp2(s * scale_log2 - m), row sum, pack to bf16 pairs, store to TMEM
-            const uint32_t tP = tmem + lane_off + ((g & 1) ? C::kColP1 : C::kColP0);
-            const uint32_t tPlo = tmem + lane_off + ((g & 1) ? C::kColPlo1 : C::kColPlo0);
+            // P over the S it came from (this thread has all of its S row in registers)
+            const uint32_t tP = tS;
+            const uint32_t tPlo = tS + C::kColPlo;
             const float neg_m = -m_run;
             const float2 sl2 = make_float2(scale_log2, scale_log2);
             const float2 nm2 = make_float2(neg_m, neg_m);
@@ -415,7 +444,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bars->p_full);
+            if (lane == 0) mbar_arrive(&bars->p_full[g & 1]);
         }
 
         if (!ok) break;

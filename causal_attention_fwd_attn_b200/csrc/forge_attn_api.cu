@@ -19,7 +19,6 @@ cudaError_t read_and_clear_device_error(unsigned int* value, cudaStream_t stream
     if (e != cudaSuccess) return e;
     unsigned int v = 0;
     if ((e = read_and_clear_device_error_fwd(&v)) != cudaSuccess) return e;
-    if ((e = read_and_clear_device_error_fwd_pair(&v)) != cudaSuccess) return e;
     if ((e = read_and_clear_device_error_bwd(&v)) != cudaSuccess) return e;
     if ((e = read_and_clear_device_error_probe(&v)) != cudaSuccess) return e;
     *value = v;
@@ -144,12 +143,6 @@ int forge_attn_fwd_ex(const void* q, const void* k, const void* v, void* o, floa
     if ((s = make_map_bf16(&tq, q, d, T, BH)) != FORGE_ATTN_OK) return s;
     if ((s = make_map_bf16(&tk, k, d, T, BH)) != FORGE_ATTN_OK) return s;
     if ((s = make_map_bf16(&tv, v, d, T, BH)) != FORGE_ATTN_OK) return s;
-    const bool precise = (flags & FORGE_ATTN_PRECISE) != 0;
-    // d = 64: two query tiles per work item (measured faster); d = 128 and precise
-    // mode: one query tile per CTA
-    if (d == 64 && !precise)
-        return cuda_status(launch_attn_fwd_pair(tq, tk, tv, o, lse, (int)BH, T, d, scale, causal,
-                                                o_f32, static_cast<cudaStream_t>(stream)));
     return cuda_status(launch_attn_fwd(tq, tk, tv, o, lse, (int)BH, T, d, scale, causal,
                                        o_f32, (flags & FORGE_ATTN_PRECISE) != 0,
                                        static_cast<cudaStream_t>(stream)));

@@ -19,11 +19,6 @@ cudaError_t launch_attn_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const 
                             void* o, float* lse, int BH, int T, int d, float scale, int causal,
                             int o_f32, int precise, cudaStream_t stream);
 
-// The two-query-tile persistent forward (no precise mode); o is bf16 or fp32 (o_f32).
-cudaError_t launch_attn_fwd_pair(const CUtensorMap& tq, const CUtensorMap& tk,
-                                 const CUtensorMap& tv, void* o, float* lse, int BH, int T, int d,
-                                 float scale, int causal, int o_f32, cudaStream_t stream);
-
 // Row statistics of the backward: fp32 [2][B*H][t_pad], t_pad = 128 * ceil(T / 128).
 cudaError_t launch_bwd_preprocess(const void* o, const void* dO, const float* lse,
                                   float* rowstats, float* dq_accum, int BH, int T, int d,
@@ -47,7 +42,6 @@ cudaError_t launch_probe_wait_timeout(unsigned long long limit_ns, cudaStream_t 
 // Device error words, one per translation unit with kernels: each reader ORs its
 // word into *value and clears it (the stream must have been synchronised).
 cudaError_t read_and_clear_device_error_fwd(unsigned int* value);
-cudaError_t read_and_clear_device_error_fwd_pair(unsigned int* value);
 cudaError_t read_and_clear_device_error_bwd(unsigned int* value);
 cudaError_t read_and_clear_device_error_probe(unsigned int* value);
 
