@@ -111,7 +111,7 @@ size_t forge_attn_bwd_workspace_size(int B, int H, int T, int d);
  * `o` is bf16 here (fp32 with forge_attn_bwd_ex and FORGE_ATTN_O_IN_F32).
  * Launch sequence on `stream`: the pre-pass (row statistics; also zeroes the dQ
  * accumulator), the dK/dV kernel over key tiles (dQ partials added into the fp32
- * accumulator by TMA reduce-add or fp32 vector reductions), and the dQ conversion.
+ * accumulator by TMA reduce-add), and the dQ conversion.
  */
 int forge_attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO,
                    const float* lse, void* dq, void* dk, void* dv, void* workspace,
@@ -136,8 +136,8 @@ int forge_attn_bwd_ex(const void* q, const void* k, const void* v, const void* o
  *   padding rows t >= T; and dq_accum (fp32 [B][H][T][d]) set to zero unless it is
  *   NULL.  flags: FORGE_ATTN_O_IN_F32 (o is fp32).
  * forge_attn_bwd_dkdv: recomputes P per key tile from the row statistics, writes dk
- *   and dv, and adds scale * dS K into dq_accum (TMA reduce-add or fp32 vector
- *   reductions).  flags: FORGE_ATTN_OUT_F32 (dk, dv fp32), FORGE_ATTN_PRECISE.
+ *   and dv, and adds scale * dS K into dq_accum (TMA reduce-add).  flags:
+ *   FORGE_ATTN_OUT_F32 (dk, dv fp32), FORGE_ATTN_PRECISE.
  * forge_attn_bwd_dq_convert: dq = bf16(dq_accum).  Only needed for bf16 dq.
  */
 int forge_attn_bwd_preprocess(const void* o, const void* dO, const float* lse, float* rowstats,
