@@ -925,14 +925,10 @@ cudaError_t launch_dkdv_dp(const CUtensorMap& tq, const CUtensorMap& tk, const C
                            float* dq_accum, void* dk, void* dv, int BH, int T, float scale,
                            int causal, int grad_f32, cudaStream_t stream) {
     using C = BwdCfg<D, PRECISE>;
-    static bool configured = false;
-    if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(attn_bwd_dkdv_kernel<D, PRECISE>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             C::kSmemBytes);
-        if (e != cudaSuccess) return e;
-        configured = true;
-    }
+    static std::atomic<unsigned long long> configured{0};
+    cudaError_t e =
+        set_max_dynamic_smem(attn_bwd_dkdv_kernel<D, PRECISE>, C::kSmemBytes, configured);
+    if (e != cudaSuccess) return e;
     const int n_kvtiles = (T + kTile - 1) / kTile;
     const long long items = (long long)BH * n_kvtiles;
     if (items > 0x7fffffff) return cudaErrorInvalidValue;

@@ -525,14 +525,9 @@ cudaError_t launch_fwd_dp(const CUtensorMap& tq, const CUtensorMap& tk, const CU
                           void* o, float* lse, int BH, int T, float scale, int causal, int o_f32,
                           cudaStream_t stream) {
     using C = FwdCfg<D>;
-    static bool configured = false;
-    if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D, PRECISE>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             C::kSmemBytes);
-        if (e != cudaSuccess) return e;
-        configured = true;
-    }
+    static std::atomic<unsigned long long> configured{0};
+    cudaError_t e = set_max_dynamic_smem(attn_fwd_kernel<D, PRECISE>, C::kSmemBytes, configured);
+    if (e != cudaSuccess) return e;
     const int n_qtiles = (T + kTile - 1) / kTile;
     const int n_items = BH * n_qtiles;
     const int grid = n_items < sm_count() ? n_items : sm_count();

@@ -7,10 +7,29 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <atomic>
+
 namespace forge {
 
 // Tile geometry common to all attention kernels: 128 query rows x 128 keys.
 constexpr int kTile = 128;
+
+// Raises `kernel`'s dynamic shared memory limit to `bytes` on the current device.
+// The attribute is per device, so `done` keeps one bit per device already set
+// (devices 64 and up are set on every call).  Concurrent first calls may both set
+// it, which is harmless.
+template <typename Kernel>
+cudaError_t set_max_dynamic_smem(Kernel* kernel, int bytes,
+                                 std::atomic<unsigned long long>& done) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const unsigned long long bit = (dev >= 0 && dev < 64) ? (1ull << dev) : 0ull;
+    if (bit != 0 && (done.load(std::memory_order_relaxed) & bit) != 0) return cudaSuccess;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess) done.fetch_or(bit, std::memory_order_relaxed);
+    return e;
+}
 
 // Launchers.  Tensor maps describe bf16 [B*H][T][d] tensors with a
 // {64, 128, 1} box and 128-byte swizzle.

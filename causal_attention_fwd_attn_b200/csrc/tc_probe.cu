@@ -151,13 +151,9 @@ __global__ void probe_wait_timeout_kernel(unsigned long long limit_ns) {
 
 cudaError_t launch_probe_mma(const CUtensorMap& ta, const CUtensorMap& tb, const void* a_raw,
                              float* d_out, int N, int K, int mode, cudaStream_t stream) {
-    static bool configured = false;
-    if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(
-            probe_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kProbeSmem);
-        if (e != cudaSuccess) return e;
-        configured = true;
-    }
+    static std::atomic<unsigned long long> configured{0};
+    cudaError_t e = set_max_dynamic_smem(probe_mma_kernel, kProbeSmem, configured);
+    if (e != cudaSuccess) return e;
     probe_mma_kernel<<<1, kProbeThreads, kProbeSmem, stream>>>(
         ta, tb, static_cast<const __nv_bfloat16*>(a_raw), d_out, N, K, mode);
     return cudaGetLastError();
