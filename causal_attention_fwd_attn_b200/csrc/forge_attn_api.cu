@@ -83,8 +83,8 @@ int check_shape(int B, int H, int T, int d) {
     if (d != 64 && d != 128) return FORGE_ATTN_ERR_UNSUPPORTED;
     const long long n = (long long)B * H * T * d;
     if (n >= (1ll << 31)) return FORGE_ATTN_ERR_UNSUPPORTED;
+    // with d >= 64 this also keeps B*H and every row index (< 2^25) well inside int
     if ((long long)B * H > 0x7fffffffll) return FORGE_ATTN_ERR_UNSUPPORTED;
-    if ((T + 127) / 128 > 65535) return FORGE_ATTN_ERR_UNSUPPORTED;
     return FORGE_ATTN_OK;
 }
 
