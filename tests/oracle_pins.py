@@ -12,13 +12,19 @@ None of these re-types the oracle's own formulas:
   * closed forms: Q = 0 gives uniform weights over the allowed keys, T = 1 gives
     O = v0, LSE = scale q0.k0 and zero dQ, dK with dV = dO;
   * invariants: softmax rows sum to 1, row i ignores keys > i under the causal
-    mask, each row of dS sums to 0, and dO = 0 gives zero gradients.
+    mask, each row of dS sums to 0, and dO = 0 gives zero gradients;
+  * worked examples (tests/golden/): every forward and backward output of a small
+    case stated as an exact expression derived by hand.
 """
 from __future__ import annotations
 
+import glob
 import math
+import os
 
 import numpy as np
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
 
 
 def brute_fwd(q, k, v, scale, causal):
@@ -174,6 +180,70 @@ def check_rows_match_full(orc, T=11, d=3, causal=1, scale=0.66, seed=9):
     return None
 
 
+def _golden_eval(expr: str) -> float:
+    return float(eval(expr, {"__builtins__": {}}, {"log": math.log}))
+
+
+def _golden_split(rhs: str):
+    # entries are separated by commas outside parentheses
+    out, depth, cur = [], 0, ""
+    for ch in rhs:
+        if ch == "," and depth == 0:
+            out.append(cur)
+            cur = ""
+            continue
+        depth += ch == "("
+        depth -= ch == ")"
+        cur += ch
+    out.append(cur)
+    return [_golden_eval(e.strip()) for e in out if e.strip()]
+
+
+def golden_fixtures():
+    return sorted(glob.glob(os.path.join(GOLDEN, "worked_*.txt")))
+
+
+def load_golden(path):
+    """A worked example: {name: array}; "name = ..." is a vector, "name[i] = ..."
+    row i of a matrix; entries are exact expressions (log = natural log)."""
+    vec, mat = {}, {}
+    with open(path) as f:
+        for line in f:
+            line = line.split("#", 1)[0].strip()
+            if not line:
+                continue
+            lhs, rhs = (x.strip() for x in line.split("=", 1))
+            vals = _golden_split(rhs)
+            if "[" in lhs:
+                name, idx = lhs[:-1].split("[")
+                mat.setdefault(name, {})[int(idx)] = vals
+            else:
+                vec[lhs] = vals
+    for name, rows in mat.items():
+        vec[name] = [rows[i] for i in range(len(rows))]
+    return {k: np.array(v, dtype=np.float64) for k, v in vec.items()}
+
+
+def check_worked_examples(orc, tol=1e-13):
+    """The oracle's P, LSE, O, D, dS, dV, dK, dQ against every worked example."""
+    paths = golden_fixtures()
+    if not paths:
+        return "no worked examples found"
+    for path in paths:
+        fx = load_golden(path)
+        scale, causal = float(fx["scale"][0]), int(fx["causal"][0])
+        q, k, v, dO = (fx[n].reshape(-1, 1) for n in ("q", "k", "v", "dO"))
+        o, lse, p = orc.fwd_head(q, k, v, scale, causal, want_p=True)
+        dq, dk, dv, ds, dvec = orc.bwd_head(q, k, v, dO, scale, causal, want_ds=True)
+        got = {"p": p, "lse": lse, "o": o[:, 0], "D": dvec, "ds": ds, "dv": dv[:, 0],
+               "dk": dk[:, 0], "dq": dq[:, 0]}
+        for name, value in got.items():
+            err = float(np.max(np.abs(value - fx[name])))
+            if not err <= tol:
+                return f"worked example {os.path.basename(path)}: {name} off by {err:.3g}"
+    return None
+
+
 def all_checks(orc):
     """Run every pin; return the list of failure messages (empty when all pass)."""
     out = []
@@ -192,6 +262,7 @@ def all_checks(orc):
         (check_zero_dO, {}),
         (check_rows_match_full, dict(causal=1)),
         (check_rows_match_full, dict(causal=0)),
+        (check_worked_examples, {}),
     ]:
         try:
             msg = fn(orc, **kw)

@@ -38,3 +38,20 @@ def test_pins_catch_mutation(name, tmp_path):
     lib = oracle.build(path, os.path.join(tmp_path, "libmutant.so"))
     failures = pins.all_checks(oracle.Oracle(lib))
     assert failures, f"no pin caught: {name}"
+
+
+# Every planted mistake in the full-matrix path (all but the row sampler's) is also
+# caught by the hand-derived worked examples alone.
+@pytest.mark.parametrize("name", sorted(n for n in MUTATIONS if not n.startswith("row sampler")))
+def test_worked_examples_alone_catch_mutation(name, tmp_path):
+    src = open(oracle.SOURCE).read()
+    old, new = MUTATIONS[name]
+    path = os.path.join(tmp_path, "mutant.c")
+    with open(path, "w") as f:
+        f.write(src.replace(old, new))
+    lib = oracle.build(path, os.path.join(tmp_path, "libmutant.so"))
+    try:
+        msg = pins.check_worked_examples(oracle.Oracle(lib))
+    except Exception as e:  # a crash in a mutated oracle counts as caught
+        msg = repr(e)
+    assert msg, f"the worked examples did not catch: {name}"
