@@ -3,8 +3,8 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 
 One step is one pass of the whole path over one batch of the workload: the
-forward (one kernel) and the backward (D pre-pass, dK/dV kernel with dQ atomics,
-dQ conversion), all through the C ABI.  FLOPs are the causal counts (forward
+forward (one kernel) and the backward (D pre-pass, dK/dV kernel with the dQ partials
+added by TMA reduce-add into an fp32 accumulator, dQ conversion), all through the C ABI.  FLOPs are the causal counts (forward
 2*B*H*T^2*d, backward 2.5x that).  Inputs are synthetic (seeded bf16 Gaussian
 with the workload's shape and distribution) and resident in HBM; successive
 steps rotate over several input sets whose total is larger than the 126 MB L2.
@@ -14,7 +14,9 @@ every rank runs its own batch (independent heads, no collective on the data
 path: weak scaling); the time is the max over ranks.
 
 --impl reference times the fp64 CPU oracle instead (the slow, plain reference
-this library is checked against) on a bounded sample of the workload.
+this library is checked against): every step is a bounded sample of whole heads of
+the workload, sized so the run takes about --reference-seconds in all (default 150 s
+over 3 warm-up and 50 timed steps; a step is never less than one head pass).
 """
 from __future__ import annotations
 
@@ -394,20 +396,29 @@ def run_e2e(args, w, ci, dev, stream, o, lse, dq, dk, dv, ws, world):
 
 
 # ---------------------------------------------------------- CPU oracle leg ----
-def oracle_sample(w, ci, budget_s, threads):
-    """Time the fp64 oracle (forward + backward, the full T x T definition) on as
-    many heads of the workload as fit in about budget_s seconds on `threads` host
-    threads.  Returns (TFLOP/s in the workload's causal-FLOP convention, cores,
-    sample description)."""
-    import oracle
+class OracleSampler:
+    """Times the fp64 oracle (forward + backward, the full T x T definition) on whole
+    heads of a workload, on the host's cores.  The inputs are prepared and the time
+    of one head pass on one thread is measured once; each sample then runs as many
+    head passes as fit its time budget (at least one), one head per thread, cycling
+    through the workload's heads."""
 
-    orc = oracle.default()
-    x = wl.make_inputs(ci)
-    heads = [(b, h) for b in range(w.B) for h in range(w.H)]
-    f = {n: x[n].double().numpy() for n in x}
+    def __init__(self, w, ci, threads):
+        import oracle
 
-    def run(hs):
+        self.w = w
+        self.orc = oracle.default()
+        x = wl.make_inputs(ci)
+        self.f = {n: x[n].double().numpy() for n in x}
+        self.heads = [(b, h) for b in range(w.B) for h in range(w.H)]
+        self.threads = max(1, threads)
+        self.cursor = 0
+        self.t_head = max(self._run(self.heads[:1], 1), 1e-4)
+
+    def _run(self, hs, threads):
         from concurrent.futures import ThreadPoolExecutor
+
+        f, w, orc = self.f, self.w, self.orc
 
         def one(bh):
             b, h = bh
@@ -420,34 +431,42 @@ def oracle_sample(w, ci, budget_s, threads):
             list(ex.map(one, hs))
         return time.perf_counter() - t
 
-    # calibrate on one head per thread, then scale the sample to the budget (whole
-    # passes over the workload's heads are repeated when the workload is small)
-    first = heads[:min(threads, len(heads))]
-    t_first = run(first)
-    per_head = max(t_first, 1e-3) / len(first)
-    n = max(len(first), int(budget_s / per_head))
-    sample = [heads[j % len(heads)] for j in range(n)]
-    elapsed = run(sample)
-    flops_per_head = w.flops_total() / w.BH
-    value = flops_per_head * len(sample) / elapsed / 1e12
-    desc = (f"{len(sample)} head passes over the {w.BH} heads of {w.name} (T={w.T}, d={w.d}), "
-            f"fp64 oracle forward + backward, {elapsed:.1f} s on {threads} threads")
-    return value, threads, desc, elapsed
+    def sample(self, budget_s):
+        """(TFLOP/s in the workload's causal-FLOP convention, threads used,
+        description, elapsed seconds) of one sample of about budget_s seconds."""
+        w = self.w
+        n = max(1, int(budget_s / self.t_head * self.threads))
+        threads = min(self.threads, n)
+        hs = [self.heads[(self.cursor + j) % len(self.heads)] for j in range(n)]
+        self.cursor = (self.cursor + n) % len(self.heads)
+        elapsed = self._run(hs, threads)
+        value = w.flops_total() / w.BH * n / elapsed / 1e12
+        desc = (f"{n} head passes over the {w.BH} heads of {w.name} (T={w.T}, d={w.d}), "
+                f"fp64 oracle forward + backward, {elapsed:.2f} s on {threads} threads")
+        return value, threads, desc, elapsed
+
+
+def oracle_sample(w, ci, budget_s, threads):
+    """One oracle sample of about budget_s seconds (see OracleSampler)."""
+    return OracleSampler(w, ci, threads).sample(budget_s)
 
 
 def run_reference(args, rank, world):
+    """The oracle as it stands, timed on the host cores: each of the warm-up and timed
+    steps is one bounded sample of the workload, sized so that the whole run takes
+    about args.reference_seconds (a step is never less than one head pass)."""
     if rank != 0:
         return None
     ci, w = find_workload(args.workload)
-    threads = os.cpu_count() or 1
-    steps_v = []
-    descs = []
-    budget = max(2.0, 150.0 / max(1, args.steps + args.warmup))
+    sampler = OracleSampler(w, ci, os.cpu_count() or 1)
+    budget = args.reference_seconds / max(1, args.steps + args.warmup)
+    steps_v, descs, threads = [], [], 1
     for i in range(args.warmup + args.steps):
-        v, cores, desc, el = oracle_sample(w, ci, budget, threads)
+        v, cores, desc, el = sampler.sample(budget)
         if i >= args.warmup:
             steps_v.append((v, el))
             descs.append(desc)
+            threads = max(threads, cores)
     value = statistics.median(v for v, _ in steps_v)
     ms = statistics.median(el for _, el in steps_v) * 1e3
     return {
@@ -470,14 +489,25 @@ def main():
     ap = argparse.ArgumentParser(description=__doc__,
                                  formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
-    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=None,
+                    help="timed steps (default 2000; 50 for --impl reference)")
+    ap.add_argument("--warmup", type=int, default=None,
+                    help="untimed warm-up steps, at least 3 (default 20; 3 for --impl reference)")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-baseline-seconds", type=float, default=12.0,
                     help="budget of the oracle sample timed beside the GPU run (rank 0, N=1)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--reference-seconds", type=float, default=150.0,
+                    help="--impl reference: total oracle time over all warm-up and timed steps "
+                         "(each step is at least one head pass)")
     args = ap.parse_args()
+    # the reference arm's steps are oracle samples of whole heads (about 0.3 s each at
+    # the gpt2-small shape on one core), so its default run is shorter
+    if args.steps is None:
+        args.steps = 50 if args.impl == "reference" else 2000
+    if args.warmup is None:
+        args.warmup = 3 if args.impl == "reference" else 20
     if args.warmup < 3:
         raise SystemExit("--warmup must be at least 3")
 
