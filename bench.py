@@ -398,10 +398,10 @@ def run_e2e(args, w, ci, dev, stream, o, lse, dq, dk, dv, ws, world):
 # ---------------------------------------------------------- CPU oracle leg ----
 class OracleSampler:
     """Times the fp64 oracle (forward + backward, the full T x T definition) on whole
-    heads of a workload, on the host's cores.  The inputs are prepared and the time
-    of one head pass on one thread is measured once; each sample then runs as many
-    head passes as fit its time budget (at least one), one head per thread, cycling
-    through the workload's heads."""
+    heads of a workload, on the host's cores.  The inputs are prepared and the rate
+    of head passes with every thread busy is measured once; each sample then runs as
+    many head passes as fit its time budget at that rate (at least one), one head per
+    thread, cycling through the workload's heads."""
 
     def __init__(self, w, ci, threads):
         import oracle
@@ -413,7 +413,8 @@ class OracleSampler:
         self.heads = [(b, h) for b in range(w.B) for h in range(w.H)]
         self.threads = max(1, threads)
         self.cursor = 0
-        self.t_head = max(self._run(self.heads[:1], 1), 1e-4)
+        nb = min(self.threads, len(self.heads))
+        self.rate = nb / max(self._run(self.heads[:nb], nb), 1e-4)  # head passes per second
 
     def _run(self, hs, threads):
         from concurrent.futures import ThreadPoolExecutor
@@ -435,7 +436,7 @@ class OracleSampler:
         """(TFLOP/s in the workload's causal-FLOP convention, threads used,
         description, elapsed seconds) of one sample of about budget_s seconds."""
         w = self.w
-        n = max(1, int(budget_s / self.t_head * self.threads))
+        n = max(1, int(budget_s * self.rate))
         threads = min(self.threads, n)
         hs = [self.heads[(self.cursor + j) % len(self.heads)] for j in range(n)]
         self.cursor = (self.cursor + n) % len(self.heads)
@@ -502,8 +503,8 @@ def main():
                     help="--impl reference: total oracle time over all warm-up and timed steps "
                          "(each step is at least one head pass)")
     args = ap.parse_args()
-    # the reference arm's steps are oracle samples of whole heads (about 0.3 s each at
-    # the gpt2-small shape on one core), so its default run is shorter
+    # the reference arm's steps are oracle samples of whole heads (one head pass takes
+    # about 0.3 s at the gpt2-small shape on one core), so its default run is shorter
     if args.steps is None:
         args.steps = 50 if args.impl == "reference" else 2000
     if args.warmup is None:
