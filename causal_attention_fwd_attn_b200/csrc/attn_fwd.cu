@@ -72,6 +72,7 @@ struct FwdCfg {
     static constexpr int kBarBytes = 256;
     // 1 KB of slack for aligning the dynamic shared memory base to 1024 bytes.
     static constexpr int kSmemBytes = kOffBar + kBarBytes + 1024;
+    static_assert(kSmemBytes <= 232448, "shared memory budget");
     // tensor memory columns
     // two S buffers; tile g uses buffer g & 1, and its P (bf16, 64 columns; the lo
     // half of precise mode in the next 64) is written over the S it came from
@@ -109,6 +110,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                     int n_qtiles, int n_items, float scale_log2, int negate_scores, int causal,
                     int o_f32) {
     using C = FwdCfg<D>;
+    static_assert(sizeof(FwdBarriers) <= C::kBarBytes, "barrier block");
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
