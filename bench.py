@@ -287,61 +287,67 @@ def run_ours(args, rank, world, local_rank):
     # ---- end to end through the C ABI with host buffers (pinned) ----------------
     e2e = run_e2e(args, w, ci, dev, stream, o, lse, dq, dk, dv, ws, world)
 
-    result = None
-    if rank == 0:
-        peaks = measured_peaks()
-        flops = w.flops_total()
-        value = job_tflops(flops, args.steps, world, max_ms)
-        dkdv_flops = w.flops_bwd()
-        achieved = dkdv_flops / (avg["dkdv"] * 1e-3) / 1e12
-        dominant = max(avg, key=avg.get)
-        traffic = recorded_traffic("attn_bwd_dkdv", w.name)
-        result = {
-            "metric": METRIC,
-            "value": round(value, 2),
-            "unit": UNIT,
-            "n_gpus": world,
-            "steps": args.steps,
-            "warmup": args.warmup,
-            "ms_per_step": round(max_ms / args.steps, 4),
-            "higher_is_better": True,
-            "scaling": "weak",
-            "vs_baseline": None,
-            "dtype": "bf16",
-            "data": "synthetic",
-            "config": {
-                "workload": w.name, "B": B, "H": H, "T": T, "d": d, "causal": w.causal,
-                "scale": "1/sqrt(d)", "inputs": "seeded iid Gaussian bf16, resident in HBM",
-                "l2": f"rotating {n_sets} input sets, {n_sets * set_bytes / 2**20:.0f} MiB of "
-                      f"inputs > 126 MB L2",
-                "parallelism": f"replicas x{world} (independent heads per GPU)",
-            },
-            "pct_of_peak": {"measured_bf16": round(100 * value / world / peaks["bf16_tflops"], 2),
-                            "spec_2250": round(100 * value / world / 2250.0, 2)},
-            "fwd_ms": round(avg["fwd"], 4),
-            "bwd_ms": round(avg["pre"] + avg["dkdv"] + avg["cvt"], 4),
-            "kernel_ms": {k: round(v, 4) for k, v in avg.items()},
-            "fwd_tflops": round(w.flops_fwd() / (avg["fwd"] * 1e-3) / 1e12, 1),
-            "bwd_tflops": round(w.flops_bwd() / ((avg["pre"] + avg["dkdv"] + avg["cvt"]) * 1e-3)
-                                / 1e12, 1),
-            "roofline": {
-                "kernel": "attn_bwd_dkdv",
-                "bound": "tensor",
-                "achieved": round(achieved, 1),
-                "peak": peaks["bf16_tflops"],
-                "unit": "TFLOP/s",
-                "frac": round(achieved / peaks["bf16_tflops"], 4),
-                "traffic": traffic,
-                "peak_source": f"{peaks['source']} bf16_tflops (burst)",
-                "dominant_by_time": dominant,
-                "algorithmic_flops_per_launch": dkdv_flops,
-            },
-            "clocks": clk,
-            "e2e": e2e,
-            "gpu_launches": launches_per_step * args.steps,
-            "library": os.path.relpath(_lib.library_path(), ROOT),
-        }
-    return result
+    if rank != 0:
+        return None
+    return ours_line(w, args.steps, args.warmup, world, max_ms, avg, clk, e2e,
+                     launches_per_step, n_sets, set_bytes, measured_peaks(),
+                     recorded_traffic("attn_bwd_dkdv", w.name),
+                     os.path.relpath(_lib.library_path(), ROOT))
+
+
+def ours_line(w, steps, warmup, world, max_ms, avg, clk, e2e, launches_per_step, n_sets,
+              set_bytes, peaks, traffic, library):
+    """The JSON line of the GPU arm from its measurements: max_ms is the slowest
+    rank's time for `steps` steps; avg holds each kernel's mean CUDA-event time (ms)
+    per launch ("fwd", "pre", "dkdv", "cvt")."""
+    value = job_tflops(w.flops_total(), steps, world, max_ms)
+    bwd_ms = avg["pre"] + avg["dkdv"] + avg["cvt"]
+    dkdv_flops = w.flops_bwd()
+    achieved = dkdv_flops / (avg["dkdv"] * 1e-3) / 1e12
+    return {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": UNIT,
+        "n_gpus": world,
+        "steps": steps,
+        "warmup": warmup,
+        "ms_per_step": round(max_ms / steps, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {
+            "workload": w.name, "B": w.B, "H": w.H, "T": w.T, "d": w.d, "causal": w.causal,
+            "scale": "1/sqrt(d)", "inputs": "seeded iid Gaussian bf16, resident in HBM",
+            "l2": f"rotating {n_sets} input sets, {n_sets * set_bytes / 2**20:.0f} MiB of "
+                  f"inputs > 126 MB L2",
+            "parallelism": f"replicas x{world} (independent heads per GPU)",
+        },
+        "pct_of_peak": {"measured_bf16": round(100 * value / world / peaks["bf16_tflops"], 2),
+                        "spec_2250": round(100 * value / world / 2250.0, 2)},
+        "fwd_ms": round(avg["fwd"], 4),
+        "bwd_ms": round(bwd_ms, 4),
+        "kernel_ms": {k: round(v, 4) for k, v in avg.items()},
+        "fwd_tflops": round(w.flops_fwd() / (avg["fwd"] * 1e-3) / 1e12, 1),
+        "bwd_tflops": round(w.flops_bwd() / (bwd_ms * 1e-3) / 1e12, 1),
+        "roofline": {
+            "kernel": "attn_bwd_dkdv",
+            "bound": "tensor",
+            "achieved": round(achieved, 1),
+            "peak": peaks["bf16_tflops"],
+            "unit": "TFLOP/s",
+            "frac": round(achieved / peaks["bf16_tflops"], 4),
+            "traffic": traffic,
+            "peak_source": f"{peaks['source']} bf16_tflops (burst)",
+            "dominant_by_time": max(avg, key=avg.get),
+            "algorithmic_flops_per_launch": dkdv_flops,
+        },
+        "clocks": clk,
+        "e2e": e2e,
+        "gpu_launches": launches_per_step * steps,
+        "library": library,
+    }
 
 
 def run_e2e(args, w, ci, dev, stream, o, lse, dq, dk, dv, ws, world):
