@@ -31,6 +31,11 @@ class Workload:
     sigma_v: float
     sigma_do: float
     causal: int = 1
+    # "default": bf16 outputs, bf16 tensor-core operands.  "accuracy": fp32 O, dQ, dK,
+    # dV, D from the fp32 O, P and dS split into hi + lo bf16 operands (the mode a
+    # workload needs when its outputs reach magnitudes where bf16 rounding alone
+    # exceeds the 2e-2 absolute tolerance).
+    mode: str = "default"
 
     @property
     def scale(self) -> float:
@@ -63,8 +68,17 @@ WORKLOADS = [
     Workload("gpt2small_b8h12t1024d64", 8, 12, 1024, 64, 1.0, 1.0, 1.0, 1.0),
     Workload("decoder200m_b4h16t2048d64", 4, 16, 2048, 64, 1.0, 1.0, 1.0, 1.0),
     Workload("hd128_b2h16t4096d128", 2, 16, 4096, 128, 1.0, 1.0, 0.5, 0.5),
-    Workload("ragged_b1h32t8000d128", 1, 32, 8000, 128, 3.0, 3.0, 1.0, 1.0),
+    Workload("ragged_b1h32t8000d128", 1, 32, 8000, 128, 3.0, 3.0, 1.0, 1.0, mode="accuracy"),
 ]
+
+# Option settings of each mode (the library's option bits are named after them).
+MODES = {
+    "default": {"o_f32": False, "grad_f32": False, "precise": False,
+                "desc": "bf16 O, dQ, dK, dV; P and dS enter the tensor-core products as bf16"},
+    "accuracy": {"o_f32": True, "grad_f32": True, "precise": True,
+                 "desc": "fp32 O, dQ, dK, dV; D from the fp32 O; P and dS enter the "
+                         "tensor-core products as two bf16 terms hi + lo"},
+}
 
 TENSOR_INDEX = {"q": 0, "k": 1, "v": 2, "dO": 3}
 
@@ -73,26 +87,67 @@ def seed_for(workload_index: int, tensor: str) -> int:
     return 1000 * workload_index + TENSOR_INDEX[tensor]
 
 
-def gaussian_bf16(shape, sigma: float, seed: int) -> torch.Tensor:
-    """fp32 randn(shape) * sigma from a seeded CPU generator, rounded to bf16."""
+def gaussian_bf16(shape, sigma: float, seed: int, dtype=torch.bfloat16) -> torch.Tensor:
+    """fp32 randn(shape) * sigma from a seeded CPU generator, rounded (to nearest even)
+    to bf16, or to another floating type `dtype` (fp16 for the fp16-operand mode)."""
     g = torch.Generator(device="cpu")
     g.manual_seed(seed)
     x = torch.randn(*shape, generator=g, dtype=torch.float32)
     if sigma != 1.0:
         x.mul_(sigma)
-    return x.to(torch.bfloat16)
+    return x.to(dtype)
 
 
-def make_inputs(workload_index: int, w: Workload | None = None, seed_offset: int = 0):
-    """Seeded bf16 CPU tensors q, k, v, dO for a workload (or a variant ``w`` of it)."""
+def make_inputs(workload_index: int, w: Workload | None = None, seed_offset: int = 0,
+                dtype=torch.bfloat16):
+    """Seeded bf16 (or `dtype`) CPU tensors q, k, v, dO for a workload (or a variant
+    ``w`` of it)."""
     w = w or WORKLOADS[workload_index]
     shape = (w.B, w.H, w.T, w.d)
     sig = {"q": w.sigma_q, "k": w.sigma_k, "v": w.sigma_v, "dO": w.sigma_do}
-    return {t: gaussian_bf16(shape, sig[t], seed_for(workload_index, t) + seed_offset)
+    return {t: gaussian_bf16(shape, sig[t], seed_for(workload_index, t) + seed_offset, dtype)
             for t in ("q", "k", "v", "dO")}
 
 
-def custom(B, H, T, d, sigma=1.0, causal=1, name=None) -> Workload:
+def custom(B, H, T, d, sigma=1.0, causal=1, name=None, mode="default") -> Workload:
     """A workload of any shape with one sigma for all four tensors (tests, edge cases)."""
     return Workload(name or f"b{B}h{H}t{T}d{d}", B, H, T, d, sigma, sigma, sigma, sigma,
-                    causal)
+                    causal, mode)
+
+
+def find(name: str):
+    """(index, workload) of the named workload."""
+    for i, w in enumerate(WORKLOADS):
+        if w.name == name:
+            return i, w
+    raise KeyError(f"unknown workload {name}; choose from {[w.name for w in WORKLOADS]}")
+
+
+# ------------------------------------------------------------------ AdamW ----
+# Parameter tensors of a GPT-2-small-shaped model (embed 768, 12 layers, 50257-token
+# vocabulary, 1024 positions): 148 tensors, 124.4M parameters.  Rank-2 tensors take
+# decoupled weight decay; vectors (biases, norm scales and shifts) do not.
+def gpt2small_param_shapes(n_layer=12, n_embd=768, vocab=50257, n_ctx=1024):
+    shapes = [(vocab, n_embd), (n_ctx, n_embd)]
+    for _ in range(n_layer):
+        shapes += [(n_embd,), (n_embd,), (3 * n_embd, n_embd), (3 * n_embd,),
+                   (n_embd, n_embd), (n_embd,), (n_embd,), (n_embd,),
+                   (4 * n_embd, n_embd), (4 * n_embd,), (n_embd, 4 * n_embd), (n_embd,)]
+    shapes += [(n_embd,), (n_embd,)]
+    return shapes
+
+
+def make_adamw_inputs(shapes, seed: int):
+    """Seeded fp32 CPU tensors for one AdamW step: per shape a parameter ~ N(0, 0.02^2),
+    a gradient ~ N(0, 0.01^2), a first moment ~ N(0, 0.001^2) and a second moment
+    |N(0, 1e-4)| (the state after some earlier steps).  Returns a list of dicts."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    out = []
+    for shp in shapes:
+        out.append({"param": torch.randn(*shp, generator=g) * 0.02,
+                    "grad": torch.randn(*shp, generator=g) * 0.01,
+                    "exp_avg": torch.randn(*shp, generator=g) * 1e-3,
+                    "exp_avg_sq": (torch.randn(*shp, generator=g) * 1e-4).abs(),
+                    "decay": len(shp) >= 2})
+    return out
