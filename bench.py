@@ -1,22 +1,31 @@
-"""Benchmark: causal attention forward + backward, bf16, TFLOP/s on B200.
+"""Benchmark: causal attention forward + backward on B200, TFLOP/s and % of the
+dense BF16 tensor peak.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--impl ours|reference] [--no-sub-results] [--no-cpu-baseline]
 
-One step is one pass of the whole path over one batch of the workload: the
-forward (one kernel) and the backward (D pre-pass, dK/dV kernel with the dQ partials
-added by TMA reduce-add into an fp32 accumulator, dQ conversion), all through the C ABI.  FLOPs are the causal counts (forward
-2*B*H*T^2*d, backward 2.5x that).  Inputs are synthetic (seeded bf16 Gaussian
-with the workload's shape and distribution) and resident in HBM; successive
-steps rotate over several input sets whose total is larger than the 126 MB L2.
+One step is one pass of the whole path over one batch of the workload: the forward
+(one kernel) and the backward (the D pre-pass, the dK/dV kernel with the dQ partials
+added by TMA reduce-add into an fp32 accumulator, and the dQ conversion when dQ is
+bf16), all through the C ABI.  FLOPs are the causal counts (forward 2*B*H*T^2*d,
+backward 2.5x that; the extra products of the accuracy mode's hi + lo operand
+split are not counted).  Inputs are synthetic (seeded bf16 Gaussian with the
+workload's shape and distribution) and resident in HBM; successive steps rotate
+over several input sets whose total is larger than the 126 MB L2.
+
+The headline workload is the largest one, B=1 H=32 T=8000 d=128 (ragged T), in the
+mode that meets the parity tolerances there (its "accuracy" mode: fp32 outputs, D
+from the fp32 O, P and dS split into two bf16 terms).  The same line carries
+sub-results for the other workloads and for full (non-causal) attention, each timed
+over at least half a second of GPU work.
 
 Prints ONE JSON line on rank 0.  With N > 1 (launched by torch.distributed.run)
-every rank runs its own batch (independent heads, no collective on the data
-path: weak scaling); the time is the max over ranks.
+every rank runs its own batch (independent heads, no collective on the data path:
+weak scaling); the time is the max over ranks.
 
---impl reference times the fp64 CPU oracle instead (the slow, plain reference
-this library is checked against): every step is a bounded sample of whole heads of
-the workload, sized so the run takes about --reference-seconds in all (default 150 s
-over 3 warm-up and 50 timed steps; a step is never less than one head pass).
+--impl reference times the fp64 CPU oracle instead (the slow, plain reference this
+library is checked against) on the same workload: every step is a bounded sample
+of whole heads; the steps run concurrently on the host's cores.
 """
 from __future__ import annotations
 
@@ -39,9 +48,21 @@ from causal_attention_fwd_attn_b200 import workloads as wl  # noqa: E402
 
 METRIC = "causal attention fwd+bwd TFLOP/s (bf16) and % of B200 dense BF16 peak"
 UNIT = "TFLOP/s"
-DEFAULT_WORKLOAD = "gpt2small_b8h12t1024d64"
+DEFAULT_WORKLOAD = "ragged_b1h32t8000d128"
 L2_BYTES = 126 * 1024 * 1024
 PROFILES = os.path.join(ROOT, "profiles")
+# Sub-results beside the headline: (workload, mode, causal).  Every causal workload
+# in the mode its parity tests use, the long workload also in the default bf16 mode
+# (context: outside the tolerance there), and full attention at two shapes.
+SUB_RESULTS = [
+    ("gpt2small_b8h12t1024d64", "default", 1),
+    ("decoder200m_b4h16t2048d64", "default", 1),
+    ("hd128_b2h16t4096d128", "default", 1),
+    ("ragged_b1h32t8000d128", "default", 1),
+    ("gpt2small_b8h12t1024d64", "default", 0),
+    ("hd128_b2h16t4096d128", "default", 0),
+]
+SUB_RESULT_SECONDS = 0.5
 
 
 def measured_peaks():
@@ -64,7 +85,7 @@ def kernel_source_sha():
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(kernel, workload):
+def recorded_traffic(kernel, key):
     """DRAM bytes per launch from a committed ncu capture, if the kernel sources
     are unchanged since it was taken (else None)."""
     path = os.path.join(PROFILES, "traffic.json")
@@ -72,40 +93,63 @@ def recorded_traffic(kernel, workload):
         return None
     with open(path) as f:
         rec = json.load(f)
-    e = rec.get(kernel, {}).get(workload)
+    e = rec.get(kernel, {}).get(key)
     if not e or e.get("source_sha") != kernel_source_sha():
         return None
     return e.get("dram_bytes_per_launch")
 
 
 def find_workload(name):
-    for i, w in enumerate(wl.WORKLOADS):
-        if w.name == name:
-            return i, w
-    raise SystemExit(f"unknown workload {name}; choose from {[w.name for w in wl.WORKLOADS]}")
+    try:
+        return wl.find(name)
+    except KeyError as e:
+        raise SystemExit(str(e)) from None
+
+
+def causal_flops(w, causal):
+    """(forward, backward) FLOPs of one pass: the causal counts, twice that for full
+    attention."""
+    f = 1.0 if causal else 2.0
+    return f * w.flops_fwd(), f * w.flops_bwd()
+
+
+def n_input_sets(w):
+    set_bytes = 4 * w.B * w.H * w.T * w.d * 2
+    return max(2, math.ceil(3 * L2_BYTES / set_bytes)), set_bytes
+
+
+def config_of(w, mode, causal, world):
+    """The workload description both arms print (identical keys and values)."""
+    n_sets, set_bytes = n_input_sets(w)
+    return {
+        "workload": w.name, "B": w.B, "H": w.H, "T": w.T, "d": w.d, "causal": causal,
+        "scale": "1/sqrt(d)", "mode": mode,
+        "inputs": "seeded iid Gaussian bf16 (seed 1000*workload + tensor), resident in HBM",
+        "l2": f"inputs larger than L2: rotating {n_sets} input sets, "
+              f"{n_sets * set_bytes / 2**20:.0f} MiB > 126 MB L2",
+        "parallelism": f"replicas x{world} (independent heads per GPU)",
+    }
 
 
 class ClockSampler:
     """SM clock, power and clock-event reasons sampled every few milliseconds by an NVML
-    thread while the timed region runs.
-
-    mark_begin()/mark_end() bracket the timed region on the host; only samples taken
-    between them are reported."""
+    thread.  window_begin()/window_end() bracket a timed region on the host; stats()
+    summarises the samples taken inside one window."""
 
     REASON_BITS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40,
                    "sw_thermal_slowdown": 0x20, "sw_power_cap": 0x4,
                    "hw_power_brake_slowdown": 0x80}
 
-    def __init__(self, device_index, period_s=0.004):
+    def __init__(self, device_index, period_s=0.002):
         self.dev = device_index
         self.period = period_s
         self.samples = []  # (host time, sm MHz, power W, reasons bitmask)
+        self.lock = threading.Lock()
         self.handle = None
         self.nvml = None
         self.sm_max = None
         self.thread = None
         self.stop_flag = False
-        self.window = [None, None]
         self.error = None
         try:
             import pynvml
@@ -135,41 +179,48 @@ class ClockSampler:
         while not self.stop_flag:
             try:
                 sm, pw, rs = self._read()
-                self.samples.append((time.perf_counter(), sm, pw, rs))
+                with self.lock:
+                    self.samples.append((time.perf_counter(), sm, pw, rs))
             except Exception as e:  # noqa: BLE001
                 self.error = f"nvml read failed: {type(e).__name__}"
                 return
             time.sleep(self.period)
 
     def start(self):
-        if self.nvml is None:
-            return
-        self.thread = threading.Thread(target=self._loop, daemon=True)
-        self.thread.start()
-
-    def mark_begin(self):
-        self.window[0] = time.perf_counter()
-
-    def mark_end(self):
-        self.window[1] = time.perf_counter()
+        if self.nvml is not None and self.thread is None:
+            self.thread = threading.Thread(target=self._loop, daemon=True)
+            self.thread.start()
+        return self
 
     def stop(self):
         if self.thread is not None:
             self.stop_flag = True
             self.thread.join(timeout=5)
-        lo, hi = self.window
-        rows = [s for s in self.samples
-                if (lo is None or s[0] >= lo) and (hi is None or s[0] <= hi)]
-        if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": self.sm_max,
-                    "reasons": [self.error or "no samples in the timed region"], "samples": 0}
-        reasons = sorted({name for s in rows for name, bit in self.REASON_BITS.items()
-                          if s[3] & bit})
-        return {"sm_mhz": statistics.median(s[1] for s in rows), "sm_max_mhz": self.sm_max,
-                "sm_min_mhz": min(s[1] for s in rows),
-                "power_w_median": round(statistics.median(s[2] for s in rows), 1),
-                "reasons": reasons, "samples": len(rows), "source": "nvml",
-                "period_ms": round(1000 * self.period, 1)}
+            self.thread = None
+
+    @staticmethod
+    def now():
+        return time.perf_counter()
+
+    def stats(self, lo, hi):
+        with self.lock:
+            rows = [s for s in self.samples if lo <= s[0] <= hi]
+        return summarise_clocks(rows, self.sm_max, self.error, self.period)
+
+
+def summarise_clocks(rows, sm_max, error=None, period=0.002):
+    """Median SM clock, power and the clock-event reasons seen in `rows` of
+    (time, sm MHz, power W, reasons bitmask)."""
+    if not rows:
+        return {"sm_mhz": None, "sm_max_mhz": sm_max,
+                "reasons": [error or "no samples in the timed region"], "samples": 0}
+    reasons = sorted({name for s in rows for name, bit in ClockSampler.REASON_BITS.items()
+                      if s[3] & bit})
+    return {"sm_mhz": statistics.median(s[1] for s in rows), "sm_max_mhz": sm_max,
+            "sm_min_mhz": min(s[1] for s in rows),
+            "power_w_median": round(statistics.median(s[2] for s in rows), 1),
+            "reasons": reasons, "samples": len(rows), "source": "nvml",
+            "period_ms": round(1000 * period, 1)}
 
 
 # ------------------------------------------------------ multi-rank helpers ----
@@ -196,190 +247,289 @@ def job_tflops(flops_per_step: float, steps: int, world: int, max_ms: float) -> 
     return flops_per_step * steps * world / (max_ms * 1e-3) / 1e12
 
 
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
 # ------------------------------------------------------------------- ours ----
-def run_ours(args, rank, world, local_rank):
-    from causal_attention_fwd_attn_b200 import _lib
+class Pass:
+    """Device buffers and the launches of one step (forward + backward) of a workload
+    in a mode, through the C ABI's stage entry points."""
 
-    ci, w = find_workload(args.workload)
-    dev = torch.device("cuda", local_rank)
-    torch.cuda.set_device(dev)
-    B, H, T, d = w.B, w.H, w.T, w.d
-    scale = w.scale
-    set_bytes = 4 * B * H * T * d * 2
-    out_bytes = B * H * T * d * 2 * 4 + B * H * T * 4
-    n_sets = max(2, math.ceil(3 * L2_BYTES / set_bytes))
-    sets = []
-    for s in range(n_sets):
-        x = wl.make_inputs(ci, seed_offset=replica_seed_offset(s, rank))
-        sets.append({n: t.to(dev) for n, t in x.items()})
-    o = torch.empty((B, H, T, d), dtype=torch.bfloat16, device=dev)
-    lse = torch.empty((B, H, T), dtype=torch.float32, device=dev)
-    dq, dk, dv = (torch.empty((B, H, T, d), dtype=torch.bfloat16, device=dev) for _ in range(3))
-    ws_n = _lib.forge_attn_bwd_workspace_size(B, H, T, d)
-    ws = torch.empty(ws_n, dtype=torch.uint8, device=dev)
-    rowstats_p = ws.data_ptr()
-    acc_p = ws.data_ptr() + _lib.rowstats_bytes(B, H, T)
-    stream = torch.cuda.current_stream(dev)
-    s = stream.cuda_stream
+    def __init__(self, w, mode, causal, dev):
+        from causal_attention_fwd_attn_b200 import _lib
 
-    def step(x, ev=None):
+        self.lib = _lib
+        self.w, self.mode, self.causal = w, mode, causal
+        m = wl.MODES[mode]
+        B, H, T, d = w.B, w.H, w.T, w.d
+        odt = torch.float32 if m["o_f32"] else torch.bfloat16
+        gdt = torch.float32 if m["grad_f32"] else torch.bfloat16
+        self.o = torch.empty((B, H, T, d), dtype=odt, device=dev)
+        self.lse = torch.empty((B, H, T), dtype=torch.float32, device=dev)
+        self.dq, self.dk, self.dv = (torch.empty((B, H, T, d), dtype=gdt, device=dev)
+                                     for _ in range(3))
+        self.ws_n = _lib.forge_attn_bwd_workspace_size(B, H, T, d)
+        self.ws = torch.empty(self.ws_n, dtype=torch.uint8, device=dev)
+        self.rowstats = self.ws.data_ptr()
+        # with fp32 gradients the dQ accumulator is dq itself, and there is no conversion
+        self.acc = (self.dq.data_ptr() if m["grad_f32"]
+                    else self.ws.data_ptr() + _lib.rowstats_bytes(B, H, T))
+        p = _lib.PRECISE if m["precise"] else 0
+        self.fwd_flags = (_lib.OUT_F32 if m["o_f32"] else 0) | p
+        self.pre_flags = _lib.O_IN_F32 if m["o_f32"] else 0
+        self.dkdv_flags = (_lib.OUT_F32 if m["grad_f32"] else 0) | p
+        self.bwd_flags = self.pre_flags | self.dkdv_flags
+        self.kernels = ["fwd", "pre", "dkdv"] + ([] if m["grad_f32"] else ["cvt"])
+        self.stream = torch.cuda.current_stream(dev)
+
+    def step(self, x, ev=None):
+        L, w, s = self.lib, self.w, self.stream.cuda_stream
+        B, H, T, d = w.B, w.H, w.T, w.d
         q, k, v, dO = x["q"], x["k"], x["v"], x["dO"]
         if ev:
-            ev[0].record(stream)
-        _lib.check(_lib.forge_attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
-                                       lse.data_ptr(), B, H, T, d, scale, w.causal, s), "fwd")
+            ev[0].record(self.stream)
+        L.check(L.forge_attn_fwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), self.o.data_ptr(),
+                                    self.lse.data_ptr(), B, H, T, d, w.scale, self.causal,
+                                    self.fwd_flags, s), "fwd")
         if ev:
-            ev[1].record(stream)
-        _lib.check(_lib.forge_attn_bwd_preprocess(o.data_ptr(), dO.data_ptr(), lse.data_ptr(),
-                                                  rowstats_p, acc_p, B, H, T, d, 0, s), "pre")
+            ev[1].record(self.stream)
+        L.check(L.forge_attn_bwd_preprocess(self.o.data_ptr(), dO.data_ptr(), self.lse.data_ptr(),
+                                            self.rowstats, self.acc, B, H, T, d, self.pre_flags,
+                                            s), "pre")
         if ev:
-            ev[2].record(stream)
-        _lib.check(_lib.forge_attn_bwd_dkdv(q.data_ptr(), k.data_ptr(), v.data_ptr(),
-                                            dO.data_ptr(), rowstats_p, acc_p, dk.data_ptr(),
-                                            dv.data_ptr(), B, H, T, d, scale, w.causal, 0, s),
-                   "dkdv")
+            ev[2].record(self.stream)
+        L.check(L.forge_attn_bwd_dkdv(q.data_ptr(), k.data_ptr(), v.data_ptr(), dO.data_ptr(),
+                                      self.rowstats, self.acc, self.dk.data_ptr(),
+                                      self.dv.data_ptr(), B, H, T, d, w.scale, self.causal,
+                                      self.dkdv_flags, s), "dkdv")
         if ev:
-            ev[3].record(stream)
-        _lib.check(_lib.forge_attn_bwd_dq_convert(acc_p, dq.data_ptr(), B, H, T, d, s), "cvt")
+            ev[3].record(self.stream)
+        if "cvt" in self.kernels:
+            L.check(L.forge_attn_bwd_dq_convert(self.acc, self.dq.data_ptr(), B, H, T, d, s),
+                    "cvt")
         if ev:
-            ev[4].record(stream)
+            ev[4].record(self.stream)
 
-    launches_per_step = 4
-    for i in range(args.warmup):
-        step(sets[i % n_sets])
+    def kernel_times(self, evs):
+        """Mean CUDA-event time (ms) of each kernel over the steps of `evs`."""
+        per = {k: [] for k in self.kernels}
+        for e in evs:
+            for a, k in enumerate(("fwd", "pre", "dkdv", "cvt")):
+                if k in per:
+                    per[k].append(e[a].elapsed_time(e[a + 1]))
+        return {k: sum(v) / len(v) for k, v in per.items()}
+
+    def check_device(self, when):
+        st, detail = self.lib.forge_attn_check_device_error(self.stream.cuda_stream)
+        if st != self.lib.OK:
+            raise RuntimeError(f"device wait timed out {when}: 0x{detail:08x}")
+
+
+def input_sets(ci, w, rank, dev):
+    n_sets, _ = n_input_sets(w)
+    return [{n: t.to(dev) for n, t in
+             wl.make_inputs(ci, w, seed_offset=replica_seed_offset(s, rank)).items()}
+            for s in range(n_sets)]
+
+
+def timed_run(p, sets, warmup, steps, world, dev, clocks):
+    """`warmup` untimed steps, then exactly `steps` steps between barriers and device
+    synchronisations.  Returns (max-over-ranks ms, per-kernel mean ms, clock stats)."""
+    n_sets = len(sets)
+    for i in range(warmup):
+        p.step(sets[i % n_sets])
     torch.cuda.synchronize()
-    st, detail = _lib.forge_attn_check_device_error(s)
-    if st != _lib.OK:
-        raise RuntimeError(f"device wait timed out during warm-up: 0x{detail:08x}")
-
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    p.check_device("during warm-up")
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(steps)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    clocks = ClockSampler(local_rank)
-    clocks.start()
-    if world > 1:
-        torch.distributed.barrier()
+    barrier(world)
     torch.cuda.synchronize()
-    clocks.mark_begin()
-    t0.record(stream)
-    for i in range(args.steps):
-        step(sets[(args.warmup + i) % n_sets], evs[i])
-    t1.record(stream)
+    lo = clocks.now()
+    t0.record(p.stream)
+    for i in range(steps):
+        p.step(sets[(warmup + i) % n_sets], evs[i])
+    t1.record(p.stream)
     torch.cuda.synchronize()
-    clocks.mark_end()
-    if world > 1:
-        torch.distributed.barrier()
-    clk = clocks.stop()
-    elapsed_ms = t0.elapsed_time(t1)
-    st, detail = _lib.forge_attn_check_device_error(s)
-    if st != _lib.OK:
-        raise RuntimeError(f"device wait timed out: 0x{detail:08x}")
-
-    per = {"fwd": [], "pre": [], "dkdv": [], "cvt": []}
-    for e in evs:
-        per["fwd"].append(e[0].elapsed_time(e[1]))
-        per["pre"].append(e[1].elapsed_time(e[2]))
-        per["dkdv"].append(e[2].elapsed_time(e[3]))
-        per["cvt"].append(e[3].elapsed_time(e[4]))
-    avg = {k: sum(v) / len(v) for k, v in per.items()}
-
-    max_ms = max_over_ranks(elapsed_ms, world, dev)
-
-    # ---- end to end through the C ABI with host buffers (pinned) ----------------
-    e2e = run_e2e(args, w, ci, dev, stream, o, lse, dq, dk, dv, ws, world)
-
-    if rank != 0:
-        return None
-    return ours_line(w, args.steps, args.warmup, world, max_ms, avg, clk, e2e,
-                     launches_per_step, n_sets, set_bytes, measured_peaks(),
-                     recorded_traffic("attn_bwd_dkdv", w.name),
-                     os.path.relpath(_lib.library_path(), ROOT))
+    hi = clocks.now()
+    barrier(world)
+    p.check_device("in the timed region")
+    max_ms = max_over_ranks(t0.elapsed_time(t1), world, dev)
+    return max_ms, p.kernel_times(evs), clocks.stats(lo, hi)
 
 
-def ours_line(w, steps, warmup, world, max_ms, avg, clk, e2e, launches_per_step, n_sets,
-              set_bytes, peaks, traffic, library):
+def dominant(avg):
+    return max(avg, key=avg.get)
+
+
+def roofline_of(w, causal, avg, peaks, traffic):
+    """Roofline object of the dK/dV kernel (the dominant one): its algorithmic FLOPs
+    per launch (the backward's causal count) over its mean CUDA-event duration."""
+    _, bwd_flops = causal_flops(w, causal)
+    achieved = bwd_flops / (avg["dkdv"] * 1e-3) / 1e12
+    return {
+        "kernel": "attn_bwd_dkdv",
+        "bound": "tensor",
+        "achieved": round(achieved, 1),
+        "peak": peaks["bf16_tflops"],
+        "unit": "TFLOP/s",
+        "frac": round(achieved / peaks["bf16_tflops"], 4),
+        "traffic": traffic,
+        "peak_source": f"{peaks['source']} bf16_tflops (burst)",
+        "dominant_by_time": dominant(avg),
+        "algorithmic_flops_per_launch": bwd_flops,
+    }
+
+
+def result_fields(w, causal, steps, world, max_ms, avg, peaks):
+    """Throughput fields shared by the headline and the sub-results."""
+    fwd_flops, bwd_flops = causal_flops(w, causal)
+    value = job_tflops(fwd_flops + bwd_flops, steps, world, max_ms)
+    bwd_ms = sum(v for k, v in avg.items() if k != "fwd")
+    return {
+        "value": round(value, 2),
+        "ms_per_step": round(max_ms / steps, 4),
+        "pct_of_peak": {"measured_bf16" if peaks["source"] == "measured" else "fallback_bf16":
+                        round(100 * value / world / peaks["bf16_tflops"], 2),
+                        "spec_2250": round(100 * value / world / 2250.0, 2)},
+        "fwd_ms": round(avg["fwd"], 4),
+        "bwd_ms": round(bwd_ms, 4),
+        "kernel_ms": {k: round(v, 4) for k, v in avg.items()},
+        "fwd_tflops": round(fwd_flops / (avg["fwd"] * 1e-3) / 1e12, 1),
+        "bwd_tflops": round(bwd_flops / (bwd_ms * 1e-3) / 1e12, 1),
+    }
+
+
+def ours_line(w, mode, causal, steps, warmup, world, max_ms, avg, clk, e2e, launches_per_step,
+              peaks, traffic, library, sub_results=None):
     """The JSON line of the GPU arm from its measurements: max_ms is the slowest
     rank's time for `steps` steps; avg holds each kernel's mean CUDA-event time (ms)
-    per launch ("fwd", "pre", "dkdv", "cvt")."""
-    value = job_tflops(w.flops_total(), steps, world, max_ms)
-    bwd_ms = avg["pre"] + avg["dkdv"] + avg["cvt"]
-    dkdv_flops = w.flops_bwd()
-    achieved = dkdv_flops / (avg["dkdv"] * 1e-3) / 1e12
-    return {
+    per launch ("fwd", "pre", "dkdv" and, with bf16 gradients, "cvt")."""
+    r = result_fields(w, causal, steps, world, max_ms, avg, peaks)
+    line = {
         "metric": METRIC,
-        "value": round(value, 2),
+        "value": r.pop("value"),
         "unit": UNIT,
         "n_gpus": world,
         "steps": steps,
         "warmup": warmup,
-        "ms_per_step": round(max_ms / steps, 4),
+        "ms_per_step": r.pop("ms_per_step"),
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic",
-        "config": {
-            "workload": w.name, "B": w.B, "H": w.H, "T": w.T, "d": w.d, "causal": w.causal,
-            "scale": "1/sqrt(d)", "inputs": "seeded iid Gaussian bf16, resident in HBM",
-            "l2": f"rotating {n_sets} input sets, {n_sets * set_bytes / 2**20:.0f} MiB of "
-                  f"inputs > 126 MB L2",
-            "parallelism": f"replicas x{world} (independent heads per GPU)",
-        },
-        "pct_of_peak": {"measured_bf16": round(100 * value / world / peaks["bf16_tflops"], 2),
-                        "spec_2250": round(100 * value / world / 2250.0, 2)},
-        "fwd_ms": round(avg["fwd"], 4),
-        "bwd_ms": round(bwd_ms, 4),
-        "kernel_ms": {k: round(v, 4) for k, v in avg.items()},
-        "fwd_tflops": round(w.flops_fwd() / (avg["fwd"] * 1e-3) / 1e12, 1),
-        "bwd_tflops": round(w.flops_bwd() / (bwd_ms * 1e-3) / 1e12, 1),
-        "roofline": {
-            "kernel": "attn_bwd_dkdv",
-            "bound": "tensor",
-            "achieved": round(achieved, 1),
-            "peak": peaks["bf16_tflops"],
-            "unit": "TFLOP/s",
-            "frac": round(achieved / peaks["bf16_tflops"], 4),
-            "traffic": traffic,
-            "peak_source": f"{peaks['source']} bf16_tflops (burst)",
-            "dominant_by_time": max(avg, key=avg.get),
-            "algorithmic_flops_per_launch": dkdv_flops,
-        },
+        "config": config_of(w, mode, causal, world),
+        "mode_desc": wl.MODES[mode]["desc"],
+    }
+    line.update(r)
+    line.update({
+        "roofline": roofline_of(w, causal, avg, peaks, traffic),
         "clocks": clk,
         "e2e": e2e,
         "gpu_launches": launches_per_step * steps,
         "library": library,
-    }
+    })
+    if sub_results is not None:
+        line["sub_results"] = sub_results
+    return line
 
 
-def run_e2e(args, w, ci, dev, stream, o, lse, dq, dk, dv, ws, world):
-    """Same metric through the C ABI, with each step's inputs copied from pinned host
-    memory and its outputs copied back, all inside the timed region."""
+def sub_result(w, mode, causal, steps, world, max_ms, avg, clk, peaks):
+    r = result_fields(w, causal, steps, world, max_ms, avg, peaks)
+    _, bwd_flops = causal_flops(w, causal)
+    dkdv_tf = bwd_flops / (avg["dkdv"] * 1e-3) / 1e12
+    r.update({"workload": w.name, "mode": mode, "causal": causal, "steps": steps,
+              "dominant_kernel": dominant(avg),
+              "dkdv_frac": round(dkdv_tf / peaks["bf16_tflops"], 4),
+              "clocks": {k: clk.get(k) for k in ("sm_mhz", "samples", "reasons")}})
+    return r
+
+
+def run_sub_results(rank, world, dev, clocks, peaks, warmup):
+    """Each (workload, mode, causal) of SUB_RESULTS timed over at least
+    SUB_RESULT_SECONDS of GPU work (the step count is sized from the warm-up steps and
+    agreed over ranks)."""
+    out = []
+    for name, mode, causal in SUB_RESULTS:
+        ci, w = find_workload(name)
+        sets = input_sets(ci, w, rank, dev)
+        p = Pass(w, mode, causal, dev)
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        for i in range(warmup):
+            p.step(sets[i % len(sets)])
+        t0.record(p.stream)
+        for i in range(3):
+            p.step(sets[i % len(sets)])
+        t1.record(p.stream)
+        torch.cuda.synchronize()
+        est_ms = max_over_ranks(t0.elapsed_time(t1) / 3, world, dev)
+        steps = max(20, min(20000, math.ceil(SUB_RESULT_SECONDS * 1e3 / est_ms)))
+        max_ms, avg, clk = timed_run(p, sets, 3, steps, world, dev, clocks)
+        out.append(sub_result(w, mode, causal, steps, world, max_ms, avg, clk, peaks))
+        del sets, p
+        torch.cuda.empty_cache()
+    return out
+
+
+def run_ours(args, rank, world, local_rank):
     from causal_attention_fwd_attn_b200 import _lib
 
+    ci, w = find_workload(args.workload)
+    mode = args.mode or w.mode
+    causal = w.causal
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    peaks = measured_peaks()
+    clocks = ClockSampler(local_rank).start()
+    try:
+        sets = input_sets(ci, w, rank, dev)
+        p = Pass(w, mode, causal, dev)
+        max_ms, avg, clk = timed_run(p, sets, args.warmup, args.steps, world, dev, clocks)
+        del sets
+        torch.cuda.empty_cache()
+        # ---- end to end through the public C ABI with host buffers (pinned) ------
+        e2e = run_e2e(args, w, ci, mode, causal, dev, p, world)
+        subs = None
+        if not args.no_sub_results:
+            subs = run_sub_results(rank, world, dev, clocks, peaks, 3)
+    finally:
+        clocks.stop()
+    if rank != 0:
+        return None
+    traffic = recorded_traffic("attn_bwd_dkdv", f"{w.name}/{mode}")
+    return ours_line(w, mode, causal, args.steps, args.warmup, world, max_ms, avg, clk, e2e,
+                     len(p.kernels), peaks, traffic,
+                     os.path.relpath(_lib.library_path(), ROOT), subs)
+
+
+def run_e2e(args, w, ci, mode, causal, dev, p, world):
+    """Same metric through the public C ABI (forge_attn_fwd_ex, forge_attn_bwd_ex), with
+    each step's inputs copied from pinned host memory and its outputs copied back,
+    all inside the timed region."""
+    L = p.lib
     B, H, T, d = w.B, w.H, w.T, w.d
-    x = wl.make_inputs(ci, seed_offset=7)
+    x = wl.make_inputs(ci, w, seed_offset=7)
     host_in = {n: t.pin_memory() for n, t in x.items()}
     dev_in = {n: torch.empty_like(t, device=dev) for n, t in x.items()}
-    host_out = {"o": torch.empty_like(o, device="cpu").pin_memory(),
-                "lse": torch.empty_like(lse, device="cpu").pin_memory(),
-                "dq": torch.empty_like(dq, device="cpu").pin_memory(),
-                "dk": torch.empty_like(dk, device="cpu").pin_memory(),
-                "dv": torch.empty_like(dv, device="cpu").pin_memory()}
-    dev_out = {"o": o, "lse": lse, "dq": dq, "dk": dk, "dv": dv}
+    dev_out = {"o": p.o, "lse": p.lse, "dq": p.dq, "dk": p.dk, "dv": p.dv}
+    host_out = {n: torch.empty_like(t, device="cpu").pin_memory() for n, t in dev_out.items()}
     h2d = sum(t.numel() * t.element_size() for t in host_in.values())
     d2h = sum(t.numel() * t.element_size() for t in host_out.values())
-    s = stream.cuda_stream
-    ws_n = ws.numel()
+    s = p.stream.cuda_stream
 
     def step():
         for n in host_in:
             dev_in[n].copy_(host_in[n], non_blocking=True)
         q, k, v, dO = dev_in["q"], dev_in["k"], dev_in["v"], dev_in["dO"]
-        _lib.check(_lib.forge_attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
-                                       lse.data_ptr(), B, H, T, d, w.scale, w.causal, s), "fwd")
-        _lib.check(_lib.forge_attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
-                                       dO.data_ptr(), lse.data_ptr(), dq.data_ptr(),
-                                       dk.data_ptr(), dv.data_ptr(), ws.data_ptr(), ws_n, B, H,
-                                       T, d, w.scale, w.causal, s), "bwd")
+        L.check(L.forge_attn_fwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), p.o.data_ptr(),
+                                    p.lse.data_ptr(), B, H, T, d, w.scale, causal, p.fwd_flags,
+                                    s), "fwd")
+        L.check(L.forge_attn_bwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), p.o.data_ptr(),
+                                    dO.data_ptr(), p.lse.data_ptr(), p.dq.data_ptr(),
+                                    p.dk.data_ptr(), p.dv.data_ptr(), p.ws.data_ptr(), p.ws_n,
+                                    B, H, T, d, w.scale, causal, p.bwd_flags, s), "bwd")
         for n in host_out:
             host_out[n].copy_(dev_out[n], non_blocking=True)
 
@@ -387,106 +537,123 @@ def run_e2e(args, w, ci, dev, stream, o, lse, dq, dk, dv, ws, world):
     for _ in range(2):
         step()
     torch.cuda.synchronize()
-    if world > 1:
-        torch.distributed.barrier()
+    barrier(world)
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    t0.record(stream)
+    t0.record(p.stream)
     for _ in range(steps):
         step()
-    t1.record(stream)
+    t1.record(p.stream)
     torch.cuda.synchronize()
+    p.check_device("in the end-to-end run")
     ms = max_over_ranks(t0.elapsed_time(t1), world, dev)
-    value = job_tflops(w.flops_total(), steps, world, ms)
+    fwd_flops, bwd_flops = causal_flops(w, causal)
+    value = job_tflops(fwd_flops + bwd_flops, steps, world, ms)
     return {"value": round(value, 2), "unit": UNIT, "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": d2h, "steps": steps, "ms_per_step": round(ms / steps, 4)}
+            "d2h_bytes_per_step": d2h, "steps": steps, "ms_per_step": round(ms / steps, 4),
+            "api": "forge_attn_fwd_ex + forge_attn_bwd_ex"}
 
 
 # ---------------------------------------------------------- CPU oracle leg ----
 class OracleSampler:
     """Times the fp64 oracle (forward + backward, the full T x T definition) on whole
-    heads of a workload, on the host's cores.  The inputs are prepared and the rate
-    of head passes with every thread busy is measured once; each sample then runs as
-    many head passes as fit its time budget at that rate (at least one), one head per
-    thread, cycling through the workload's heads."""
+    heads of a workload, on the host's cores, cycling through the workload's heads.
+    The oracle is single-threaded per head; a task is a run of consecutive head passes
+    on one thread, and tasks run concurrently, one per thread."""
 
-    def __init__(self, w, ci, threads):
+    def __init__(self, w, ci, threads, causal=None):
         import oracle
 
         self.w = w
+        self.causal = w.causal if causal is None else causal
         self.orc = oracle.default()
         x = wl.make_inputs(ci)
         self.f = {n: x[n].double().numpy() for n in x}
         self.heads = [(b, h) for b in range(w.B) for h in range(w.H)]
         self.threads = max(1, threads)
         self.cursor = 0
-        nb = min(self.threads, len(self.heads))
-        self.rate = nb / max(self._run(self.heads[:nb], nb), 1e-4)  # head passes per second
+        self.head_s = None  # seconds per head pass on one thread, once measured
 
-    def _run(self, hs, threads):
-        from concurrent.futures import ThreadPoolExecutor
-
-        f, w, orc = self.f, self.w, self.orc
-
-        def one(bh):
-            b, h = bh
-            orc.fwd_head(f["q"][b, h], f["k"][b, h], f["v"][b, h], w.scale, w.causal)
-            orc.bwd_head(f["q"][b, h], f["k"][b, h], f["v"][b, h], f["dO"][b, h], w.scale,
-                         w.causal)
-
-        t = time.perf_counter()
-        with ThreadPoolExecutor(max_workers=threads) as ex:
-            list(ex.map(one, hs))
-        return time.perf_counter() - t
-
-    def sample(self, budget_s):
-        """(TFLOP/s in the workload's causal-FLOP convention, threads used,
-        description, elapsed seconds) of one sample of about budget_s seconds."""
-        w = self.w
-        n = max(1, int(budget_s * self.rate))
-        threads = min(self.threads, n)
+    def _take(self, n):
         hs = [self.heads[(self.cursor + j) % len(self.heads)] for j in range(n)]
         self.cursor = (self.cursor + n) % len(self.heads)
-        elapsed = self._run(hs, threads)
-        value = w.flops_total() / w.BH * n / elapsed / 1e12
-        desc = (f"{n} head passes over the {w.BH} heads of {w.name} (T={w.T}, d={w.d}), "
-                f"fp64 oracle forward + backward, {elapsed:.2f} s on {threads} threads")
-        return value, threads, desc, elapsed
+        return hs
 
+    def _one(self, bh):
+        f, w, orc = self.f, self.w, self.orc
+        b, h = bh
+        orc.fwd_head(f["q"][b, h], f["k"][b, h], f["v"][b, h], w.scale, self.causal)
+        orc.bwd_head(f["q"][b, h], f["k"][b, h], f["v"][b, h], f["dO"][b, h], w.scale,
+                     self.causal)
 
-def oracle_sample(w, ci, budget_s, threads):
-    """One oracle sample of about budget_s seconds (see OracleSampler)."""
-    return OracleSampler(w, ci, threads).sample(budget_s)
+    def run_tasks(self, n_tasks, heads_per_task):
+        """Runs n_tasks tasks of heads_per_task head passes each, concurrently on
+        min(threads, n_tasks) threads; returns (wall seconds, threads used)."""
+        from concurrent.futures import ThreadPoolExecutor
+
+        tasks = [self._take(heads_per_task) for _ in range(n_tasks)]
+        threads = min(self.threads, n_tasks)
+        t = time.perf_counter()
+        with ThreadPoolExecutor(max_workers=threads) as ex:
+            list(ex.map(lambda hs: [self._one(bh) for bh in hs], tasks))
+        wall = time.perf_counter() - t
+        if heads_per_task == 1 and n_tasks <= threads:
+            self.head_s = wall
+        return wall, threads
+
+    def flops_per_head(self):
+        fwd, bwd = causal_flops(self.w, self.causal)
+        return (fwd + bwd) / self.w.BH
+
+    def sample(self, budget_s):
+        """(TFLOP/s in the workload's FLOP convention, threads used, description, wall
+        seconds) of one sample of about budget_s seconds with every thread busy: a first
+        round of one head pass per thread measures the rate; if that round already took
+        most of the budget it is the sample, else a second round of longer tasks is."""
+        n = min(self.threads, len(self.heads))
+        wall, threads = self.run_tasks(n, 1)
+        per_task = 1
+        if wall < 0.5 * budget_s:
+            per_task = max(1, int(budget_s / max(self.head_s, 1e-6)))
+            wall, threads = self.run_tasks(n, per_task)
+        passes = n * per_task
+        value = self.flops_per_head() * passes / wall / 1e12
+        desc = (f"{passes} head passes over the {self.w.BH} heads of {self.w.name} "
+                f"(T={self.w.T}, d={self.w.d}), fp64 oracle forward + backward, "
+                f"{wall:.2f} s on {threads} threads")
+        return value, threads, desc, wall
 
 
 def run_reference(args, rank, world):
-    """The oracle as it stands, timed on the host cores: each of the warm-up and timed
-    steps is one bounded sample of the workload, sized so that the whole run takes
-    about args.reference_seconds (a step is never less than one head pass)."""
+    """The oracle as it stands, timed on the host cores.  A step is a bounded sample of
+    the workload: a run of consecutive whole-head passes (forward + backward) on one
+    thread.  The warm-up steps are one head pass each and also measure the per-head
+    time; the timed steps are sized so that the timed phase takes about
+    args.reference_seconds, and run concurrently, one per thread."""
     if rank != 0:
         return None
     ci, w = find_workload(args.workload)
-    sampler = OracleSampler(w, ci, os.cpu_count() or 1)
-    budget = args.reference_seconds / max(1, args.steps + args.warmup)
-    steps_v, descs, threads = [], [], 1
-    for i in range(args.warmup + args.steps):
-        v, cores, desc, el = sampler.sample(budget)
-        if i >= args.warmup:
-            steps_v.append((v, el))
-            descs.append(desc)
-            threads = max(threads, cores)
-    value = statistics.median(v for v, _ in steps_v)
-    ms = statistics.median(el for _, el in steps_v) * 1e3
+    mode = getattr(args, "mode", None) or w.mode
+    threads = max(1, os.cpu_count() or 1)
+    sampler = OracleSampler(w, ci, threads)
+    t_warm, _ = sampler.run_tasks(args.warmup, 1)
+    head_s = sampler.head_s or t_warm
+    rounds = math.ceil(args.steps / min(threads, args.steps))
+    per_step = max(1, int(args.reference_seconds / (rounds * head_s)))
+    wall, used = sampler.run_tasks(args.steps, per_step)
+    passes = args.steps * per_step
+    value = sampler.flops_per_head() * passes / wall / 1e12
+    desc = (f"{args.steps} steps of {per_step} head passes each over the {w.BH} heads of "
+            f"{w.name} (T={w.T}, d={w.d}), fp64 oracle forward + backward, run "
+            f"concurrently: {wall:.2f} s on {used} threads")
     return {
         "impl": "reference",
         "metric": METRIC, "value": round(value, 6), "unit": UNIT, "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 2),
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(wall * 1e3 / args.steps, 2),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
-        "config": {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "d": w.d,
-                   "causal": w.causal, "scale": "1/sqrt(d)",
-                   "note": "each step is a bounded sample of the workload's heads"},
-        "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": threads,
-                         "kind": "oracle", "sample": descs[-1]},
+        "config": config_of(w, mode, w.causal, world),
+        "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": used,
+                         "kind": "oracle", "sample": desc},
         "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -497,26 +664,29 @@ def main():
                                  formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=None,
-                    help="timed steps (default 2000; 50 for --impl reference)")
+                    help="timed steps (default 300; 20 for --impl reference)")
     ap.add_argument("--warmup", type=int, default=None,
-                    help="untimed warm-up steps, at least 3 (default 20; 3 for --impl reference)")
+                    help="untimed warm-up steps, at least 3 (default 10; 5 for --impl reference)")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--mode", choices=sorted(wl.MODES), default=None,
+                    help="default: the mode the workload's parity tests use")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-baseline-seconds", type=float, default=12.0,
                     help="budget of the oracle sample timed beside the GPU run (rank 0, N=1)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--reference-seconds", type=float, default=150.0,
-                    help="--impl reference: total oracle time over all warm-up and timed steps "
+    ap.add_argument("--no-sub-results", action="store_true")
+    ap.add_argument("--reference-seconds", type=float, default=90.0,
+                    help="--impl reference: about how long the timed steps take in all "
                          "(each step is at least one head pass)")
     args = ap.parse_args()
-    # the reference arm's steps are oracle samples of whole heads (one head pass takes
-    # about 0.3 s at the gpt2-small shape on one core), so its default run is shorter
     if args.steps is None:
-        args.steps = 50 if args.impl == "reference" else 2000
+        args.steps = 20 if args.impl == "reference" else 300
     if args.warmup is None:
-        args.warmup = 3 if args.impl == "reference" else 20
+        args.warmup = 5 if args.impl == "reference" else 10
     if args.warmup < 3:
         raise SystemExit("--warmup must be at least 3")
+    if args.steps < 1:
+        raise SystemExit("--steps must be at least 1")
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -541,8 +711,8 @@ def main():
         res = run_ours(args, rank, world, local_rank)
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
             ci, w = find_workload(args.workload)
-            v, cores, desc, _ = oracle_sample(w, ci, args.cpu_baseline_seconds,
-                                              os.cpu_count() or 1)
+            v, cores, desc, _ = OracleSampler(w, ci, os.cpu_count() or 1).sample(
+                args.cpu_baseline_seconds)
             res["cpu_baseline"] = {"value": round(v, 6), "unit": UNIT, "cores": cores,
                                    "kind": "oracle", "sample": desc}
         elif rank == 0:

@@ -31,15 +31,17 @@ def assert_close(name, gpu, ref, what=""):
     return rel, mx
 
 
-def run_gpu(x, scale, causal, o_dtype=torch.bfloat16, grad_dtype=torch.bfloat16, bwd=True,
-            precise=False):
-    """Forward (and backward) through the C ABI on cuda:0.  x: dict of CPU bf16 tensors.
-    With an fp32 O the backward reads that fp32 O for its D pre-pass."""
+def run_gpu(x, scale, causal, o_dtype=None, grad_dtype=None, bwd=True, precise=False):
+    """Forward (and backward) through the C ABI on cuda:0.  x: dict of CPU bf16 (or fp16:
+    the fp16-operand mode) tensors.  Outputs default to the inputs' dtype.  With an
+    fp32 O the backward reads that fp32 O for its D pre-pass."""
     dev = torch.device("cuda", 0)
     q, k, v, dO = (x[n].to(dev) for n in ("q", "k", "v", "dO"))
     B, H, T, d = q.shape
     s = torch.cuda.current_stream(dev).cuda_stream
-    pflag = _lib.PRECISE if precise else 0
+    o_dtype = o_dtype or q.dtype
+    grad_dtype = grad_dtype or q.dtype
+    pflag = (_lib.PRECISE if precise else 0) | (_lib.FP16 if q.dtype == torch.float16 else 0)
     o = torch.empty((B, H, T, d), dtype=o_dtype, device=dev)
     lse = torch.empty((B, H, T), dtype=torch.float32, device=dev)
     fflags = (_lib.OUT_F32 if o_dtype == torch.float32 else 0) | pflag
@@ -63,6 +65,26 @@ def run_gpu(x, scale, causal, o_dtype=torch.bfloat16, grad_dtype=torch.bfloat16,
     st, detail = _lib.forge_attn_check_device_error(s)
     assert st == _lib.OK, f"device wait timed out: 0x{detail:08x}"
     return {n: t.float().cpu().numpy() for n, t in out.items()}
+
+
+def mode_kwargs(mode):
+    """run_gpu keyword arguments of a workload mode ("default" or "accuracy")."""
+    m = wl.MODES[mode]
+    return dict(o_dtype=torch.float32 if m["o_f32"] else torch.bfloat16,
+                grad_dtype=torch.float32 if m["grad_f32"] else torch.bfloat16,
+                precise=m["precise"])
+
+
+def oracle_threads(T):
+    """Host threads for the full oracle at sequence length T: one head per thread,
+    capped by the memory its T x T buffers take (three fp64 matrices per head)."""
+    import os
+
+    import psutil
+
+    per_head = 3 * 8 * T * T + (64 << 20)
+    avail = psutil.virtual_memory().available
+    return max(1, min(os.cpu_count() or 1, int(0.7 * avail // per_head)))
 
 
 def as_f64(x):

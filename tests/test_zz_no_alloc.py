@@ -11,9 +11,10 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 from causal_attention_fwd_attn_b200 import _lib, build
 from causal_attention_fwd_attn_b200 import workloads as wl
-from tests.gpu_helpers import TOL, errors
+from tests.gpu_helpers import TOL, as_f64, assert_close, errors
 
 P = 4096  # a 16-byte aligned fake address; never dereferenced (rejected first)
 
@@ -58,12 +59,14 @@ def _backward_both_ways(x, w, dev, s):
     return ([t.float().cpu().numpy() for t in ref], [t.float().cpu().numpy() for t in got])
 
 
+# (1, 96, 384, 64): 288 key-tile items, about two per persistent CTA
 @pytest.mark.gpu
-@pytest.mark.parametrize("shape", [(2, 3, 300, 64), (1, 4, 513, 128)])
+@pytest.mark.parametrize("shape", [(2, 3, 300, 64), (1, 4, 513, 128), (1, 96, 384, 64)])
 def test_noalloc_matches_workspace_backward_twice(shape):
     dev = torch.device("cuda", 0)
     s = torch.cuda.current_stream(dev).cuda_stream
     w = wl.custom(*shape)
+    orc = oracle.default()
     # two calls in a row on different inputs: the second must not see the first's scratch
     for call in range(2):
         x = wl.make_inputs(0, w, seed_offset=1000 + 37 * call + shape[3])
@@ -75,3 +78,8 @@ def test_noalloc_matches_workspace_backward_twice(shape):
             assert rel <= trel and mx <= tabs, f"call {call} {name}: {rel:.3e} {mx:.3e}"
         # dK and dV come from the same deterministic kernel with the same inputs
         assert np.array_equal(got[1], ref[1]) and np.array_equal(got[2], ref[2])
+        # and all three against the fp64 oracle on the same inputs
+        f = as_f64(x)
+        exact = orc.bwd(f["q"], f["k"], f["v"], f["dO"], w.scale, 1, threads=8)
+        for name, a, b in zip(("dq", "dk", "dv"), got, exact):
+            assert_close(name, a, b, f"noalloc call {call} {w.describe()}")
