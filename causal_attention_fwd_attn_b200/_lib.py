@@ -23,6 +23,7 @@ ERR_WORKSPACE = 6
 OUT_F32 = 1
 O_IN_F32 = 2
 PRECISE = 4
+FP16 = 8
 
 PROBE_SS_KK = 0
 PROBE_SS_KMN = 1
@@ -32,10 +33,20 @@ PROBE_SS_MNMN = 3
 EXPORTED = [
     "forge_attn_fwd", "forge_attn_fwd_ex", "forge_attn_bwd_workspace_size", "forge_attn_bwd",
     "forge_attn_bwd_ex", "forge_attn_bwd_preprocess", "forge_attn_bwd_dkdv",
-    "forge_attn_bwd_dq_convert", "forge_attn_status_string", "forge_attn_check_device_error",
-    "forge_attn_version", "forge_probe_mma", "forge_probe_wait_timeout",
-    "forge_attn_bwd_noalloc",
+    "forge_attn_bwd_dq_convert", "forge_attn_bwd_dq_convert_ex", "forge_attn_status_string",
+    "forge_attn_check_device_error", "forge_attn_version", "forge_probe_mma", "forge_probe_wait_timeout",
+    "forge_attn_bwd_noalloc", "forge_adamw_workspace_size", "forge_adamw_step",
 ]
+
+ADAMW_MAX_TENSORS_PER_LAUNCH = 256
+
+
+class AdamWTensor(ctypes.Structure):
+    """forge_adamw_tensor of include/forge_adamw.h (device pointers and a size)."""
+    _fields_ = [("param", ctypes.c_void_p), ("grad", ctypes.c_void_p),
+                ("exp_avg", ctypes.c_void_p), ("exp_avg_sq", ctypes.c_void_p),
+                ("n", ctypes.c_longlong), ("decay", ctypes.c_int)]
+
 
 _vp = ctypes.c_void_p
 _i = ctypes.c_int
@@ -54,6 +65,7 @@ _SIGNATURES = {
     "forge_attn_bwd_dkdv": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i,
                                  _i, _vp]),
     "forge_attn_bwd_dq_convert": (_i, [_vp, _vp, _i, _i, _i, _i, _vp]),
+    "forge_attn_bwd_dq_convert_ex": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _vp]),
     "forge_attn_status_string": (ctypes.c_char_p, [_i]),
     "forge_attn_check_device_error": (_i, [_vp, ctypes.POINTER(ctypes.c_uint)]),
     "forge_attn_version": (_i, []),
@@ -61,6 +73,9 @@ _SIGNATURES = {
     "forge_probe_wait_timeout": (_i, [ctypes.c_ulonglong, _vp]),
     "forge_attn_bwd_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i,
                                     _f, _i, _vp]),
+    "forge_adamw_workspace_size": (_sz, [_i]),
+    "forge_adamw_step": (_i, [ctypes.POINTER(AdamWTensor), _i, _f, _f, _f, _f, _f, _i, _f, _vp,
+                              _vp, _sz, _vp]),
 }
 
 _lib = None
@@ -150,12 +165,31 @@ def forge_attn_bwd_dq_convert(dq_accum, dq, B, H, T, d, stream):
     return load().forge_attn_bwd_dq_convert(dq_accum, dq, B, H, T, d, stream)
 
 
+def forge_attn_bwd_dq_convert_ex(dq_accum, dq, B, H, T, d, flags, stream):
+    return load().forge_attn_bwd_dq_convert_ex(dq_accum, dq, B, H, T, d, flags, stream)
+
+
 def forge_attn_bwd_noalloc(q, k, v, o, dO, lse, dq, dk, dv, B, H, T, d, scale, causal, stream):
     return load().forge_attn_bwd_noalloc(q, k, v, o, dO, lse, dq, dk, dv, B, H, T, d, scale,
                                          causal, stream)
 
 
 NOALLOC_SCRATCH_BYTES = 64 << 20
+
+
+def forge_adamw_workspace_size(n_tensors):
+    return load().forge_adamw_workspace_size(n_tensors)
+
+
+def forge_adamw_step(tensors, lr, beta1, beta2, eps, weight_decay, step, max_norm,
+                     grad_norm_out, workspace, workspace_bytes, stream):
+    """tensors: a sequence of (param, grad, exp_avg, exp_avg_sq, n, decay) tuples of device
+    addresses and sizes, or AdamWTensor values."""
+    arr = (AdamWTensor * max(1, len(tensors)))()
+    for i, t in enumerate(tensors):
+        arr[i] = t if isinstance(t, AdamWTensor) else AdamWTensor(*t)
+    return load().forge_adamw_step(arr, len(tensors), lr, beta1, beta2, eps, weight_decay, step,
+                                   max_norm, grad_norm_out, workspace, workspace_bytes, stream)
 
 
 def forge_attn_check_device_error(stream):

@@ -87,7 +87,7 @@ enum : uint32_t {
     kSiteAccFree
 };
 
-template <int D, bool PRECISE>
+template <int D, bool PRECISE, bool F16>
 struct BwdCfg {
     static constexpr int kChunks = D / 64;
     static constexpr int kChunkBytes = kTile * 128;        // 128 rows x 128 bytes
@@ -158,9 +158,10 @@ struct BwdCfg {
     static_assert(128 * kRegsDrain + 256 * kRegsCompute + 128 * kRegsCtl <=
                       kBwdThreads * kLaunchRegs,
                   "register split exceeds the block's launch allocation");
-    static constexpr uint32_t kIdescScore = idesc_bf16_f32(128, 128, false, false);
-    static constexpr uint32_t kIdescGrad = idesc_bf16_f32(128, D, false, true);  // dV, dK
-    static constexpr uint32_t kIdescDQ = idesc_bf16_f32(128, D, true, true);     // dQ
+    // every operand bf16, or every operand fp16 (F16)
+    static constexpr uint32_t kIdescScore = idesc_f16kind_f32(128, 128, false, false, F16);
+    static constexpr uint32_t kIdescGrad = idesc_f16kind_f32(128, D, false, true, F16);  // dV, dK
+    static constexpr uint32_t kIdescDQ = idesc_f16kind_f32(128, D, true, true, F16);     // dQ
 };
 
 struct BwdBarriers {
@@ -179,15 +180,16 @@ struct BwdBarriers {
 };
 static_assert(sizeof(BwdBarriers) <= 256, "barrier block");
 
-// Eight fp32 values as bf16 into a 16-byte chunk at base + off; in precise mode the
-// remainders x - bf16(x), rounded to bf16, go to the same place in the lo buffer
-// (base + lo_stride + off).
-template <bool PRECISE>
+// Eight fp32 values as bf16 (fp16 with F16) into a 16-byte chunk at base + off; in
+// precise mode (bf16 only) the remainders x - bf16(x), rounded to bf16, go to the same
+// place in the lo buffer (base + lo_stride + off).
+template <bool PRECISE, bool F16>
 __device__ __forceinline__ void store_split8(uint8_t* base, int lo_stride, uint32_t off,
                                              const float* x) {
+    static_assert(!(PRECISE && F16), "the hi + lo split is a bf16-operand mode");
     uint32_t h[4];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) h[e] = pack_bf16x2(x[2 * e], x[2 * e + 1]);
+    for (int e = 0; e < 4; ++e) h[e] = pack16x2<F16>(x[2 * e], x[2 * e + 1]);
     *reinterpret_cast<uint4*>(base + off) = make_uint4(h[0], h[1], h[2], h[3]);
     if (PRECISE) {
         uint32_t l[4];
@@ -204,7 +206,7 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, uint32
     return __all_sync(0xffffffffu, mbar_wait(bar, parity, site, abort));
 }
 
-template <int D, bool PRECISE>
+template <int D, bool PRECISE, bool F16>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmap_q,
                          const __grid_constant__ CUtensorMap tmap_k,
@@ -215,7 +217,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                          void* __restrict__ dk_out, void* __restrict__ dv_out, int T, int BH,
                          int n_kvtiles, int n_items, float scale, float scale_log2, int causal,
                          int grad_f32) {
-    using C = BwdCfg<D, PRECISE>;
+    using C = BwdCfg<D, PRECISE, F16>;
     extern __shared__ __align__(1024) uint8_t smem[];
     BwdBarriers* bars = reinterpret_cast<BwdBarriers*>(smem + C::kOffBar);
     volatile int* abort = &bars->abort;
@@ -406,17 +408,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                                                    __uint_as_float(r[4 * e + 3]) * mul);
                         } else {
                             uint4* o = reinterpret_cast<uint4*>(
-                                reinterpret_cast<__nv_bfloat16*>(out) + base + c * 32);
+                                reinterpret_cast<uint16_t*>(out) + base + c * 32);
 #pragma unroll
                             for (int e = 0; e < 4; ++e)
-                                o[e] = make_uint4(pack_bf16x2(__uint_as_float(r[8 * e]) * mul,
-                                                              __uint_as_float(r[8 * e + 1]) * mul),
-                                                  pack_bf16x2(__uint_as_float(r[8 * e + 2]) * mul,
-                                                              __uint_as_float(r[8 * e + 3]) * mul),
-                                                  pack_bf16x2(__uint_as_float(r[8 * e + 4]) * mul,
-                                                              __uint_as_float(r[8 * e + 5]) * mul),
-                                                  pack_bf16x2(__uint_as_float(r[8 * e + 6]) * mul,
-                                                              __uint_as_float(r[8 * e + 7]) * mul));
+                                o[e] = make_uint4(
+                                    pack16x2<F16>(__uint_as_float(r[8 * e]) * mul,
+                                                  __uint_as_float(r[8 * e + 1]) * mul),
+                                    pack16x2<F16>(__uint_as_float(r[8 * e + 2]) * mul,
+                                                  __uint_as_float(r[8 * e + 3]) * mul),
+                                    pack16x2<F16>(__uint_as_float(r[8 * e + 4]) * mul,
+                                                  __uint_as_float(r[8 * e + 5]) * mul),
+                                    pack16x2<F16>(__uint_as_float(r[8 * e + 6]) * mul,
+                                                  __uint_as_float(r[8 * e + 7]) * mul));
                         }
                     }
                 }
@@ -500,7 +503,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             {
                 uint32_t pk[32];
 #pragma unroll
-                for (int e = 0; e < 32; ++e) pk[e] = pack_bf16x2(p[2 * e], p[2 * e + 1]);
+                for (int e = 0; e < 32; ++e) pk[e] = pack16x2<F16>(p[2 * e], p[2 * e + 1]);
                 const uint32_t tp = tmem + lane_off + C::p_col(4 * (int)half);
                 tc_fence_after();
                 if constexpr (PRECISE) {
@@ -554,8 +557,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                         ds[2 * e] = dsv.x;
                         ds[2 * e + 1] = dsv.y;
                     }
-                    store_split8<PRECISE>(ds_smem, C::kScoreBytes, sw128_offset(row, c * 4 + ch),
-                                          ds);
+                    store_split8<PRECISE, F16>(ds_smem, C::kScoreBytes,
+                                               sw128_offset(row, c * 4 + ch), ds);
                 }
             }
             tc_fence_before();
@@ -840,12 +843,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 // Row statistics of the backward, padded per head to t_pad = 128 * ceil(T / 128) rows:
 // rowstats[0][bh][t] = -LSE * log2(e) (negated: it is the addend of the exponent) and
 // rowstats[1][bh][t] = D = rowsum(dO o O) (fp32; -inf and 0 past T), and the dQ
-// accumulator cleared.  O is bf16 or fp32
-// (TO); dO is bf16.  A group of D/8 consecutive threads covers one row, 8 elements
-// each, so every load of a warp is one contiguous span.
-template <int D, typename TO>
+// accumulator cleared.  O is fp32, or 16-bit like dO (F16: fp16, else bf16).  A
+// group of D/8 consecutive threads covers one row, 8 elements each, so every load of
+// a warp is one contiguous span.
+template <int D, bool O_F32, bool F16>
 __global__ void __launch_bounds__(256) attn_bwd_preprocess_kernel(
-    const TO* __restrict__ o, const __nv_bfloat16* __restrict__ dO,
+    const void* __restrict__ o_in, const uint16_t* __restrict__ dO,
     const float* __restrict__ lse, float* __restrict__ rowstats, float* __restrict__ dq_accum,
     int T, int t_pad, long long padded_rows) {
     constexpr int kGroup = D / 8;  // threads per row
@@ -859,26 +862,29 @@ __global__ void __launch_bounds__(256) attn_bwd_preprocess_kernel(
     float acc = 0.f;
     if (valid) {
         const uint4 b = reinterpret_cast<const uint4*>(dO + r * D)[part];
-        const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&b);
+        const uint32_t bw[4] = {b.x, b.y, b.z, b.w};
         float fo[8];
-        if constexpr (sizeof(TO) == 2) {
-            const uint4 a = reinterpret_cast<const uint4*>(o + r * D)[part];
-            const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a);
+        if constexpr (!O_F32) {
+            const uint4 a = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(o_in) +
+                                                           r * D)[part];
+            const uint32_t aw[4] = {a.x, a.y, a.z, a.w};
 #pragma unroll
             for (int h = 0; h < 4; ++h) {
-                const float2 f = __bfloat1622float2(a2[h]);
+                const float2 f = unpack16x2<F16>(aw[h]);
                 fo[2 * h] = f.x;
                 fo[2 * h + 1] = f.y;
             }
         } else {
-            const float4 a0 = reinterpret_cast<const float4*>(o + r * D)[2 * part];
-            const float4 a1 = reinterpret_cast<const float4*>(o + r * D)[2 * part + 1];
+            const float4* o4 = reinterpret_cast<const float4*>(static_cast<const float*>(o_in) +
+                                                               r * D);
+            const float4 a0 = o4[2 * part];
+            const float4 a1 = o4[2 * part + 1];
             fo[0] = a0.x; fo[1] = a0.y; fo[2] = a0.z; fo[3] = a0.w;
             fo[4] = a1.x; fo[5] = a1.y; fo[6] = a1.z; fo[7] = a1.w;
         }
 #pragma unroll
         for (int h = 0; h < 4; ++h) {
-            const float2 fb = __bfloat1622float2(b2[h]);
+            const float2 fb = unpack16x2<F16>(bw[h]);
             acc = fmaf(fo[2 * h], fb.x, acc);
             acc = fmaf(fo[2 * h + 1], fb.y, acc);
         }
@@ -896,39 +902,29 @@ __global__ void __launch_bounds__(256) attn_bwd_preprocess_kernel(
     }
 }
 
-// dQ = bf16(accumulator), 8 elements per thread.
+// dQ = bf16(accumulator) (fp16 with F16), 8 elements per thread.
+template <bool F16>
 __global__ void __launch_bounds__(256) attn_bwd_dq_convert_kernel(const float* __restrict__ acc,
-                                                                  __nv_bfloat16* __restrict__ dq,
+                                                                  uint16_t* __restrict__ dq,
                                                                   long long n8) {
     const long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     if (t >= n8) return;
     const float4 a = reinterpret_cast<const float4*>(acc)[2 * t];
     const float4 b = reinterpret_cast<const float4*>(acc)[2 * t + 1];
-    reinterpret_cast<uint4*>(dq)[t] = make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w),
-                                                 pack_bf16x2(b.x, b.y), pack_bf16x2(b.z, b.w));
+    reinterpret_cast<uint4*>(dq)[t] =
+        make_uint4(pack16x2<F16>(a.x, a.y), pack16x2<F16>(a.z, a.w), pack16x2<F16>(b.x, b.y),
+                   pack16x2<F16>(b.z, b.w));
 }
 
-int sm_count() {
-    static int n = 0;
-    if (n == 0) {
-        int dev = 0;
-        if (cudaGetDevice(&dev) != cudaSuccess ||
-            cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-            n <= 0)
-            n = 148;
-    }
-    return n;
-}
-
-template <int D, bool PRECISE>
+template <int D, bool PRECISE, bool F16>
 cudaError_t launch_dkdv_dp(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                            const CUtensorMap& tdo, const CUtensorMap& tdq, const float* rowstats,
                            float* dq_accum, void* dk, void* dv, int BH, int T, float scale,
                            int causal, int grad_f32, cudaStream_t stream) {
-    using C = BwdCfg<D, PRECISE>;
+    using C = BwdCfg<D, PRECISE, F16>;
     static std::atomic<unsigned long long> configured{0};
     cudaError_t e =
-        set_max_dynamic_smem(attn_bwd_dkdv_kernel<D, PRECISE>, C::kSmemBytes, configured);
+        set_max_dynamic_smem(attn_bwd_dkdv_kernel<D, PRECISE, F16>, C::kSmemBytes, configured);
     if (e != cudaSuccess) return e;
     const int n_kvtiles = (T + kTile - 1) / kTile;
     const long long items = (long long)BH * n_kvtiles;
@@ -936,13 +932,13 @@ cudaError_t launch_dkdv_dp(const CUtensorMap& tq, const CUtensorMap& tk, const C
     const int n_items = (int)items;
     // persistent: one CTA per SM (shared memory and tensor memory allow no more)
     const int grid = n_items < sm_count() ? n_items : sm_count();
-    attn_bwd_dkdv_kernel<D, PRECISE><<<grid, kBwdThreads, C::kSmemBytes, stream>>>(
+    attn_bwd_dkdv_kernel<D, PRECISE, F16><<<grid, kBwdThreads, C::kSmemBytes, stream>>>(
         tq, tk, tv, tdo, tdq, rowstats, dq_accum, dk, dv, T, BH, n_kvtiles, n_items, scale,
         scale * kLog2e, causal, grad_f32);
     return cudaGetLastError();
 }
 
-template <int D, typename TO>
+template <int D, bool O_F32, bool F16>
 void launch_pre(const void* o, const void* dO, const float* lse, float* rowstats,
                 float* dq_accum, int BH, int T, cudaStream_t stream) {
     const int t_pad = ((T + kTile - 1) / kTile) * kTile;
@@ -950,52 +946,70 @@ void launch_pre(const void* o, const void* dO, const float* lse, float* rowstats
     const int threads = 256;
     const long long total = padded_rows * (D / 8);
     const unsigned blocks = (unsigned)((total + threads - 1) / threads);
-    attn_bwd_preprocess_kernel<D, TO><<<blocks, threads, 0, stream>>>(
-        static_cast<const TO*>(o), static_cast<const __nv_bfloat16*>(dO), lse, rowstats, dq_accum,
-        T, t_pad, padded_rows);
+    attn_bwd_preprocess_kernel<D, O_F32, F16><<<blocks, threads, 0, stream>>>(
+        o, static_cast<const uint16_t*>(dO), lse, rowstats, dq_accum, T, t_pad, padded_rows);
+}
+
+template <int D>
+void launch_pre_d(const void* o, const void* dO, const float* lse, float* rowstats,
+                  float* dq_accum, int BH, int T, int o_f32, int f16, cudaStream_t stream) {
+    if (o_f32) {
+        if (f16) launch_pre<D, true, true>(o, dO, lse, rowstats, dq_accum, BH, T, stream);
+        else launch_pre<D, true, false>(o, dO, lse, rowstats, dq_accum, BH, T, stream);
+    } else {
+        if (f16) launch_pre<D, false, true>(o, dO, lse, rowstats, dq_accum, BH, T, stream);
+        else launch_pre<D, false, false>(o, dO, lse, rowstats, dq_accum, BH, T, stream);
+    }
+}
+
+template <int D>
+cudaError_t launch_dkdv_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                          const CUtensorMap& tdo, const CUtensorMap& tdq, const float* rowstats,
+                          float* dq_accum, void* dk, void* dv, int BH, int T, float scale,
+                          int causal, int grad_f32, int precise, int f16, cudaStream_t stream) {
+    if (f16)
+        return launch_dkdv_dp<D, false, true>(tq, tk, tv, tdo, tdq, rowstats, dq_accum, dk, dv,
+                                              BH, T, scale, causal, grad_f32, stream);
+    if (precise)
+        return launch_dkdv_dp<D, true, false>(tq, tk, tv, tdo, tdq, rowstats, dq_accum, dk, dv,
+                                              BH, T, scale, causal, grad_f32, stream);
+    return launch_dkdv_dp<D, false, false>(tq, tk, tv, tdo, tdq, rowstats, dq_accum, dk, dv, BH,
+                                           T, scale, causal, grad_f32, stream);
 }
 
 }  // namespace
 
 cudaError_t launch_bwd_preprocess(const void* o, const void* dO, const float* lse,
                                   float* rowstats, float* dq_accum, int BH, int T, int d,
-                                  int o_f32, cudaStream_t stream) {
-    if (d == 64) {
-        if (o_f32) launch_pre<64, float>(o, dO, lse, rowstats, dq_accum, BH, T, stream);
-        else launch_pre<64, __nv_bfloat16>(o, dO, lse, rowstats, dq_accum, BH, T, stream);
-    } else {
-        if (o_f32) launch_pre<128, float>(o, dO, lse, rowstats, dq_accum, BH, T, stream);
-        else launch_pre<128, __nv_bfloat16>(o, dO, lse, rowstats, dq_accum, BH, T, stream);
-    }
+                                  int o_f32, int f16, cudaStream_t stream) {
+    if (d == 64) launch_pre_d<64>(o, dO, lse, rowstats, dq_accum, BH, T, o_f32, f16, stream);
+    else launch_pre_d<128>(o, dO, lse, rowstats, dq_accum, BH, T, o_f32, f16, stream);
     return cudaGetLastError();
 }
 
 cudaError_t launch_bwd_dkdv(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             const CUtensorMap& tdo, const CUtensorMap& tdq, const float* rowstats,
                             float* dq_accum, void* dk, void* dv, int BH, int T, int d,
-                            float scale, int causal, int grad_f32, int precise,
+                            float scale, int causal, int grad_f32, int precise, int f16,
                             cudaStream_t stream) {
-    if (d == 64) {
-        if (precise)
-            return launch_dkdv_dp<64, true>(tq, tk, tv, tdo, tdq, rowstats, dq_accum, dk, dv, BH,
-                                            T, scale, causal, grad_f32, stream);
-        return launch_dkdv_dp<64, false>(tq, tk, tv, tdo, tdq, rowstats, dq_accum, dk, dv, BH, T,
-                                         scale, causal, grad_f32, stream);
-    }
-    if (precise)
-        return launch_dkdv_dp<128, true>(tq, tk, tv, tdo, tdq, rowstats, dq_accum, dk, dv, BH, T,
-                                         scale, causal, grad_f32, stream);
-    return launch_dkdv_dp<128, false>(tq, tk, tv, tdo, tdq, rowstats, dq_accum, dk, dv, BH, T,
-                                      scale, causal, grad_f32, stream);
+    if (d == 64)
+        return launch_dkdv_d<64>(tq, tk, tv, tdo, tdq, rowstats, dq_accum, dk, dv, BH, T, scale,
+                                 causal, grad_f32, precise, f16, stream);
+    return launch_dkdv_d<128>(tq, tk, tv, tdo, tdq, rowstats, dq_accum, dk, dv, BH, T, scale,
+                              causal, grad_f32, precise, f16, stream);
 }
 
-cudaError_t launch_bwd_dq_convert(const float* dq_accum, void* dq, long long n,
+cudaError_t launch_bwd_dq_convert(const float* dq_accum, void* dq, long long n, int f16,
                                   cudaStream_t stream) {
     const long long n8 = n / 8;  // d is a multiple of 8, so n is too
     const int threads = 256;
     const unsigned blocks = (unsigned)((n8 + threads - 1) / threads);
-    attn_bwd_dq_convert_kernel<<<blocks, threads, 0, stream>>>(
-        dq_accum, static_cast<__nv_bfloat16*>(dq), n8);
+    if (f16)
+        attn_bwd_dq_convert_kernel<true><<<blocks, threads, 0, stream>>>(
+            dq_accum, static_cast<uint16_t*>(dq), n8);
+    else
+        attn_bwd_dq_convert_kernel<false><<<blocks, threads, 0, stream>>>(
+            dq_accum, static_cast<uint16_t*>(dq), n8);
     return cudaGetLastError();
 }
 

@@ -16,8 +16,9 @@
 // heaviest first, zigzag over the CTAs, and every role walks the same item sequence,
 // so one item's epilogue and the next item's Q load overlap the neighbouring item's
 // products.
-//   warp 0      TMA producer: Q per item (once the item before has finished its
-//               score products), then K/V tiles into an NS-stage ring.
+//   warp 0      TMA producer: Q per item into one of two buffers (d = 64; one at
+//               d = 128), once the item that used the buffer before has finished its
+//               score products, then K/V tiles into an NS-stage ring.
 //   warp 1      MMA issuer (converged warp, one elected lane issues): S = Q K^T into
 //               TMEM, then O += P V with P read from TMEM (tcgen05.mma with A in
 //               tensor memory).  An item's first P V waits until the previous
@@ -59,14 +60,17 @@ enum : uint32_t {
     kSitePV, kSiteODone, kSiteQEmpty, kSiteOFree
 };
 
-template <int D>
+template <int D, bool F16>
 struct FwdCfg {
     static constexpr int kChunks = D / 64;               // 128-byte column chunks per row
     static constexpr int kChunkBytes = kTile * 128;      // 128 rows x 128 bytes
     static constexpr int kTileBytes = kChunks * kChunkBytes;
     static constexpr int kStages = D == 64 ? 4 : 3;
+    // Q buffers: with two (d = 64), the next item's Q is loaded while this item runs,
+    // so its first score product never waits for the load; d = 128 has room for one.
+    static constexpr int kQBufs = D == 64 ? 2 : 1;
     static constexpr int kOffQ = 0;
-    static constexpr int kOffK = kOffQ + kTileBytes;
+    static constexpr int kOffK = kOffQ + kQBufs * kTileBytes;
     static constexpr int kOffV = kOffK + kStages * kTileBytes;
     static constexpr int kOffBar = kOffV + kStages * kTileBytes;
     static constexpr int kBarBytes = 256;
@@ -78,12 +82,13 @@ struct FwdCfg {
     // half of precise mode in the next 64) is written over the S it came from
     static constexpr uint32_t kColS0 = 0, kColBuf = 128, kColPlo = 64, kColO = 256;
     static constexpr uint32_t kTmemCols = 512;
-    static constexpr uint32_t kIdescS = idesc_bf16_f32(128, 128, false, false);
-    static constexpr uint32_t kIdescPV = idesc_bf16_f32(128, D, false, true);
+    // Q, K, V and P are all bf16, or all fp16 (F16)
+    static constexpr uint32_t kIdescS = idesc_f16kind_f32(128, 128, false, false, F16);
+    static constexpr uint32_t kIdescPV = idesc_f16kind_f32(128, D, false, true, F16);
 };
 
 struct FwdBarriers {
-    uint64_t q_full, q_empty;
+    uint64_t q_full[2], q_empty[2];  // per Q buffer
     uint64_t k_full[4];
     uint64_t v_full[4];
     uint64_t kv_empty[4];
@@ -101,7 +106,7 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, uint32
     return __all_sync(0xffffffffu, mbar_wait(bar, parity, site, abort));
 }
 
-template <int D, bool PRECISE>
+template <int D, bool PRECISE, bool F16>
 __global__ void __launch_bounds__(kFwdThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
                     const __grid_constant__ CUtensorMap tmap_k,
@@ -109,8 +114,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                     void* __restrict__ o_out, float* __restrict__ lse_out, int T, int BH,
                     int n_qtiles, int n_items, float scale_log2, int negate_scores, int causal,
                     int o_f32) {
-    using C = FwdCfg<D>;
+    using C = FwdCfg<D, F16>;
     static_assert(sizeof(FwdBarriers) <= C::kBarBytes, "barrier block");
+    static_assert(!(PRECISE && F16), "the hi + lo split is a bf16-operand mode");
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -135,8 +141,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     const uint32_t lane = lane_id();
 
     if (threadIdx.x == 0) {
-        mbar_init(&bars->q_full, 1);
-        mbar_init(&bars->q_empty, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&bars->q_full[b], 1);
+            mbar_init(&bars->q_empty[b], 1);
+        }
         for (int s = 0; s < C::kStages; ++s) {
             mbar_init(&bars->k_full[s], 1);
             mbar_init(&bars->v_full[s], 1);
@@ -168,20 +176,22 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             tma_prefetch_desc(&tmap_q);
             tma_prefetch_desc(&tmap_k);
             tma_prefetch_desc(&tmap_v);
-            int last_use[4] = {-1, -1, -1, -1}, last_q = -1;
+            int last_use[4] = {-1, -1, -1, -1}, last_q[2] = {-1, -1};
             int g = 0;  // key tiles so far (all items)
             bool run = true;
             int bh, qt;
             for (int item = 0; run && item_of(item, bh, qt); ++item) {
-                // Q of the item, once the previous item's last score product has read Q
-                if (item > 0 &&
-                    !mbar_wait(&bars->q_empty, (item - 1) & 1, kSiteQEmpty, abort))
+                // Q of the item into its buffer, once the last score product of the item
+                // that used that buffer before has read it
+                const int qb = item % C::kQBufs, uq = item / C::kQBufs;
+                if (uq > 0 &&
+                    !mbar_wait(&bars->q_empty[qb], (uq - 1) & 1, kSiteQEmpty, abort))
                     break;
-                mbar_arrive_expect_tx(&bars->q_full, C::kTileBytes);
+                mbar_arrive_expect_tx(&bars->q_full[qb], C::kTileBytes);
                 for (int c = 0; c < C::kChunks; ++c)
-                    tma_load_3d(smem + C::kOffQ + c * C::kChunkBytes, &tmap_q, &bars->q_full,
-                                64 * c, qt * kTile, bh);
-                last_q = item;
+                    tma_load_3d(smem + C::kOffQ + qb * C::kTileBytes + c * C::kChunkBytes,
+                                &tmap_q, &bars->q_full[qb], 64 * c, qt * kTile, bh);
+                last_q[qb] = uq;
                 const int n_tiles = tiles_of(qt);
                 for (int n = 0; n < n_tiles; ++n, ++g) {
                     const int st = g % C::kStages;
@@ -205,7 +215,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             }
             if (*abort) {
                 // let copies already issued land before the CTA's memory is released
-                if (last_q >= 0) mbar_wait_drain(&bars->q_full, last_q & 1);
+                for (int b = 0; b < C::kQBufs; ++b)
+                    if (last_q[b] >= 0) mbar_wait_drain(&bars->q_full[b], last_q[b] & 1);
                 for (int s = 0; s < C::kStages; ++s)
                     if (last_use[s] >= 0) {
                         mbar_wait_drain(&bars->k_full[s], last_use[s] & 1);
@@ -218,7 +229,6 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         // The whole warp runs this loop; one elected lane issues each MMA.
         {
             const uint32_t tO = tmem + C::kColO;
-            const uint32_t q_addr = smem_u32(smem + C::kOffQ);
             // bit 13 of the instruction descriptor negates A: S = (-Q) K^T for scale < 0
             const uint32_t idesc_s = C::kIdescS | (negate_scores ? (1u << 13) : 0u);
             // Two cursors walk the CTA's key tiles over all items: the score products
@@ -251,7 +261,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             auto issue_s = [&](const Cursor& c) -> bool {
                 const int g = c.g;
                 const int st = g % C::kStages;
-                if (c.n == 0 && !warp_wait(&bars->q_full, c.item & 1, kSiteQ, abort)) return false;
+                const int qb = c.item % C::kQBufs;
+                if (c.n == 0 &&
+                    !warp_wait(&bars->q_full[qb], (c.item / C::kQBufs) & 1, kSiteQ, abort))
+                    return false;
                 if (!warp_wait(&bars->k_full[st], (g / C::kStages) & 1, kSiteKFull, abort))
                     return false;
                 if (g >= 2 && !warp_wait(&bars->pv_done, (g - 2) & 1, kSiteSFree, abort))
@@ -259,6 +272,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 tc_fence_after();
                 const uint32_t tS = tmem + C::kColS0 + (g & 1) * C::kColBuf;
                 const uint32_t k_addr = smem_u32(smem + C::kOffK + st * C::kTileBytes);
+                const uint32_t q_addr = smem_u32(smem + C::kOffQ + qb * C::kTileBytes);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t koff = (kk >> 2) * C::kChunkBytes + (kk & 3) * 32;
@@ -268,7 +282,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 }
                 mma_commit_warp(&bars->s_full[g & 1]);
                 // the item's last score product is the last reader of Q
-                if (c.n == c.n_tiles - 1) mma_commit_warp(&bars->q_empty);
+                if (c.n == c.n_tiles - 1) mma_commit_warp(&bars->q_empty[qb]);
                 return true;
             };
             // O += P(g) V(g).  An item's first P V overwrites O, so it waits until the
@@ -432,7 +446,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                         p.y = c + 1 > key_lim ? 0.f : p.y;
                     }
                     ls[e & 3] = fadd2(ls[e & 3], p);
-                    pk[e] = pack_bf16x2(p.x, p.y);
+                    pk[e] = pack16x2<F16>(p.x, p.y);
                     if (PRECISE)
                         pl[e] = pack_bf16x2(p.x - bf16_lo_to_float(pk[e]),
                                             p.y - bf16_hi_to_float(pk[e]));
@@ -479,17 +493,17 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                                              __uint_as_float(r[4 * e + 3]) * inv_l);
                 } else {
                     uint4* dst =
-                        reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(o_out) + base);
+                        reinterpret_cast<uint4*>(static_cast<uint16_t*>(o_out) + base);
 #pragma unroll
                     for (int e = 0; e < 4; ++e)
-                        dst[e] = make_uint4(pack_bf16x2(__uint_as_float(r[8 * e]) * inv_l,
-                                                        __uint_as_float(r[8 * e + 1]) * inv_l),
-                                            pack_bf16x2(__uint_as_float(r[8 * e + 2]) * inv_l,
-                                                        __uint_as_float(r[8 * e + 3]) * inv_l),
-                                            pack_bf16x2(__uint_as_float(r[8 * e + 4]) * inv_l,
-                                                        __uint_as_float(r[8 * e + 5]) * inv_l),
-                                            pack_bf16x2(__uint_as_float(r[8 * e + 6]) * inv_l,
-                                                        __uint_as_float(r[8 * e + 7]) * inv_l));
+                        dst[e] = make_uint4(pack16x2<F16>(__uint_as_float(r[8 * e]) * inv_l,
+                                                          __uint_as_float(r[8 * e + 1]) * inv_l),
+                                            pack16x2<F16>(__uint_as_float(r[8 * e + 2]) * inv_l,
+                                                          __uint_as_float(r[8 * e + 3]) * inv_l),
+                                            pack16x2<F16>(__uint_as_float(r[8 * e + 4]) * inv_l,
+                                                          __uint_as_float(r[8 * e + 5]) * inv_l),
+                                            pack16x2<F16>(__uint_as_float(r[8 * e + 6]) * inv_l,
+                                                          __uint_as_float(r[8 * e + 7]) * inv_l));
                 }
             }
         }
@@ -510,30 +524,19 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     }
 }
 
-int sm_count() {
-    static int n = 0;
-    if (n == 0) {
-        int dev = 0;
-        if (cudaGetDevice(&dev) != cudaSuccess ||
-            cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-            n <= 0)
-            n = 148;
-    }
-    return n;
-}
-
-template <int D, bool PRECISE>
+template <int D, bool PRECISE, bool F16>
 cudaError_t launch_fwd_dp(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                           void* o, float* lse, int BH, int T, float scale, int causal, int o_f32,
                           cudaStream_t stream) {
-    using C = FwdCfg<D>;
+    using C = FwdCfg<D, F16>;
     static std::atomic<unsigned long long> configured{0};
-    cudaError_t e = set_max_dynamic_smem(attn_fwd_kernel<D, PRECISE>, C::kSmemBytes, configured);
+    cudaError_t e =
+        set_max_dynamic_smem(attn_fwd_kernel<D, PRECISE, F16>, C::kSmemBytes, configured);
     if (e != cudaSuccess) return e;
     const int n_qtiles = (T + kTile - 1) / kTile;
     const int n_items = BH * n_qtiles;
     const int grid = n_items < sm_count() ? n_items : sm_count();
-    attn_fwd_kernel<D, PRECISE><<<grid, kFwdThreads, C::kSmemBytes, stream>>>(
+    attn_fwd_kernel<D, PRECISE, F16><<<grid, kFwdThreads, C::kSmemBytes, stream>>>(
         tq, tk, tv, o, lse, T, BH, n_qtiles, n_items, fabsf(scale) * kLog2e,
         scale < 0.f ? 1 : 0, causal, o_f32);
     return cudaGetLastError();
@@ -542,20 +545,26 @@ cudaError_t launch_fwd_dp(const CUtensorMap& tq, const CUtensorMap& tk, const CU
 template <int D>
 cudaError_t launch_fwd_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                          void* o, float* lse, int BH, int T, float scale, int causal, int o_f32,
-                         int precise, cudaStream_t stream) {
+                         int precise, int f16, cudaStream_t stream) {
+    if (f16)
+        return launch_fwd_dp<D, false, true>(tq, tk, tv, o, lse, BH, T, scale, causal, o_f32,
+                                             stream);
     if (precise)
-        return launch_fwd_dp<D, true>(tq, tk, tv, o, lse, BH, T, scale, causal, o_f32, stream);
-    return launch_fwd_dp<D, false>(tq, tk, tv, o, lse, BH, T, scale, causal, o_f32, stream);
+        return launch_fwd_dp<D, true, false>(tq, tk, tv, o, lse, BH, T, scale, causal, o_f32,
+                                             stream);
+    return launch_fwd_dp<D, false, false>(tq, tk, tv, o, lse, BH, T, scale, causal, o_f32, stream);
 }
 
 }  // namespace
 
 cudaError_t launch_attn_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             void* o, float* lse, int BH, int T, int d, float scale, int causal,
-                            int o_f32, int precise, cudaStream_t stream) {
+                            int o_f32, int precise, int f16, cudaStream_t stream) {
     if (d == 64)
-        return launch_fwd_d<64>(tq, tk, tv, o, lse, BH, T, scale, causal, o_f32, precise, stream);
-    return launch_fwd_d<128>(tq, tk, tv, o, lse, BH, T, scale, causal, o_f32, precise, stream);
+        return launch_fwd_d<64>(tq, tk, tv, o, lse, BH, T, scale, causal, o_f32, precise, f16,
+                                stream);
+    return launch_fwd_d<128>(tq, tk, tv, o, lse, BH, T, scale, causal, o_f32, precise, f16,
+                             stream);
 }
 
 cudaError_t read_and_clear_device_error_fwd(unsigned int* value) {

@@ -41,18 +41,20 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
-// bf16 tensor viewed as [planes][rows][inner] (inner contiguous), loaded in
-// {64, 128, 1} boxes with 128-byte swizzle.  Rows past `rows` read as zero and are
-// clipped on store, so a ragged last tile never touches the next plane.
-int make_map_bf16(CUtensorMap* map, const void* base, long long inner, long long rows,
-                  long long planes) {
+// 16-bit (bf16, or fp16 when f16) tensor viewed as [planes][rows][inner] (inner
+// contiguous), loaded in {64, 128, 1} boxes with 128-byte swizzle.  Rows past `rows`
+// read as zero and are clipped on store, so a ragged last tile never touches the next
+// plane.
+int make_map_16(CUtensorMap* map, const void* base, long long inner, long long rows,
+                long long planes, bool f16 = false) {
     auto fn = encode_fn();
     if (!fn) return FORGE_ATTN_ERR_CUDA;
     cuuint64_t dims[3] = {(cuuint64_t)inner, (cuuint64_t)rows, (cuuint64_t)planes};
     cuuint64_t strides[2] = {(cuuint64_t)(inner * 2), (cuuint64_t)(inner * rows * 2)};
     cuuint32_t box[3] = {64, 128, 1};
     cuuint32_t estr[3] = {1, 1, 1};
-    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+    CUresult r = fn(map, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                    3, const_cast<void*>(base), dims,
                     strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -133,18 +135,21 @@ int forge_attn_fwd_ex(const void* q, const void* k, const void* v, void* o, floa
     if (!q || !k || !v || !o || !lse) return FORGE_ATTN_ERR_INVALID_ARG;
     int s = check_common(B, H, T, d, scale, causal);
     if (s != FORGE_ATTN_OK) return s;
-    if (flags & ~(FORGE_ATTN_OUT_F32 | FORGE_ATTN_PRECISE)) return FORGE_ATTN_ERR_INVALID_ARG;
+    if (flags & ~(FORGE_ATTN_OUT_F32 | FORGE_ATTN_PRECISE | FORGE_ATTN_FP16))
+        return FORGE_ATTN_ERR_INVALID_ARG;
+    const bool f16 = (flags & FORGE_ATTN_FP16) != 0;
+    if (f16 && (flags & FORGE_ATTN_PRECISE)) return FORGE_ATTN_ERR_UNSUPPORTED;
     const bool o_f32 = (flags & FORGE_ATTN_OUT_F32) != 0;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
         (reinterpret_cast<uintptr_t>(lse) & 3u))
         return FORGE_ATTN_ERR_MISALIGNED;
     const long long BH = (long long)B * H;
     CUtensorMap tq, tk, tv;
-    if ((s = make_map_bf16(&tq, q, d, T, BH)) != FORGE_ATTN_OK) return s;
-    if ((s = make_map_bf16(&tk, k, d, T, BH)) != FORGE_ATTN_OK) return s;
-    if ((s = make_map_bf16(&tv, v, d, T, BH)) != FORGE_ATTN_OK) return s;
+    if ((s = make_map_16(&tq, q, d, T, BH, f16)) != FORGE_ATTN_OK) return s;
+    if ((s = make_map_16(&tk, k, d, T, BH, f16)) != FORGE_ATTN_OK) return s;
+    if ((s = make_map_16(&tv, v, d, T, BH, f16)) != FORGE_ATTN_OK) return s;
     return cuda_status(launch_attn_fwd(tq, tk, tv, o, lse, (int)BH, T, d, scale, causal,
-                                       o_f32, (flags & FORGE_ATTN_PRECISE) != 0,
+                                       o_f32, (flags & FORGE_ATTN_PRECISE) != 0, f16,
                                        static_cast<cudaStream_t>(stream)));
 }
 
@@ -165,12 +170,13 @@ int forge_attn_bwd_preprocess(const void* o, const void* dO, const float* lse, f
     if (!o || !dO || !lse || !rowstats) return FORGE_ATTN_ERR_INVALID_ARG;
     int s = check_shape(B, H, T, d);
     if (s != FORGE_ATTN_OK) return s;
-    if (flags & ~FORGE_ATTN_O_IN_F32) return FORGE_ATTN_ERR_INVALID_ARG;
+    if (flags & ~(FORGE_ATTN_O_IN_F32 | FORGE_ATTN_FP16)) return FORGE_ATTN_ERR_INVALID_ARG;
     if (!aligned16(o) || !aligned16(dO) || (reinterpret_cast<uintptr_t>(lse) & 3u) ||
         !aligned16(rowstats) || (dq_accum && !aligned16(dq_accum)))
         return FORGE_ATTN_ERR_MISALIGNED;
     return cuda_status(launch_bwd_preprocess(o, dO, lse, rowstats, dq_accum, B * H, T, d,
                                              (flags & FORGE_ATTN_O_IN_F32) != 0,
+                                             (flags & FORGE_ATTN_FP16) != 0,
                                              static_cast<cudaStream_t>(stream)));
 }
 
@@ -181,31 +187,41 @@ int forge_attn_bwd_dkdv(const void* q, const void* k, const void* v, const void*
         return FORGE_ATTN_ERR_INVALID_ARG;
     int s = check_common(B, H, T, d, scale, causal);
     if (s != FORGE_ATTN_OK) return s;
-    if (flags & ~(FORGE_ATTN_OUT_F32 | FORGE_ATTN_PRECISE)) return FORGE_ATTN_ERR_INVALID_ARG;
+    if (flags & ~(FORGE_ATTN_OUT_F32 | FORGE_ATTN_PRECISE | FORGE_ATTN_FP16))
+        return FORGE_ATTN_ERR_INVALID_ARG;
+    const bool f16 = (flags & FORGE_ATTN_FP16) != 0;
+    if (f16 && (flags & FORGE_ATTN_PRECISE)) return FORGE_ATTN_ERR_UNSUPPORTED;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dO) || !aligned16(dk) ||
         !aligned16(dv) || !aligned16(dq_accum) || !aligned16(rowstats))
         return FORGE_ATTN_ERR_MISALIGNED;
     const long long BH = (long long)B * H;
     CUtensorMap tq, tk, tv, tdo, tdq;
-    if ((s = make_map_bf16(&tq, q, d, T, BH)) != FORGE_ATTN_OK) return s;
-    if ((s = make_map_bf16(&tk, k, d, T, BH)) != FORGE_ATTN_OK) return s;
-    if ((s = make_map_bf16(&tv, v, d, T, BH)) != FORGE_ATTN_OK) return s;
-    if ((s = make_map_bf16(&tdo, dO, d, T, BH)) != FORGE_ATTN_OK) return s;
+    if ((s = make_map_16(&tq, q, d, T, BH, f16)) != FORGE_ATTN_OK) return s;
+    if ((s = make_map_16(&tk, k, d, T, BH, f16)) != FORGE_ATTN_OK) return s;
+    if ((s = make_map_16(&tv, v, d, T, BH, f16)) != FORGE_ATTN_OK) return s;
+    if ((s = make_map_16(&tdo, dO, d, T, BH, f16)) != FORGE_ATTN_OK) return s;
     if ((s = make_map_f32(&tdq, dq_accum, d, T, BH)) != FORGE_ATTN_OK) return s;
     return cuda_status(launch_bwd_dkdv(tq, tk, tv, tdo, tdq, rowstats, dq_accum, dk, dv, (int)BH, T,
                                        d, scale, causal, (flags & FORGE_ATTN_OUT_F32) != 0,
-                                       (flags & FORGE_ATTN_PRECISE) != 0,
+                                       (flags & FORGE_ATTN_PRECISE) != 0, f16,
                                        static_cast<cudaStream_t>(stream)));
+}
+
+int forge_attn_bwd_dq_convert_ex(const float* dq_accum, void* dq, int B, int H, int T, int d,
+                                 int flags, void* stream) {
+    if (!dq_accum || !dq) return FORGE_ATTN_ERR_INVALID_ARG;
+    int s = check_shape(B, H, T, d);
+    if (s != FORGE_ATTN_OK) return s;
+    if (flags & ~FORGE_ATTN_FP16) return FORGE_ATTN_ERR_INVALID_ARG;
+    if (!aligned16(dq_accum) || !aligned16(dq)) return FORGE_ATTN_ERR_MISALIGNED;
+    return cuda_status(launch_bwd_dq_convert(dq_accum, dq, (long long)B * H * T * d,
+                                             (flags & FORGE_ATTN_FP16) != 0,
+                                             static_cast<cudaStream_t>(stream)));
 }
 
 int forge_attn_bwd_dq_convert(const float* dq_accum, void* dq, int B, int H, int T, int d,
                               void* stream) {
-    if (!dq_accum || !dq) return FORGE_ATTN_ERR_INVALID_ARG;
-    int s = check_shape(B, H, T, d);
-    if (s != FORGE_ATTN_OK) return s;
-    if (!aligned16(dq_accum) || !aligned16(dq)) return FORGE_ATTN_ERR_MISALIGNED;
-    return cuda_status(launch_bwd_dq_convert(dq_accum, dq, (long long)B * H * T * d,
-                                             static_cast<cudaStream_t>(stream)));
+    return forge_attn_bwd_dq_convert_ex(dq_accum, dq, B, H, T, d, 0, stream);
 }
 
 int forge_attn_bwd_ex(const void* q, const void* k, const void* v, const void* o,
@@ -216,8 +232,9 @@ int forge_attn_bwd_ex(const void* q, const void* k, const void* v, const void* o
         return FORGE_ATTN_ERR_INVALID_ARG;
     int s = check_common(B, H, T, d, scale, causal);
     if (s != FORGE_ATTN_OK) return s;
-    if (flags & ~(FORGE_ATTN_OUT_F32 | FORGE_ATTN_O_IN_F32 | FORGE_ATTN_PRECISE))
+    if (flags & ~(FORGE_ATTN_OUT_F32 | FORGE_ATTN_O_IN_F32 | FORGE_ATTN_PRECISE | FORGE_ATTN_FP16))
         return FORGE_ATTN_ERR_INVALID_ARG;
+    if ((flags & FORGE_ATTN_FP16) && (flags & FORGE_ATTN_PRECISE)) return FORGE_ATTN_ERR_UNSUPPORTED;
     const bool grad_f32 = (flags & FORGE_ATTN_OUT_F32) != 0;
     const size_t need = forge_attn_bwd_workspace_size(B, H, T, d);
     if (!workspace || workspace_bytes < need) return FORGE_ATTN_ERR_WORKSPACE;
@@ -231,14 +248,15 @@ int forge_attn_bwd_ex(const void* q, const void* k, const void* v, const void* o
                           : reinterpret_cast<float*>(static_cast<char*>(workspace) +
                                                      rowstats_bytes(B, H, T));
     if ((s = forge_attn_bwd_preprocess(o, dO, lse, rowstats, acc, B, H, T, d,
-                                       flags & FORGE_ATTN_O_IN_F32, stream)) != FORGE_ATTN_OK)
+                                       flags & (FORGE_ATTN_O_IN_F32 | FORGE_ATTN_FP16),
+                                       stream)) != FORGE_ATTN_OK)
         return s;
     if ((s = forge_attn_bwd_dkdv(q, k, v, dO, rowstats, acc, dk, dv, B, H, T, d, scale, causal,
-                                 flags & (FORGE_ATTN_OUT_F32 | FORGE_ATTN_PRECISE), stream)) !=
-        FORGE_ATTN_OK)
+                                 flags & (FORGE_ATTN_OUT_F32 | FORGE_ATTN_PRECISE | FORGE_ATTN_FP16),
+                                 stream)) != FORGE_ATTN_OK)
         return s;
     if (!grad_f32)
-        s = forge_attn_bwd_dq_convert(acc, dq, B, H, T, d, stream);
+        s = forge_attn_bwd_dq_convert_ex(acc, dq, B, H, T, d, flags & FORGE_ATTN_FP16, stream);
     return s;
 }
 
@@ -269,14 +287,14 @@ int forge_probe_mma(const void* a, const void* b, float* d_out, int N, int K, in
     int s;
     // A: [128][K] (modes 0-2) or [K][128] (mode 3); B: [N][K] (mode 0) or [K][N]
     if (mode == 3)
-        s = make_map_bf16(&ta, a, 128, K, 1);
+        s = make_map_16(&ta, a, 128, K, 1);
     else
-        s = make_map_bf16(&ta, a, K, 128, 1);
+        s = make_map_16(&ta, a, K, 128, 1);
     if (s != FORGE_ATTN_OK) return s;
     if (mode == 0)
-        s = make_map_bf16(&tb, b, K, N, 1);
+        s = make_map_16(&tb, b, K, N, 1);
     else
-        s = make_map_bf16(&tb, b, N, K, 1);
+        s = make_map_16(&tb, b, N, K, 1);
     if (s != FORGE_ATTN_OK) return s;
     return cuda_status(
         launch_probe_mma(ta, tb, a, d_out, N, K, mode, static_cast<cudaStream_t>(stream)));

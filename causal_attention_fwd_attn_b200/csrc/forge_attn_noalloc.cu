@@ -29,26 +29,72 @@ namespace {
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[FORGE_ATTN_NOALLOC_SCRATCH_BYTES];
 
-constexpr int kMaxDevices = 64;
+// Device addresses of the array, one per CUDA context it was looked up in.  The
+// array's address belongs to the copy of the library's device code loaded into a
+// context; a new context on the same device (after cudaDeviceReset, or a
+// caller-created context) has its own copy, so entries are keyed by the context's
+// process-unique ID rather than by the device ordinal.
+struct ScratchEntry {
+    unsigned long long ctx_id;
+    void* addr;
+};
+constexpr int kMaxContexts = 64;
 std::mutex g_scratch_mutex;
-void* g_scratch_addr[kMaxDevices] = {};
+ScratchEntry g_scratch_addr[kMaxContexts] = {};
+int g_scratch_next = 0;
 
-// Device address of the scratch array on the current device.  The host-side name
+using GetCurrentFn = CUresult (*)(CUcontext*);
+using GetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+// ID of the calling thread's current context (0 when none is current or the driver
+// cannot say).
+unsigned long long current_context_id() {
+    static GetCurrentFn get_current = nullptr;
+    static GetIdFn get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) ==
+                cudaSuccess && q == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<GetCurrentFn>(p);
+        p = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<GetIdFn>(p);
+    });
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx) return 0;
+    if (get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+    return id;
+}
+
+// Device address of the scratch array in the current context.  The host-side name
 // g_noalloc_scratch is only a stand-in for the symbol; the address a kernel can use
-// comes from cudaGetSymbolAddress, taken once per device with that device current.
+// comes from cudaGetSymbolAddress, looked up once per context with that context
+// current (the first call in a context also loads the library's device code there).
 cudaError_t scratch_address(void** out) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
     std::lock_guard<std::mutex> lock(g_scratch_mutex);
-    if (!g_scratch_addr[dev]) {
-        void* p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-        if (e != cudaSuccess) return e;
-        g_scratch_addr[dev] = p;
+    unsigned long long id = current_context_id();
+    if (id != 0)
+        for (const ScratchEntry& s : g_scratch_addr)
+            if (s.ctx_id == id && s.addr) {
+                *out = s.addr;
+                return cudaSuccess;
+            }
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    if (id == 0) id = current_context_id();  // the lookup made the primary context current
+    if (id != 0) {
+        g_scratch_addr[g_scratch_next] = {id, p};
+        g_scratch_next = (g_scratch_next + 1) % kMaxContexts;
     }
-    *out = g_scratch_addr[dev];
+    *out = p;
     return cudaSuccess;
 }
 

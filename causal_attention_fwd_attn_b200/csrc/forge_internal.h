@@ -31,26 +31,46 @@ cudaError_t set_max_dynamic_smem(Kernel* kernel, int bytes,
     return e;
 }
 
+// Number of SMs of the current device: the persistent kernels launch one CTA per SM.
+// Cached per device ordinal (devices 64 and up query on every call); concurrent
+// first calls may both query, which is harmless.
+inline int sm_count() {
+    static std::atomic<int> cache[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    const bool cached = dev >= 0 && dev < 64;
+    if (cached) {
+        const int n = cache[dev].load(std::memory_order_relaxed);
+        if (n > 0) return n;
+    }
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+        return 148;
+    if (cached) cache[dev].store(n, std::memory_order_relaxed);
+    return n;
+}
+
 // Launchers.  Tensor maps describe bf16 [B*H][T][d] tensors with a
 // {64, 128, 1} box and 128-byte swizzle.
-// The one-query-tile persistent forward; o is bf16 or fp32 (o_f32).
+// f16: q, k, v (and dO) are fp16 and the 16-bit outputs are fp16; else bf16.
+// The one-query-tile persistent forward; o is 16-bit or fp32 (o_f32).
 cudaError_t launch_attn_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             void* o, float* lse, int BH, int T, int d, float scale, int causal,
-                            int o_f32, int precise, cudaStream_t stream);
+                            int o_f32, int precise, int f16, cudaStream_t stream);
 
 // Row statistics of the backward: fp32 [2][B*H][t_pad], t_pad = 128 * ceil(T / 128).
 cudaError_t launch_bwd_preprocess(const void* o, const void* dO, const float* lse,
                                   float* rowstats, float* dq_accum, int BH, int T, int d,
-                                  int o_f32, cudaStream_t stream);
+                                  int o_f32, int f16, cudaStream_t stream);
 
 // tdq: the fp32 dQ accumulator [B*H][T][d] in {32, 128, 1} boxes, 128-byte swizzle.
 cudaError_t launch_bwd_dkdv(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             const CUtensorMap& tdo, const CUtensorMap& tdq, const float* rowstats,
                             float* dq_accum, void* dk, void* dv, int BH, int T, int d,
-                            float scale, int causal, int grad_f32, int precise,
+                            float scale, int causal, int grad_f32, int precise, int f16,
                             cudaStream_t stream);
 
-cudaError_t launch_bwd_dq_convert(const float* dq_accum, void* dq, long long n,
+cudaError_t launch_bwd_dq_convert(const float* dq_accum, void* dq, long long n, int f16,
                                   cudaStream_t stream);
 
 cudaError_t launch_probe_mma(const CUtensorMap& ta, const CUtensorMap& tb, const void* a_raw,

@@ -8,6 +8,7 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -338,17 +339,22 @@ __device__ __forceinline__ void regs_inc() {
 }
 
 // ------------------------------------------------------------- descriptors --
-// Instruction descriptor for kind::f16 with bf16 A/B and an fp32 accumulator.
-// M in {64, 128}, N a multiple of 16 in [16, 256].  a_mn / b_mn select the
-// MN-major (transposed) operand layout.
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn, bool b_mn) {
+// Instruction descriptor for kind::f16 with an fp32 accumulator and A, B both bf16
+// (f16 = false) or both fp16 (f16 = true); the two operands always share one type.
+// M in {64, 128}, N a multiple of 16 in [16, 256].  a_mn / b_mn select the MN-major
+// (transposed) operand layout.
+__host__ __device__ constexpr uint32_t idesc_f16kind_f32(int M, int N, bool a_mn, bool b_mn,
+                                                         bool f16) {
     return (1u << 4)                               // D format: f32
-           | (1u << 7)                             // A format: bf16
-           | (1u << 10)                            // B format: bf16
+           | ((f16 ? 0u : 1u) << 7)                // A format: 0 fp16, 1 bf16
+           | ((f16 ? 0u : 1u) << 10)               // B format: the same as A
            | ((a_mn ? 1u : 0u) << 15)              // A major
            | ((b_mn ? 1u : 0u) << 16)              // B major
            | ((uint32_t)(N >> 3) << 17)            // N / 8
            | ((uint32_t)(M >> 4) << 24);           // M / 16
+}
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn, bool b_mn) {
+    return idesc_f16kind_f32(M, N, a_mn, b_mn, false);
 }
 
 // Shared-memory matrix descriptor, 128-byte swizzle (the layout TMA writes with
@@ -443,6 +449,28 @@ __device__ __forceinline__ float2 exp2_poly2(float2 x) {
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// Two fp32 values as a packed pair of 16-bit floats, round to nearest even: bf16, or
+// fp16 when F16 (the operand type of the tensor-core products).
+template <bool F16>
+__device__ __forceinline__ uint32_t pack16x2(float lo, float hi) {
+    if constexpr (F16) {
+        __half2 h = __floats2half2_rn(lo, hi);
+        return *reinterpret_cast<uint32_t*>(&h);
+    } else {
+        return pack_bf16x2(lo, hi);
+    }
+}
+
+// A packed pair of 16-bit floats (bf16, or fp16 when F16) back to fp32 (exact).
+template <bool F16>
+__device__ __forceinline__ float2 unpack16x2(uint32_t packed) {
+    if constexpr (F16) {
+        return __half22float2(*reinterpret_cast<const __half2*>(&packed));
+    } else {
+        return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&packed));
+    }
 }
 
 // The two bf16 halves of a packed pair, back to fp32 (exact).

@@ -20,7 +20,9 @@
  *               library never allocates or frees device memory.
  *   Layout      q, k, v, o, dO, dq, dk, dv are contiguous row-major [B][H][T][d]
  *               (d fastest).  lse and the backward's D are fp32 [B][H][T].
- *               Elements are bf16 bit patterns unless an option bit says fp32.
+ *               Elements are bf16 bit patterns unless an option bit says fp32
+ *               (FORGE_ATTN_OUT_F32, FORGE_ATTN_O_IN_F32) or fp16
+ *               (FORGE_ATTN_FP16).
  *   Alignment   Every tensor base must be 16-byte aligned (a TMA requirement);
  *               the workspace must be 256-byte aligned.
  *   Aliasing    Outputs must not overlap inputs or each other.
@@ -77,10 +79,21 @@ typedef enum {
  *                      accumulated.  Costs one extra product per split operand;
  *                      lowers the operand rounding error from ~2^-9 to ~2^-17
  *                      relative.
+ * FORGE_ATTN_FP16      fp16 instead of bf16 for every 16-bit tensor: the inputs q,
+ *                      k, v, dO and the 16-bit outputs (o, dq, dk, dv, unless
+ *                      FORGE_ATTN_OUT_F32 makes them fp32).  P and dS then enter
+ *                      the tensor-core products as fp16 (relative rounding 2^-11
+ *                      instead of bf16's 2^-8), with fp32 accumulation as before.
+ *                      fp16's range ends at 65504: inputs, outputs and scores
+ *                      gradients must stay within it.  Not combinable with
+ *                      FORGE_ATTN_PRECISE (FORGE_ATTN_ERR_UNSUPPORTED).
+ *                      (The paper's operand-type comparison, section "Finding 4",
+ *                      measures half and bfloat operands side by side.)
  */
 #define FORGE_ATTN_OUT_F32 1
 #define FORGE_ATTN_O_IN_F32 2
 #define FORGE_ATTN_PRECISE 4
+#define FORGE_ATTN_FP16 8
 
 /*
  * Forward.  Reads q, k, v (bf16 [B][H][T][d]); writes o (bf16 [B][H][T][d]) and
@@ -90,7 +103,7 @@ typedef enum {
 int forge_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                    int H, int T, int d, float scale, int causal, void* stream);
 
-/* Forward with option bits (FORGE_ATTN_OUT_F32, FORGE_ATTN_PRECISE). */
+/* Forward with option bits (FORGE_ATTN_OUT_F32, FORGE_ATTN_PRECISE, FORGE_ATTN_FP16). */
 int forge_attn_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                       int H, int T, int d, float scale, int causal, int flags, void* stream);
 
@@ -119,8 +132,8 @@ int forge_attn_bwd(const void* q, const void* k, const void* v, const void* o, c
                    void* stream);
 
 /* Backward with option bits (FORGE_ATTN_OUT_F32, FORGE_ATTN_O_IN_F32,
- * FORGE_ATTN_PRECISE).  With FORGE_ATTN_OUT_F32 the dQ accumulator is dq itself
- * and the conversion launch is skipped. */
+ * FORGE_ATTN_PRECISE, FORGE_ATTN_FP16).  With FORGE_ATTN_OUT_F32 the dQ accumulator
+ * is dq itself and the conversion launch is skipped. */
 int forge_attn_bwd_ex(const void* q, const void* k, const void* v, const void* o,
                       const void* dO, const float* lse, void* dq, void* dk, void* dv,
                       void* workspace, size_t workspace_bytes, int B, int H, int T, int d,
@@ -134,11 +147,13 @@ int forge_attn_bwd_ex(const void* q, const void* k, const void* v, const void* o
  *   t_pad = 128 * ceil(T / 128), 16-byte aligned): rowstats[0][bh][t] = -lse * log2(e)
  *   and rowstats[1][bh][t] = D = sum_k dO[t][k] * o[t][k], with -inf and 0 in the
  *   padding rows t >= T; and dq_accum (fp32 [B][H][T][d]) set to zero unless it is
- *   NULL.  flags: FORGE_ATTN_O_IN_F32 (o is fp32).
+ *   NULL.  flags: FORGE_ATTN_O_IN_F32 (o is fp32), FORGE_ATTN_FP16 (dO, and o
+ *   unless fp32, are fp16).
  * forge_attn_bwd_dkdv: recomputes P per key tile from the row statistics, writes dk
  *   and dv, and adds scale * dS K into dq_accum (TMA reduce-add).  flags:
- *   FORGE_ATTN_OUT_F32 (dk, dv fp32), FORGE_ATTN_PRECISE.
- * forge_attn_bwd_dq_convert: dq = bf16(dq_accum).  Only needed for bf16 dq.
+ *   FORGE_ATTN_OUT_F32 (dk, dv fp32), FORGE_ATTN_PRECISE, FORGE_ATTN_FP16.
+ * forge_attn_bwd_dq_convert: dq = bf16(dq_accum).  Only needed for 16-bit dq;
+ *   forge_attn_bwd_dq_convert_ex with FORGE_ATTN_FP16 writes fp16.
  */
 int forge_attn_bwd_preprocess(const void* o, const void* dO, const float* lse, float* rowstats,
                               float* dq_accum, int B, int H, int T, int d, int flags,
@@ -148,6 +163,8 @@ int forge_attn_bwd_dkdv(const void* q, const void* k, const void* v, const void*
                         int T, int d, float scale, int causal, int flags, void* stream);
 int forge_attn_bwd_dq_convert(const float* dq_accum, void* dq, int B, int H, int T, int d,
                               void* stream);
+int forge_attn_bwd_dq_convert_ex(const float* dq_accum, void* dq, int B, int H, int T, int d,
+                                 int flags, void* stream);
 
 /*
  * Bytes of the fixed device array that forge_attn_bwd_noalloc uses in place of a
@@ -170,9 +187,10 @@ int forge_attn_bwd_dq_convert(const float* dq_accum, void* dq, int B, int H, int
  * made.
  *   - Sizes whose forge_attn_bwd_workspace_size() exceeds the array are refused
  *     with FORGE_ATTN_ERR_WORKSPACE before any launch.
- *   - The first call on a device looks up the array's device address (once per
- *     device, with that device current); make that first call before any stream
- *     capture begins.
+ *   - The first call in a CUDA context (once per device, and again in the new
+ *     primary context after cudaDeviceReset) looks up the array's device address
+ *     with that context current; make that first call before any stream capture
+ *     begins.
  *   - All calls on a device share the array, which keeps the last call's contents;
  *     each call rewrites the row statistics and clears the accumulator first.  Calls whose kernels
  *     can overlap on the GPU (unordered streams) race on the array and must not be

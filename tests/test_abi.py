@@ -10,7 +10,8 @@ import pytest
 from causal_attention_fwd_attn_b200 import _lib, build
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-HEADERS = [os.path.join(ROOT, "include", h) for h in ("forge_attn.h", "forge_attn_testing.h")]
+HEADERS = [os.path.join(ROOT, "include", h)
+           for h in ("forge_attn.h", "forge_attn_testing.h", "forge_adamw.h")]
 
 
 @pytest.fixture(scope="module")
@@ -83,8 +84,11 @@ def test_fwd_rejects_bad_arguments(lib, args, want):
 
 
 def test_fwd_rejects_unknown_flags(lib):
-    assert _lib.forge_attn_fwd_ex(P, P, P, P, P, 1, 1, 8, 64, 0.1, 1, 8, None) == \
+    assert _lib.forge_attn_fwd_ex(P, P, P, P, P, 1, 1, 8, 64, 0.1, 1, 16, None) == \
         _lib.ERR_INVALID_ARG
+    # fp16 operands and the bf16 hi + lo split do not combine
+    assert _lib.forge_attn_fwd_ex(P, P, P, P, P, 1, 1, 8, 64, 0.1, 1,
+                                  _lib.FP16 | _lib.PRECISE, None) == _lib.ERR_UNSUPPORTED
     # O_IN_F32 means nothing to the forward
     assert _lib.forge_attn_fwd_ex(P, P, P, P, P, 1, 1, 8, 64, 0.1, 1, _lib.O_IN_F32, None) == \
         _lib.ERR_INVALID_ARG
@@ -106,7 +110,8 @@ def test_bwd_rejects_bad_arguments(lib):
     bad = list(good)
     bad[14] = 80
     assert _lib.forge_attn_bwd(*bad, None) == _lib.ERR_UNSUPPORTED
-    assert _lib.forge_attn_bwd_ex(*good, 8, None) == _lib.ERR_INVALID_ARG
+    assert _lib.forge_attn_bwd_ex(*good, 16, None) == _lib.ERR_INVALID_ARG
+    assert _lib.forge_attn_bwd_ex(*good, _lib.FP16 | _lib.PRECISE, None) == _lib.ERR_UNSUPPORTED
 
 
 def test_stage_entry_points_reject_bad_arguments(lib):
@@ -121,6 +126,10 @@ def test_stage_entry_points_reject_bad_arguments(lib):
     assert _lib.forge_attn_bwd_dkdv(P, P, P, P, P, 0, P, P, 1, 1, 8, 64, 0.1, 1, 0, None) == \
         _lib.ERR_INVALID_ARG
     assert _lib.forge_attn_bwd_dq_convert(P, P, 1, 1, 8, 48, None) == _lib.ERR_UNSUPPORTED
+    assert _lib.forge_attn_bwd_dq_convert_ex(P, P, 1, 1, 8, 64, _lib.PRECISE, None) == \
+        _lib.ERR_INVALID_ARG
+    assert _lib.forge_attn_bwd_dkdv(P, P, P, P, P, P, P, P, 1, 1, 8, 64, 0.1, 1,
+                                    _lib.FP16 | _lib.PRECISE, None) == _lib.ERR_UNSUPPORTED
     assert _lib.forge_probe_mma(P, P, P, 96, 64, 0, None) == _lib.ERR_INVALID_ARG
     assert _lib.forge_probe_mma(P, P, P, 64, 64, 9, None) == _lib.ERR_INVALID_ARG
 
@@ -135,3 +144,23 @@ def test_library_has_no_oracle_dependency(lib):
     names = open(_lib.library_path(), "rb").read()
     assert b"oracle_attn" not in names
     assert ctypes.CDLL(_lib.library_path())  # loads without a GPU
+
+
+def test_adamw_rejects_bad_arguments(lib):
+    ws_n = _lib.forge_adamw_workspace_size(1)
+    assert ws_n >= 16 and _lib.forge_adamw_workspace_size(0) == 0
+    ok = [(P, P + 256, P + 512, P + 768, 8, 1)]
+    common = dict(lr=1e-3, beta1=0.9, beta2=0.95, eps=1e-8, weight_decay=0.1, max_norm=1.0,
+                  grad_norm_out=None, workspace=P + 4096, stream=None)
+    assert _lib.forge_adamw_step(ok, step=0, workspace_bytes=ws_n, **common) == \
+        _lib.ERR_INVALID_ARG
+    assert _lib.forge_adamw_step([(P + 4, P, P, P, 8, 1)], step=1, workspace_bytes=ws_n,
+                                 **common) == _lib.ERR_MISALIGNED
+    assert _lib.forge_adamw_step(ok, step=1, workspace_bytes=ws_n - 1, **common) == \
+        _lib.ERR_WORKSPACE
+    assert _lib.forge_adamw_step([(P, P, P, P, 0, 1)], step=1, workspace_bytes=ws_n,
+                                 **common) == _lib.ERR_INVALID_ARG
+    assert _lib.forge_adamw_step(ok, step=1, workspace_bytes=ws_n,
+                                 **dict(common, beta2=1.0)) == _lib.ERR_INVALID_ARG
+    assert _lib.forge_adamw_step([], step=1, workspace_bytes=ws_n, **common) == \
+        _lib.ERR_INVALID_ARG
