@@ -473,6 +473,137 @@ def run_sub_results(rank, world, dev, clocks, peaks, warmup):
     return out
 
 
+# ------------------------------------------- the other hot-path kernels -------
+# The projection GEMMs around attention and the fused AdamW step, each timed over at
+# least SUB_RESULT_SECONDS with input sets rotating through more than the L2.
+GEMM_SUB_RESULTS = [
+    # (name, tokens, in_features, out_features, product)
+    ("square4096_fwd", 4096, 4096, 4096, "fwd"),
+    ("gpt2small_mlp_fc_fwd", 8192, 768, 3072, "fwd"),
+    ("gpt2small_mlp_fc_dx", 8192, 768, 3072, "dx"),
+    ("gpt2small_mlp_fc_dw", 8192, 768, 3072, "dw"),
+]
+
+
+def gemm_flops(tokens, din, dout):
+    return 2.0 * tokens * din * dout
+
+
+def time_loop(fn, n_sets, world, dev, clocks, warmup=3):
+    """fn(i) launches step i; sizes the timed loop to SUB_RESULT_SECONDS from three
+    probe steps (agreed over ranks) and returns (steps, max-over-ranks ms, clock stats)."""
+    stream = torch.cuda.current_stream(dev)
+    for i in range(warmup):
+        fn(i % n_sets)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(3):
+        fn(i % n_sets)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    est = max_over_ranks(t0.elapsed_time(t1) / 3, world, dev)
+    steps = max(20, min(50000, math.ceil(SUB_RESULT_SECONDS * 1e3 / max(est, 1e-4))))
+    barrier(world)
+    torch.cuda.synchronize()
+    lo = clocks.now()
+    t0.record(stream)
+    for i in range(steps):
+        fn(i % n_sets)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    hi = clocks.now()
+    barrier(world)
+    return steps, max_over_ranks(t0.elapsed_time(t1), world, dev), clocks.stats(lo, hi)
+
+
+def run_gemm_sub_results(rank, world, dev, clocks, peaks):
+    from causal_attention_fwd_attn_b200 import _lib
+
+    out = []
+    s = torch.cuda.current_stream(dev).cuda_stream
+    for name, tokens, din, dout, prod in GEMM_SUB_RESULTS:
+        set_bytes = 2 * (tokens * din + dout * din + tokens * dout)
+        n_sets = max(2, math.ceil(3 * L2_BYTES / set_bytes))
+        sets = []
+        for k in range(n_sets):
+            seed = 9000 + 10 * k + 97 * rank
+            sets.append({"x": wl.gaussian_bf16((tokens, din), 1.0, seed).to(dev),
+                         "w": wl.gaussian_bf16((dout, din), 1.0, seed + 1).to(dev),
+                         "dy": wl.gaussian_bf16((tokens, dout), 1.0, seed + 2).to(dev)})
+        if prod == "fwd":
+            y = torch.empty((tokens, dout), dtype=torch.bfloat16, device=dev)
+
+            def fn(i):
+                x = sets[i]
+                _lib.check(_lib.forge_linear_fwd(x["x"].data_ptr(), x["w"].data_ptr(),
+                                                 y.data_ptr(), tokens, din, dout, 0, s), name)
+        elif prod == "dx":
+            y = torch.empty((tokens, din), dtype=torch.bfloat16, device=dev)
+
+            def fn(i):
+                x = sets[i]
+                _lib.check(_lib.forge_linear_bwd_dx(x["dy"].data_ptr(), x["w"].data_ptr(),
+                                                    y.data_ptr(), tokens, din, dout, 0, s), name)
+        else:
+            y = torch.empty((dout, din), dtype=torch.float32, device=dev)
+
+            def fn(i):
+                x = sets[i]
+                _lib.check(_lib.forge_linear_bwd_dw(x["dy"].data_ptr(), x["x"].data_ptr(),
+                                                    y.data_ptr(), tokens, din, dout, 0, 0, 0,
+                                                    s), name)
+        steps, ms, clk = time_loop(fn, n_sets, world, dev, clocks)
+        tf = job_tflops(gemm_flops(tokens, din, dout), steps, world, ms)
+        out.append({"workload": name, "kind": "gemm", "tokens": tokens, "in": din, "out": dout,
+                    "product": prod, "steps": steps, "ms_per_step": round(ms / steps, 4),
+                    "value": round(tf, 2), "unit": UNIT,
+                    "frac_of_bf16_peak": round(tf / world / peaks["bf16_tflops"], 4),
+                    "split_k": (_lib.forge_linear_split_k(tokens, din, dout)
+                                if prod == "dw" else None),
+                    "clocks": {k: clk.get(k) for k in ("sm_mhz", "samples", "reasons")}})
+        del sets, y
+        torch.cuda.empty_cache()
+    return out
+
+
+def run_adamw_sub_result(rank, world, dev, clocks, peaks):
+    """One AdamW step over GPT-2-small-shaped parameters (148 tensors, 124.4M values):
+    algorithmic bytes 32 per parameter (norm pass reads the gradient; the update reads
+    parameter, gradient and both moments and writes parameter and both moments)."""
+    from causal_attention_fwd_attn_b200 import _lib
+
+    shapes = wl.gpt2small_param_shapes()
+    host = wl.make_adamw_inputs(shapes, 7000 + rank)
+    t = [{k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
+         for x in host]
+    del host
+    n_params = sum(x["param"].numel() for x in t)
+    table = [(x["param"].data_ptr(), x["grad"].data_ptr(), x["exp_avg"].data_ptr(),
+              x["exp_avg_sq"].data_ptr(), x["param"].numel(), int(x["decay"])) for x in t]
+    ws_n = _lib.forge_adamw_workspace_size(len(table))
+    ws = torch.empty(ws_n, dtype=torch.uint8, device=dev)
+    s = torch.cuda.current_stream(dev).cuda_stream
+    state = {"step": 0}
+
+    def fn(i):
+        state["step"] += 1
+        _lib.check(_lib.forge_adamw_step(table, 3e-4, 0.9, 0.95, 1e-8, 0.1, state["step"], 1.0,
+                                         None, ws.data_ptr(), ws_n, s), "adamw")
+
+    steps, ms, clk = time_loop(fn, 1, world, dev, clocks)
+    per_step = ms / steps
+    gbs = 32.0 * n_params / (per_step * 1e-3) / 1e9
+    res = {"workload": "adamw_gpt2small_124m", "kind": "adamw", "tensors": len(table),
+           "params": n_params, "steps": steps, "ms_per_step": round(per_step, 4),
+           "value": round(gbs * world, 1), "unit": "GB/s",
+           "frac_of_hbm_peak": round(gbs / peaks["hbm_gbs"], 4),
+           "algorithmic_bytes_per_step": 32 * n_params,
+           "clocks": {k: clk.get(k) for k in ("sm_mhz", "samples", "reasons")}}
+    del t, ws
+    torch.cuda.empty_cache()
+    return res
+
+
 def run_ours(args, rank, world, local_rank):
     from causal_attention_fwd_attn_b200 import _lib
 
@@ -494,6 +625,8 @@ def run_ours(args, rank, world, local_rank):
         subs = None
         if not args.no_sub_results:
             subs = run_sub_results(rank, world, dev, clocks, peaks, 3)
+            subs += run_gemm_sub_results(rank, world, dev, clocks, peaks)
+            subs.append(run_adamw_sub_result(rank, world, dev, clocks, peaks))
     finally:
         clocks.stop()
     if rank != 0:

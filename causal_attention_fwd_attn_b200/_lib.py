@@ -36,6 +36,7 @@ EXPORTED = [
     "forge_attn_bwd_dq_convert", "forge_attn_bwd_dq_convert_ex", "forge_attn_status_string",
     "forge_attn_check_device_error", "forge_attn_version", "forge_probe_mma", "forge_probe_wait_timeout",
     "forge_attn_bwd_noalloc", "forge_adamw_workspace_size", "forge_adamw_step",
+    "forge_linear_fwd", "forge_linear_bwd_dx", "forge_linear_bwd_dw", "forge_linear_split_k",
 ]
 
 ADAMW_MAX_TENSORS_PER_LAUNCH = 256
@@ -74,6 +75,10 @@ _SIGNATURES = {
     "forge_attn_bwd_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i,
                                     _f, _i, _vp]),
     "forge_adamw_workspace_size": (_sz, [_i]),
+    "forge_linear_fwd": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _vp]),
+    "forge_linear_bwd_dx": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _vp]),
+    "forge_linear_bwd_dw": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp]),
+    "forge_linear_split_k": (_i, [_i, _i, _i]),
     "forge_adamw_step": (_i, [ctypes.POINTER(AdamWTensor), _i, _f, _f, _f, _f, _f, _i, _f, _vp,
                               _vp, _sz, _vp]),
 }
@@ -190,6 +195,25 @@ def forge_adamw_step(tensors, lr, beta1, beta2, eps, weight_decay, step, max_nor
         arr[i] = t if isinstance(t, AdamWTensor) else AdamWTensor(*t)
     return load().forge_adamw_step(arr, len(tensors), lr, beta1, beta2, eps, weight_decay, step,
                                    max_norm, grad_norm_out, workspace, workspace_bytes, stream)
+
+
+def forge_linear_fwd(x, w, y, tokens, in_features, out_features, flags, stream):
+    return load().forge_linear_fwd(x, w, y, tokens, in_features, out_features, flags, stream)
+
+
+def forge_linear_bwd_dx(dy, w, dx, tokens, in_features, out_features, flags, stream):
+    return load().forge_linear_bwd_dx(dy, w, dx, tokens, in_features, out_features, flags,
+                                      stream)
+
+
+def forge_linear_bwd_dw(dy, x, dw, tokens, in_features, out_features, split_k, accumulate,
+                        flags, stream):
+    return load().forge_linear_bwd_dw(dy, x, dw, tokens, in_features, out_features, split_k,
+                                      accumulate, flags, stream)
+
+
+def forge_linear_split_k(tokens, in_features, out_features):
+    return load().forge_linear_split_k(tokens, in_features, out_features)
 
 
 def forge_attn_check_device_error(stream):

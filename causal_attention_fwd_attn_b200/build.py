@@ -20,7 +20,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIBRARY = os.path.join(PKG, "libforge_attn.so")
 SOURCES = ["forge_attn_api.cu", "attn_fwd.cu", "attn_bwd.cu", "tc_probe.cu", "forge_attn_noalloc.cu",
-           "adamw.cu"]
+           "adamw.cu", "gemm.cu"]
 HEADERS = ["sm100_ptx.cuh", "forge_internal.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
@@ -34,7 +34,8 @@ def nvcc_path() -> str:
 
 def _inputs():
     files = [os.path.join(CSRC, s) for s in SOURCES + HEADERS]
-    files += [os.path.join(INCLUDE, h) for h in ("forge_attn.h", "forge_attn_testing.h", "forge_adamw.h")]
+    files += [os.path.join(INCLUDE, h) for h in ("forge_attn.h", "forge_attn_testing.h", "forge_adamw.h",
+                                                        "forge_linear.h")]
     return files
 
 

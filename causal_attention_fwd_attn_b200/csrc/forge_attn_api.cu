@@ -21,6 +21,7 @@ cudaError_t read_and_clear_device_error(unsigned int* value, cudaStream_t stream
     if ((e = read_and_clear_device_error_fwd(&v)) != cudaSuccess) return e;
     if ((e = read_and_clear_device_error_bwd(&v)) != cudaSuccess) return e;
     if ((e = read_and_clear_device_error_probe(&v)) != cudaSuccess) return e;
+    if ((e = read_and_clear_device_error_gemm(&v)) != cudaSuccess) return e;
     *value = v;
     return cudaSuccess;
 }
@@ -79,6 +80,27 @@ int make_map_f32(CUtensorMap* map, const void* base, long long inner, long long 
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+
+// 2-D 16-bit tensor [rows][inner] (inner contiguous) in {box_inner, box_rows} boxes,
+// 128-byte swizzle, zero fill outside the tensor.
+cudaError_t encode_map_2d16(CUtensorMap* map, const void* base, long long inner, long long rows,
+                            int box_inner, int box_rows, bool f16) {
+    auto fn = encode_fn();
+    if (!fn) return cudaErrorNotSupported;
+    cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)(inner * 2)};
+    cuuint32_t box[2] = {(cuuint32_t)box_inner, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                    2, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+namespace {
 
 int check_shape(int B, int H, int T, int d) {
     if (B < 1 || H < 1 || T < 1 || d < 1) return FORGE_ATTN_ERR_INVALID_ARG;

@@ -83,5 +83,11 @@ cudaError_t launch_probe_wait_timeout(unsigned long long limit_ns, cudaStream_t 
 cudaError_t read_and_clear_device_error_fwd(unsigned int* value);
 cudaError_t read_and_clear_device_error_bwd(unsigned int* value);
 cudaError_t read_and_clear_device_error_probe(unsigned int* value);
+cudaError_t read_and_clear_device_error_gemm(unsigned int* value);
+
+// 2-D 16-bit tensor map: [rows][inner] (inner contiguous), {box_inner, box_rows} boxes,
+// 128-byte swizzle, zero fill outside the tensor (defined with the C ABI).
+cudaError_t encode_map_2d16(CUtensorMap* map, const void* base, long long inner, long long rows,
+                            int box_inner, int box_rows, bool f16);
 
 }  // namespace forge

@@ -1,0 +1,447 @@
+// gemm.cu -- the projection GEMMs around attention on tcgen05 tensor cores.
+//
+// The Forge paper ("Building an LLM Training Framework from Scratch in C++ and Metal
+// on Apple Silicon") measures, besides attention, the three products of a linear
+// layer in training (section "Results", the GEMM table; section "Finding 4.2" for
+// the transposed variants):
+//   forward   Y  = X W^T     [tokens][out] = [tokens][in] x [out][in]^T
+//   backward  dX = dY W      [tokens][in]  = [tokens][out] x [out][in]
+//             dW = dY^T X    [out][in]     = [tokens][out]^T x [tokens][in]
+// and notes that dW lags because its reduction runs over all tokens with few output
+// tiles, which split-K would fix.  All three are one kernel here,
+//   C[m][n] = sum_k A[m][k] B[n][k],
+// with each operand either K-major (stored [rows][k]) or MN-major (stored [k][rows]):
+//   Y : A = X  (K-major), B = W  (K-major)
+//   dX: A = dY (K-major), B = W  (MN-major: W is stored [out = k][in = n])
+//   dW: A = dY (MN-major), B = X (MN-major), k = tokens, split over k.
+// The transposes are descriptor choices (the operand-role exchange the paper uses for
+// its transposed attention products), never data movement.
+//
+// Design (persistent, one CTA per SM, 6 warps):
+//   warp 0      TMA producer: A and B k-blocks (64 deep) into a kStages ring.
+//   warp 1      MMA issuer (converged warp, one elected lane): 128 x BN x 16
+//               tcgen05 products into one of two tensor-memory accumulators, so one
+//               tile's epilogue overlaps the next tile's products.
+//   warps 2..5  epilogue: warp w reads TMEM lanes 32 (w % 4).. (its 32 rows of the
+//               tile), converts and stores them, or adds them (fp32 reductions) into C
+//               for split-K and accumulation.
+// Work units are (split, tile) pairs walked by all CTAs in the same order; tiles are
+// grouped eight M-rows at a time so the CTAs live at once share operand panels in L2.
+#include "forge_internal.h"
+#include "forge_linear.h"
+#include "forge_attn.h"
+#include "sm100_ptx.cuh"
+
+namespace forge {
+namespace {
+
+constexpr int kGemmThreads = 192;
+constexpr int kBM = 128, kBK = 64;
+constexpr int kGroupM = 8;
+
+enum : uint32_t { kGSiteFull = 1, kGSiteEmpty, kGSiteAccFull, kGSiteAccEmpty };
+enum OutMode : int { kOut16 = 0, kOutF32 = 1, kOutF32Add = 2 };
+
+template <int BN>
+struct GemmCfg {
+    static constexpr int kABytes = kBM * kBK * 2;  // 16 KB
+    static constexpr int kBBytes = BN * kBK * 2;   // 16 or 32 KB
+    static constexpr int kStageBytes = kABytes + kBBytes;
+    static constexpr int kStages = BN == 256 ? 4 : 6;
+    static constexpr int kChunkBytes = kBK * 128;  // one 64-element MN chunk of a k-block
+    static constexpr int kOffBar = kStages * kStageBytes;
+    static constexpr int kSmemBytes = kOffBar + 256 + 1024;
+    static_assert(kSmemBytes <= 232448, "shared memory budget");
+    static constexpr uint32_t kTmemCols = 2 * BN;  // two accumulators
+};
+
+struct GemmBarriers {
+    uint64_t full[6], empty[6];
+    uint64_t acc_full[2], acc_empty[2];
+    uint64_t mma_final;
+    uint32_t tmem_base;
+    int abort;
+};
+static_assert(sizeof(GemmBarriers) <= 256, "barrier block");
+
+struct GemmShape {
+    int M, N, K;
+    int tiles_m, tiles_n, k_blocks, kb_per_split, splits, units;
+};
+
+// Tile (tm, tn) and k-block range of work unit u.
+__device__ __forceinline__ void unit_of(const GemmShape& s, int u, int& tm, int& tn, int& kb0,
+                                        int& kb1) {
+    const int tiles = s.tiles_m * s.tiles_n;
+    const int split = u / tiles;
+    const int t = u - split * tiles;
+    // groups of kGroupM tile rows, column-major inside a group
+    const int per_group = kGroupM * s.tiles_n;
+    const int grp = t / per_group;
+    const int first_m = grp * kGroupM;
+    const int rows = min(kGroupM, s.tiles_m - first_m);
+    const int r = t - grp * per_group;
+    tm = first_m + r % rows;
+    tn = r / rows;
+    kb0 = split * s.kb_per_split;
+    kb1 = min(kb0 + s.kb_per_split, s.k_blocks);
+}
+
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, uint32_t site,
+                                          volatile int* abort) {
+    return __all_sync(0xffffffffu, mbar_wait(bar, parity, site, abort));
+}
+
+template <int BN, bool A_MN, bool B_MN, int OUT, bool F16>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
+                const __grid_constant__ CUtensorMap tmap_b, void* __restrict__ c_out,
+                const GemmShape shape) {
+    using C = GemmCfg<BN>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    GemmBarriers* bars = reinterpret_cast<GemmBarriers*>(smem + C::kOffBar);
+    volatile int* abort = &bars->abort;
+    const uint32_t warp = warp_id(), lane = lane_id();
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::kStages; ++s) {
+            mbar_init(&bars->full[s], 1);
+            mbar_init(&bars->empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&bars->acc_full[b], 1);
+            mbar_init(&bars->acc_empty[b], 4);
+        }
+        mbar_init(&bars->mma_final, 1);
+        bars->abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(&bars->tmem_base, C::kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = bars->tmem_base;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            tma_prefetch_desc(&tmap_a);
+            tma_prefetch_desc(&tmap_b);
+            int it = 0;  // k-blocks loaded so far (all units)
+            int last_use[6] = {-1, -1, -1, -1, -1, -1};
+            bool run = true;
+            for (int u = blockIdx.x; run && u < shape.units; u += gridDim.x) {
+                int tm, tn, kb0, kb1;
+                unit_of(shape, u, tm, tn, kb0, kb1);
+                for (int kb = kb0; kb < kb1; ++kb, ++it) {
+                    const int st = it % C::kStages, use = it / C::kStages;
+                    if (use > 0 &&
+                        !mbar_wait(&bars->empty[st], (use - 1) & 1, kGSiteEmpty, abort)) {
+                        run = false;
+                        break;
+                    }
+                    uint8_t* sa = smem + st * C::kStageBytes;
+                    uint8_t* sb = sa + C::kABytes;
+                    mbar_arrive_expect_tx(&bars->full[st], C::kStageBytes);
+                    if constexpr (A_MN) {
+                        for (int c = 0; c < kBM / 64; ++c)
+                            tma_load_2d(sa + c * C::kChunkBytes, &tmap_a, &bars->full[st],
+                                        tm * kBM + 64 * c, kb * kBK);
+                    } else {
+                        tma_load_2d(sa, &tmap_a, &bars->full[st], kb * kBK, tm * kBM);
+                    }
+                    if constexpr (B_MN) {
+                        for (int c = 0; c < BN / 64; ++c)
+                            tma_load_2d(sb + c * C::kChunkBytes, &tmap_b, &bars->full[st],
+                                        tn * BN + 64 * c, kb * kBK);
+                    } else {
+                        tma_load_2d(sb, &tmap_b, &bars->full[st], kb * kBK, tn * BN);
+                    }
+                    last_use[st] = use;
+                }
+            }
+            if (*abort)  // let copies already issued land before the CTA's memory goes
+                for (int s = 0; s < C::kStages; ++s)
+                    if (last_use[s] >= 0) mbar_wait_drain(&bars->full[s], last_use[s] & 1);
+        }
+    } else if (warp == 1) {
+        // --------------------------------------------------------- MMA issuer
+        constexpr uint32_t kIdesc = idesc_f16kind_f32(kBM, BN, A_MN, B_MN, F16);
+        int it = 0, n_unit = 0;
+        bool ok = true;
+        for (int u = blockIdx.x; ok && u < shape.units; u += gridDim.x, ++n_unit) {
+            int tm, tn, kb0, kb1;
+            unit_of(shape, u, tm, tn, kb0, kb1);
+            const int buf = n_unit & 1, use = n_unit >> 1;
+            // the accumulator must have been read out by the epilogue of two units ago
+            if (use > 0 &&
+                !warp_wait(&bars->acc_empty[buf], (use - 1) & 1, kGSiteAccEmpty, abort)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t tacc = tmem + buf * BN;
+            for (int kb = kb0; kb < kb1; ++kb, ++it) {
+                const int st = it % C::kStages;
+                if (!warp_wait(&bars->full[st], (it / C::kStages) & 1, kGSiteFull, abort)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t a_addr = smem_u32(smem + st * C::kStageBytes);
+                const uint32_t b_addr = a_addr + C::kABytes;
+#pragma unroll
+                for (int kk = 0; kk < kBK / 16; ++kk) {
+                    // K-major: 16 k-values = 32 bytes along the swizzled row;
+                    // MN-major: 16 k-rows = two 8-row groups of 1024 bytes
+                    const uint64_t ad = A_MN ? sdesc_sw128(a_addr + kk * 2048, C::kChunkBytes, 1024)
+                                             : sdesc_sw128(a_addr + kk * 32, 16, 1024);
+                    const uint64_t bd = B_MN ? sdesc_sw128(b_addr + kk * 2048, C::kChunkBytes, 1024)
+                                             : sdesc_sw128(b_addr + kk * 32, 16, 1024);
+                    mma_ss_warp(tacc, ad, bd, kIdesc, (kb > kb0 || kk > 0) ? 1u : 0u);
+                }
+                mma_commit_warp(&bars->empty[st]);
+            }
+            if (ok) mma_commit_warp(&bars->acc_full[buf]);
+        }
+        mma_commit_warp(&bars->mma_final);
+        mbar_wait_drain(&bars->mma_final, 0);
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const uint32_t quarter = warp & 3;
+        const uint32_t lane_off = (quarter * 32u) << 16;
+        int n_unit = 0;
+        for (int u = blockIdx.x; u < shape.units; u += gridDim.x, ++n_unit) {
+            int tm, tn, kb0, kb1;
+            unit_of(shape, u, tm, tn, kb0, kb1);
+            const int buf = n_unit & 1;
+            if (!warp_wait(&bars->acc_full[buf], (n_unit >> 1) & 1, kGSiteAccFull, abort)) break;
+            tc_fence_after();
+            const int row = tm * kBM + (int)(quarter * 32 + lane);
+#pragma unroll 1
+            for (int c = 0; c < BN / 32; ++c) {
+                uint32_t r[32];
+                tmem_ld32(tmem + lane_off + buf * BN + c * 32, r);
+                tmem_wait_ld();
+                if (c == BN / 32 - 1) {  // the accumulator has been read
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&bars->acc_empty[buf]);
+                }
+                const int col0 = tn * BN + c * 32;
+#pragma unroll
+                for (int gq = 0; gq < 4; ++gq) {  // groups of 8 columns (N % 8 == 0)
+                    const int col = col0 + 8 * gq;
+                    if (row >= shape.M || col >= shape.N) continue;
+                    const size_t off = (size_t)row * shape.N + col;
+                    if constexpr (OUT == kOut16) {
+                        *reinterpret_cast<uint4*>(static_cast<uint16_t*>(c_out) + off) =
+                            make_uint4(pack16x2<F16>(__uint_as_float(r[8 * gq]),
+                                                     __uint_as_float(r[8 * gq + 1])),
+                                       pack16x2<F16>(__uint_as_float(r[8 * gq + 2]),
+                                                     __uint_as_float(r[8 * gq + 3])),
+                                       pack16x2<F16>(__uint_as_float(r[8 * gq + 4]),
+                                                     __uint_as_float(r[8 * gq + 5])),
+                                       pack16x2<F16>(__uint_as_float(r[8 * gq + 6]),
+                                                     __uint_as_float(r[8 * gq + 7])));
+                    } else if constexpr (OUT == kOutF32) {
+                        float4* dst = reinterpret_cast<float4*>(static_cast<float*>(c_out) + off);
+                        dst[0] = make_float4(__uint_as_float(r[8 * gq]), __uint_as_float(r[8 * gq + 1]),
+                                             __uint_as_float(r[8 * gq + 2]), __uint_as_float(r[8 * gq + 3]));
+                        dst[1] = make_float4(__uint_as_float(r[8 * gq + 4]), __uint_as_float(r[8 * gq + 5]),
+                                             __uint_as_float(r[8 * gq + 6]), __uint_as_float(r[8 * gq + 7]));
+                    } else {
+                        float* dst = static_cast<float*>(c_out) + off;
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) atomicAdd(dst + e, __uint_as_float(r[8 * gq + e]));
+                    }
+                }
+            }
+        }
+    }
+
+    // ------------------------------------------------------------- teardown
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, C::kTmemCols);
+    }
+}
+
+template <int BN, bool A_MN, bool B_MN, int OUT, bool F16>
+cudaError_t launch_gemm_t(const CUtensorMap& ta, const CUtensorMap& tb, void* c,
+                          const GemmShape& s, cudaStream_t stream) {
+    using C = GemmCfg<BN>;
+    static std::atomic<unsigned long long> configured{0};
+    auto* kernel = gemm_kernel<BN, A_MN, B_MN, OUT, F16>;
+    cudaError_t e = set_max_dynamic_smem(kernel, C::kSmemBytes, configured);
+    if (e != cudaSuccess) return e;
+    const int grid = s.units < sm_count() ? s.units : sm_count();
+    kernel<<<grid, kGemmThreads, C::kSmemBytes, stream>>>(ta, tb, c, s);
+    return cudaGetLastError();
+}
+
+template <bool A_MN, bool B_MN>
+cudaError_t launch_gemm_layout(const CUtensorMap& ta, const CUtensorMap& tb, void* c,
+                               const GemmShape& s, int bn, int out, bool f16,
+                               cudaStream_t stream) {
+#define FORGE_GEMM_OUT(BN_, F16_)                                                               \
+    switch (out) {                                                                              \
+        case kOut16: return launch_gemm_t<BN_, A_MN, B_MN, kOut16, F16_>(ta, tb, c, s, stream);  \
+        case kOutF32: return launch_gemm_t<BN_, A_MN, B_MN, kOutF32, F16_>(ta, tb, c, s, stream);\
+        default: return launch_gemm_t<BN_, A_MN, B_MN, kOutF32Add, F16_>(ta, tb, c, s, stream); \
+    }
+    if (bn == 256) {
+        if (f16) { FORGE_GEMM_OUT(256, true) }
+        FORGE_GEMM_OUT(256, false)
+    }
+    if (f16) { FORGE_GEMM_OUT(128, true) }
+    FORGE_GEMM_OUT(128, false)
+#undef FORGE_GEMM_OUT
+}
+
+// Tile width: the one whose last wave of tiles is fuller (fewer idle SMs), 256 on a tie.
+int pick_bn(int M, int N) {
+    const int sms = sm_count();
+    auto waste = [&](int bn) {
+        const long long tiles = (long long)((M + kBM - 1) / kBM) * ((N + bn - 1) / bn);
+        const long long waves = (tiles + sms - 1) / sms;
+        // idle tile slots in units of 128 x 128 tiles
+        return (waves * sms - tiles) * (bn / 128);
+    };
+    return (N <= 128 || waste(128) < waste(256)) ? 128 : 256;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_dims(int tokens, int in_f, int out_f) {
+    if (tokens < 1 || in_f < 1 || out_f < 1) return FORGE_ATTN_ERR_INVALID_ARG;
+    if (tokens % 8 || in_f % 8 || out_f % 8) return FORGE_ATTN_ERR_UNSUPPORTED;
+    if ((long long)tokens * in_f >= (1ll << 31) || (long long)tokens * out_f >= (1ll << 31) ||
+        (long long)out_f * in_f >= (1ll << 31))
+        return FORGE_ATTN_ERR_UNSUPPORTED;
+    return FORGE_ATTN_OK;
+}
+
+GemmShape make_shape(int M, int N, int K, int BN, int splits) {
+    GemmShape s;
+    s.M = M;
+    s.N = N;
+    s.K = K;
+    s.tiles_m = (M + kBM - 1) / kBM;
+    s.tiles_n = (N + BN - 1) / BN;
+    s.k_blocks = (K + kBK - 1) / kBK;
+    if (splits < 1) splits = 1;
+    if (splits > s.k_blocks) splits = s.k_blocks;
+    s.kb_per_split = (s.k_blocks + splits - 1) / splits;
+    s.splits = (s.k_blocks + s.kb_per_split - 1) / s.kb_per_split;  // no empty split
+    s.units = s.splits * s.tiles_m * s.tiles_n;
+    return s;
+}
+
+int status_of(cudaError_t e) { return e == cudaSuccess ? FORGE_ATTN_OK : FORGE_ATTN_ERR_CUDA; }
+
+}  // namespace
+
+cudaError_t read_and_clear_device_error_gemm(unsigned int* value) {
+    return read_and_clear_unit_error(value);
+}
+
+}  // namespace forge
+
+using namespace forge;
+
+extern "C" {
+
+int forge_linear_fwd(const void* x, const void* w, void* y, int tokens, int in_features,
+                     int out_features, int flags, void* stream) {
+    if (!x || !w || !y) return FORGE_ATTN_ERR_INVALID_ARG;
+    int s = check_dims(tokens, in_features, out_features);
+    if (s != FORGE_ATTN_OK) return s;
+    if (flags & ~(FORGE_ATTN_OUT_F32 | FORGE_ATTN_FP16)) return FORGE_ATTN_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(w) || !aligned16(y)) return FORGE_ATTN_ERR_MISALIGNED;
+    const bool f16 = (flags & FORGE_ATTN_FP16) != 0;
+    const int bn = pick_bn(tokens, out_features);
+    CUtensorMap ta, tb;
+    if (encode_map_2d16(&ta, x, in_features, tokens, 64, kBM, f16) != cudaSuccess ||
+        encode_map_2d16(&tb, w, in_features, out_features, 64, bn, f16) != cudaSuccess)
+        return FORGE_ATTN_ERR_CUDA;
+    const GemmShape sh = make_shape(tokens, out_features, in_features, bn, 1);
+    return status_of(launch_gemm_layout<false, false>(
+        ta, tb, y, sh, bn, (flags & FORGE_ATTN_OUT_F32) ? kOutF32 : kOut16, f16,
+        static_cast<cudaStream_t>(stream)));
+}
+
+int forge_linear_bwd_dx(const void* dy, const void* w, void* dx, int tokens, int in_features,
+                        int out_features, int flags, void* stream) {
+    if (!dy || !w || !dx) return FORGE_ATTN_ERR_INVALID_ARG;
+    int s = check_dims(tokens, in_features, out_features);
+    if (s != FORGE_ATTN_OK) return s;
+    if (flags & ~(FORGE_ATTN_OUT_F32 | FORGE_ATTN_FP16)) return FORGE_ATTN_ERR_INVALID_ARG;
+    if (!aligned16(dy) || !aligned16(w) || !aligned16(dx)) return FORGE_ATTN_ERR_MISALIGNED;
+    const bool f16 = (flags & FORGE_ATTN_FP16) != 0;
+    const int bn = pick_bn(tokens, in_features);
+    CUtensorMap ta, tb;
+    // A = dY [tokens][out] (k = out contiguous); B = W [out = k][in = n], MN-major
+    if (encode_map_2d16(&ta, dy, out_features, tokens, 64, kBM, f16) != cudaSuccess ||
+        encode_map_2d16(&tb, w, in_features, out_features, 64, 64, f16) != cudaSuccess)
+        return FORGE_ATTN_ERR_CUDA;
+    const GemmShape sh = make_shape(tokens, in_features, out_features, bn, 1);
+    return status_of(launch_gemm_layout<false, true>(
+        ta, tb, dx, sh, bn, (flags & FORGE_ATTN_OUT_F32) ? kOutF32 : kOut16, f16,
+        static_cast<cudaStream_t>(stream)));
+}
+
+int forge_linear_split_k(int tokens, int in_features, int out_features) {
+    if (check_dims(tokens, in_features, out_features) != FORGE_ATTN_OK) return 0;
+    const int bn = pick_bn(out_features, in_features);
+    const long long tiles =
+        (long long)((out_features + kBM - 1) / kBM) * ((in_features + bn - 1) / bn);
+    const int k_blocks = (tokens + kBK - 1) / kBK;
+    const int sms = sm_count();
+    // enough (split, tile) units to fill every SM about twice, each split at least eight
+    // k-blocks (512 tokens) deep
+    long long splits = (2LL * sms + tiles - 1) / tiles;
+    const long long max_splits = k_blocks / 8 > 0 ? k_blocks / 8 : 1;
+    if (splits > max_splits) splits = max_splits;
+    return splits < 1 ? 1 : (int)splits;
+}
+
+int forge_linear_bwd_dw(const void* dy, const void* x, float* dw, int tokens, int in_features,
+                        int out_features, int split_k, int accumulate, int flags, void* stream) {
+    if (!dy || !x || !dw) return FORGE_ATTN_ERR_INVALID_ARG;
+    int s = check_dims(tokens, in_features, out_features);
+    if (s != FORGE_ATTN_OK) return s;
+    if (split_k < 0 || (accumulate != 0 && accumulate != 1)) return FORGE_ATTN_ERR_INVALID_ARG;
+    if (flags & ~FORGE_ATTN_FP16) return FORGE_ATTN_ERR_INVALID_ARG;
+    if (!aligned16(dy) || !aligned16(x) || !aligned16(dw)) return FORGE_ATTN_ERR_MISALIGNED;
+    const bool f16 = (flags & FORGE_ATTN_FP16) != 0;
+    const int bn = pick_bn(out_features, in_features);
+    if (split_k == 0) split_k = forge_linear_split_k(tokens, in_features, out_features);
+    const GemmShape sh = make_shape(out_features, in_features, tokens, bn, split_k);
+    CUtensorMap ta, tb;
+    // A = dY^T: dY [tokens = k][out = m], MN-major; B = X [tokens = k][in = n], MN-major
+    if (encode_map_2d16(&ta, dy, out_features, tokens, 64, 64, f16) != cudaSuccess ||
+        encode_map_2d16(&tb, x, in_features, tokens, 64, 64, f16) != cudaSuccess)
+        return FORGE_ATTN_ERR_CUDA;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    // one split overwriting dw stores; otherwise every split adds into dw, zeroed first
+    // unless accumulating
+    const bool add = accumulate || sh.splits > 1;
+    if (add && !accumulate) {
+        cudaError_t e =
+            cudaMemsetAsync(dw, 0, (size_t)out_features * in_features * sizeof(float), st);
+        if (e != cudaSuccess) return FORGE_ATTN_ERR_CUDA;
+    }
+    return status_of(launch_gemm_layout<true, true>(ta, tb, dw, sh, bn,
+                                                    add ? kOutF32Add : kOutF32, f16, st));
+}
+
+}  // extern "C"

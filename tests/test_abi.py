@@ -11,7 +11,7 @@ from causal_attention_fwd_attn_b200 import _lib, build
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADERS = [os.path.join(ROOT, "include", h)
-           for h in ("forge_attn.h", "forge_attn_testing.h", "forge_adamw.h")]
+           for h in ("forge_attn.h", "forge_attn_testing.h", "forge_adamw.h", "forge_linear.h")]
 
 
 @pytest.fixture(scope="module")
@@ -164,3 +164,18 @@ def test_adamw_rejects_bad_arguments(lib):
                                  **dict(common, beta2=1.0)) == _lib.ERR_INVALID_ARG
     assert _lib.forge_adamw_step([], step=1, workspace_bytes=ws_n, **common) == \
         _lib.ERR_INVALID_ARG
+
+
+def test_linear_rejects_bad_arguments(lib):
+    assert _lib.forge_linear_fwd(0, P, P, 64, 64, 64, 0, None) == _lib.ERR_INVALID_ARG
+    assert _lib.forge_linear_fwd(P, P, P, 64, 60, 64, 0, None) == _lib.ERR_UNSUPPORTED
+    assert _lib.forge_linear_fwd(P, P, P, 0, 64, 64, 0, None) == _lib.ERR_INVALID_ARG
+    assert _lib.forge_linear_fwd(P, P, P + 8, 64, 64, 64, 0, None) == _lib.ERR_MISALIGNED
+    assert _lib.forge_linear_fwd(P, P, P, 64, 64, 64, _lib.PRECISE, None) == _lib.ERR_INVALID_ARG
+    assert _lib.forge_linear_bwd_dx(P, P, P, 64, 64, 12, 0, None) == _lib.ERR_UNSUPPORTED
+    assert _lib.forge_linear_bwd_dw(P, P, P, 64, 64, 64, -1, 0, 0, None) == _lib.ERR_INVALID_ARG
+    assert _lib.forge_linear_bwd_dw(P, P, P, 64, 64, 64, 1, 2, 0, None) == _lib.ERR_INVALID_ARG
+    assert _lib.forge_linear_bwd_dw(P, P, P, 64, 64, 64, 1, 0, _lib.OUT_F32, None) == \
+        _lib.ERR_INVALID_ARG
+    assert _lib.forge_linear_split_k(8192, 768, 3072) >= 1
+    assert _lib.forge_linear_split_k(8, 8, 0) == 0

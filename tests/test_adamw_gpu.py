@@ -2,10 +2,11 @@
 on the same fp32 inputs (GPU).
 
 Tolerance: the step is a handful of fp32 operations per element, each rounded once
-(about 6e-8 relative), and the clip factor comes from an fp32 norm whose relative
-error is about 1e-6; so parameters and moments must agree with the fp64 oracle to a
-relative 1e-5 per element, with an absolute floor of 1e-9 (parameters) and 1e-12
-(moments) for values near zero; the global norm to 1e-5 relative.
+(2^-24 relative), and the clip factor comes from an fp32 norm whose relative error is
+about 1e-6.  A result can cancel far below its terms (m = beta1 m + (1 - beta1) g
+near zero), so the bound is relative to the element with an absolute floor relative
+to the tensor: per element |gpu - ref| <= 1e-5 |ref| + 1e-6 max|ref| (a few fp32
+ulps of the tensor's largest terms); the global norm to 1e-5 relative.
 """
 import numpy as np
 import pytest
@@ -50,10 +51,11 @@ def run_steps(shapes, seed, steps, max_norms):
         torch.cuda.synchronize()
         assert norm.item() == pytest.approx(ref_norm, rel=1e-5), f"step {step} norm"
         for i, t in enumerate(gpu):
-            for name, ref, atol in (("param", ref_p[i], 1e-9), ("exp_avg", ref_m[i], 1e-12),
-                                    ("exp_avg_sq", ref_v[i], 1e-12)):
+            for name, ref in (("param", ref_p[i]), ("exp_avg", ref_m[i]),
+                              ("exp_avg_sq", ref_v[i])):
                 got = t[name].double().cpu().numpy()
-                np.testing.assert_allclose(got, ref, rtol=1e-5, atol=atol,
+                np.testing.assert_allclose(got, ref, rtol=1e-5,
+                                           atol=1e-6 * float(np.max(np.abs(ref))),
                                            err_msg=f"step {step} tensor {i} {name}")
     return ref_norm
 

@@ -103,7 +103,7 @@ def test_fp16_operands(orc, d, T, causal):
 
 
 def test_fp16_operands_several_items_per_cta(orc):
-    w = wl.custom(4, 16, 1024, 64)
+    w = _multi(4, 16, 1024, 64)
     x = wl.make_inputs(0, w, seed_offset=77, dtype=torch.float16)
     whole_compare(orc, w, x, oracle_threads(w.T))
 
@@ -150,14 +150,21 @@ def test_full_workload_whole_tensors(orc, ci):
 # The persistent kernels walk several (head, tile) items per CTA with barrier phases
 # counted across items; these shapes have 3 or more items per CTA on 148 SMs, in
 # each head dimension and mode, compared over whole tensors.
+# V and dO have sigma 0.5 (as in the head-dim-128 workload) in the bf16-output cases:
+# with sigma 1 over 64 heads |dV| passes 4, where bf16 rounding of the output alone
+# takes up to 0.0156 of the 0.02 bound.
+def _multi(B, H, T, d, causal=1, sv=0.5):
+    return wl.Workload(f"b{B}h{H}t{T}d{d}c{causal}", B, H, T, d, 1.0, 1.0, sv, sv, causal)
+
+
 MULTI_ITEM = [
-    ("causal_d64", wl.custom(4, 16, 1024, 64), "default"),
-    ("causal_d128", wl.custom(4, 16, 1024, 128), "default"),
-    ("full_d64", wl.custom(4, 16, 1024, 64, causal=0), "default"),
-    ("full_d128", wl.custom(2, 16, 1024, 128, causal=0), "default"),
-    ("ragged_d64", wl.custom(2, 40, 1000, 64), "default"),
-    ("precise_d64", wl.custom(4, 16, 1024, 64), "accuracy"),
-    ("precise_d128", wl.custom(4, 16, 1024, 128), "accuracy"),
+    ("causal_d64", _multi(4, 16, 1024, 64), "default"),
+    ("causal_d128", _multi(4, 16, 1024, 128), "default"),
+    ("full_d64", _multi(4, 16, 1024, 64, causal=0), "default"),
+    ("full_d128", _multi(4, 16, 1024, 128, causal=0), "default"),
+    ("ragged_d64", _multi(2, 40, 1000, 64), "default"),
+    ("precise_d64", _multi(4, 16, 1024, 64, sv=1.0), "accuracy"),
+    ("precise_d128", _multi(4, 16, 1024, 128, sv=1.0), "accuracy"),
 ]
 
 
