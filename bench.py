@@ -1,8 +1,9 @@
 """Benchmark: causal attention forward + backward on B200, TFLOP/s and % of the
 dense BF16 tensor peak.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
-                    [--impl ours|reference] [--no-sub-results] [--no-cpu-baseline]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--mode MODE]
+                    [--impl ours|reference] [--sub-results all|attention|gemm|adamw|none]
+                    [--sub-seconds S] [--no-e2e] [--no-cpu-baseline]
 
 One step is one pass of the whole path over one batch of the workload: the forward
 (one kernel) and the backward (the D pre-pass, the dK/dV kernel with the dQ partials
@@ -62,7 +63,7 @@ SUB_RESULTS = [
     ("gpt2small_b8h12t1024d64", "default", 0),
     ("hd128_b2h16t4096d128", "default", 0),
 ]
-SUB_RESULT_SECONDS = 0.5
+SUB_RESULT_SECONDS = 0.5  # default; --sub-seconds
 
 
 def measured_peaks():
@@ -447,10 +448,10 @@ def sub_result(w, mode, causal, steps, world, max_ms, avg, clk, peaks):
     return r
 
 
-def run_sub_results(rank, world, dev, clocks, peaks, warmup):
-    """Each (workload, mode, causal) of SUB_RESULTS timed over at least
-    SUB_RESULT_SECONDS of GPU work (the step count is sized from the warm-up steps and
-    agreed over ranks)."""
+def run_sub_results(rank, world, dev, clocks, peaks, warmup, seconds):
+    """Each (workload, mode, causal) of SUB_RESULTS timed over at least `seconds` of GPU
+    work, 20 steps at least (the step count is sized from the warm-up steps and agreed
+    over ranks)."""
     out = []
     for name, mode, causal in SUB_RESULTS:
         ci, w = find_workload(name)
@@ -465,7 +466,7 @@ def run_sub_results(rank, world, dev, clocks, peaks, warmup):
         t1.record(p.stream)
         torch.cuda.synchronize()
         est_ms = max_over_ranks(t0.elapsed_time(t1) / 3, world, dev)
-        steps = max(20, min(20000, math.ceil(SUB_RESULT_SECONDS * 1e3 / est_ms)))
+        steps = max(20, min(20000, math.ceil(seconds * 1e3 / est_ms)))
         max_ms, avg, clk = timed_run(p, sets, 3, steps, world, dev, clocks)
         out.append(sub_result(w, mode, causal, steps, world, max_ms, avg, clk, peaks))
         del sets, p
@@ -475,7 +476,7 @@ def run_sub_results(rank, world, dev, clocks, peaks, warmup):
 
 # ------------------------------------------- the other hot-path kernels -------
 # The projection GEMMs around attention and the fused AdamW step, each timed over at
-# least SUB_RESULT_SECONDS with input sets rotating through more than the L2.
+# least --sub-seconds with input sets rotating through more than the L2.
 GEMM_SUB_RESULTS = [
     # (name, tokens, in_features, out_features, product)
     ("square4096_fwd", 4096, 4096, 4096, "fwd"),
@@ -489,8 +490,8 @@ def gemm_flops(tokens, din, dout):
     return 2.0 * tokens * din * dout
 
 
-def time_loop(fn, n_sets, world, dev, clocks, warmup=3):
-    """fn(i) launches step i; sizes the timed loop to SUB_RESULT_SECONDS from three
+def time_loop(fn, n_sets, world, dev, clocks, seconds, warmup=3):
+    """fn(i) launches step i; sizes the timed loop to `seconds` from three
     probe steps (agreed over ranks) and returns (steps, max-over-ranks ms, clock stats)."""
     stream = torch.cuda.current_stream(dev)
     for i in range(warmup):
@@ -502,7 +503,7 @@ def time_loop(fn, n_sets, world, dev, clocks, warmup=3):
     t1.record(stream)
     torch.cuda.synchronize()
     est = max_over_ranks(t0.elapsed_time(t1) / 3, world, dev)
-    steps = max(20, min(50000, math.ceil(SUB_RESULT_SECONDS * 1e3 / max(est, 1e-4))))
+    steps = max(20, min(50000, math.ceil(seconds * 1e3 / max(est, 1e-4))))
     barrier(world)
     torch.cuda.synchronize()
     lo = clocks.now()
@@ -516,7 +517,7 @@ def time_loop(fn, n_sets, world, dev, clocks, warmup=3):
     return steps, max_over_ranks(t0.elapsed_time(t1), world, dev), clocks.stats(lo, hi)
 
 
-def run_gemm_sub_results(rank, world, dev, clocks, peaks):
+def run_gemm_sub_results(rank, world, dev, clocks, peaks, seconds):
     from causal_attention_fwd_attn_b200 import _lib
 
     out = []
@@ -552,7 +553,7 @@ def run_gemm_sub_results(rank, world, dev, clocks, peaks):
                 _lib.check(_lib.forge_linear_bwd_dw(x["dy"].data_ptr(), x["x"].data_ptr(),
                                                     y.data_ptr(), tokens, din, dout, 0, 0, 0,
                                                     s), name)
-        steps, ms, clk = time_loop(fn, n_sets, world, dev, clocks)
+        steps, ms, clk = time_loop(fn, n_sets, world, dev, clocks, seconds)
         tf = job_tflops(gemm_flops(tokens, din, dout), steps, world, ms)
         out.append({"workload": name, "kind": "gemm", "tokens": tokens, "in": din, "out": dout,
                     "product": prod, "steps": steps, "ms_per_step": round(ms / steps, 4),
@@ -566,7 +567,7 @@ def run_gemm_sub_results(rank, world, dev, clocks, peaks):
     return out
 
 
-def run_adamw_sub_result(rank, world, dev, clocks, peaks):
+def run_adamw_sub_result(rank, world, dev, clocks, peaks, seconds):
     """One AdamW step over GPT-2-small-shaped parameters (148 tensors, 124.4M values):
     algorithmic bytes 32 per parameter (norm pass reads the gradient; the update reads
     parameter, gradient and both moments and writes parameter and both moments)."""
@@ -590,7 +591,7 @@ def run_adamw_sub_result(rank, world, dev, clocks, peaks):
         _lib.check(_lib.forge_adamw_step(table, 3e-4, 0.9, 0.95, 1e-8, 0.1, state["step"], 1.0,
                                          None, ws.data_ptr(), ws_n, s), "adamw")
 
-    steps, ms, clk = time_loop(fn, 1, world, dev, clocks)
+    steps, ms, clk = time_loop(fn, 1, world, dev, clocks, seconds)
     per_step = ms / steps
     gbs = 32.0 * n_params / (per_step * 1e-3) / 1e9
     res = {"workload": "adamw_gpt2small_124m", "kind": "adamw", "tensors": len(table),
@@ -621,12 +622,18 @@ def run_ours(args, rank, world, local_rank):
         del sets
         torch.cuda.empty_cache()
         # ---- end to end through the public C ABI with host buffers (pinned) ------
-        e2e = run_e2e(args, w, ci, mode, causal, dev, p, world)
+        e2e = None if args.no_e2e else run_e2e(args, w, ci, mode, causal, dev, p, world)
         subs = None
-        if not args.no_sub_results:
-            subs = run_sub_results(rank, world, dev, clocks, peaks, 3)
-            subs += run_gemm_sub_results(rank, world, dev, clocks, peaks)
-            subs.append(run_adamw_sub_result(rank, world, dev, clocks, peaks))
+        which = args.sub_results
+        if which != "none":
+            secs = args.sub_seconds
+            subs = []
+            if which in ("all", "attention"):
+                subs += run_sub_results(rank, world, dev, clocks, peaks, 3, secs)
+            if which in ("all", "gemm"):
+                subs += run_gemm_sub_results(rank, world, dev, clocks, peaks, secs)
+            if which in ("all", "adamw"):
+                subs.append(run_adamw_sub_result(rank, world, dev, clocks, peaks, secs))
     finally:
         clocks.stop()
     if rank != 0:
@@ -807,7 +814,13 @@ def main():
     ap.add_argument("--cpu-baseline-seconds", type=float, default=12.0,
                     help="budget of the oracle sample timed beside the GPU run (rank 0, N=1)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--no-sub-results", action="store_true")
+    ap.add_argument("--sub-results", choices=["all", "attention", "gemm", "adamw", "none"],
+                    default="all", help="which sub-results to time beside the headline")
+    ap.add_argument("--no-sub-results", action="store_true", help="same as --sub-results none")
+    ap.add_argument("--sub-seconds", type=float, default=SUB_RESULT_SECONDS,
+                    help="GPU time of each sub-result's timed loop (20 steps at least)")
+    ap.add_argument("--no-e2e", action="store_true",
+                    help="skip the end-to-end (host buffers) measurement")
     ap.add_argument("--reference-seconds", type=float, default=90.0,
                     help="--impl reference: about how long the timed steps take in all "
                          "(each step is at least one head pass)")
@@ -820,6 +833,8 @@ def main():
         raise SystemExit("--warmup must be at least 3")
     if args.steps < 1:
         raise SystemExit("--steps must be at least 1")
+    if args.no_sub_results:
+        args.sub_results = "none"
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

@@ -100,13 +100,23 @@ __global__ void __launch_bounds__(kAdamThreads) adamw_norm_kernel(
         const float* g = t.grad[i];
         const long long n4 = (e1 - e0) >> 2;
         const float4* g4 = reinterpret_cast<const float4*>(g + e0);
-        for (long long k = threadIdx.x; k < n4; k += blockDim.x) {
-            const float4 x = g4[k];
-            acc = fmaf(x.x, x.x, acc);
-            acc = fmaf(x.y, x.y, acc);
-            acc = fmaf(x.z, x.z, acc);
-            acc = fmaf(x.w, x.w, acc);
+        // four independent loads in flight per thread (the pass is bound by memory
+        // latency otherwise), then the remainder
+        const int bd = (int)blockDim.x;
+        long long k = threadIdx.x;
+        float a1 = 0.f, a2 = 0.f, a3 = 0.f;
+        for (; k + 3 * bd < n4; k += 4 * bd) {
+            const float4 x0 = g4[k], x1 = g4[k + bd], x2 = g4[k + 2 * bd], x3 = g4[k + 3 * bd];
+            acc = fmaf(x0.x, x0.x, fmaf(x0.y, x0.y, fmaf(x0.z, x0.z, fmaf(x0.w, x0.w, acc))));
+            a1 = fmaf(x1.x, x1.x, fmaf(x1.y, x1.y, fmaf(x1.z, x1.z, fmaf(x1.w, x1.w, a1))));
+            a2 = fmaf(x2.x, x2.x, fmaf(x2.y, x2.y, fmaf(x2.z, x2.z, fmaf(x2.w, x2.w, a2))));
+            a3 = fmaf(x3.x, x3.x, fmaf(x3.y, x3.y, fmaf(x3.z, x3.z, fmaf(x3.w, x3.w, a3))));
         }
+        for (; k < n4; k += bd) {
+            const float4 x = g4[k];
+            acc = fmaf(x.x, x.x, fmaf(x.y, x.y, fmaf(x.z, x.z, fmaf(x.w, x.w, acc))));
+        }
+        acc += (a1 + a2) + a3;
         for (long long e = e0 + 4 * n4 + threadIdx.x; e < e1; e += blockDim.x)
             acc = fmaf(g[e], g[e], acc);
     }

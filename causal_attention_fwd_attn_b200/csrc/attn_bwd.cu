@@ -283,6 +283,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = bars->tmem_base;
+    // the prologue above overlaps the previous kernel's tail (the pre-pass writes the
+    // row statistics and clears the accumulator); global memory is touched only now
+    grid_dependency_wait();
+    allow_dependents_launch();
 
     if (warp < kWarpCompute0) {
         // ---------------------------------------------------------- dQ drain
@@ -851,6 +855,8 @@ __global__ void __launch_bounds__(256) attn_bwd_preprocess_kernel(
     const void* __restrict__ o_in, const uint16_t* __restrict__ dO,
     const float* __restrict__ lse, float* __restrict__ rowstats, float* __restrict__ dq_accum,
     int T, int t_pad, long long padded_rows) {
+    grid_dependency_wait();
+    allow_dependents_launch();
     constexpr int kGroup = D / 8;  // threads per row
     const long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     const long long pr = t / kGroup;  // padded row index
@@ -907,6 +913,8 @@ template <bool F16>
 __global__ void __launch_bounds__(256) attn_bwd_dq_convert_kernel(const float* __restrict__ acc,
                                                                   uint16_t* __restrict__ dq,
                                                                   long long n8) {
+    grid_dependency_wait();
+    allow_dependents_launch();
     const long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     if (t >= n8) return;
     const float4 a = reinterpret_cast<const float4*>(acc)[2 * t];
@@ -932,34 +940,34 @@ cudaError_t launch_dkdv_dp(const CUtensorMap& tq, const CUtensorMap& tk, const C
     const int n_items = (int)items;
     // persistent: one CTA per SM (shared memory and tensor memory allow no more)
     const int grid = n_items < sm_count() ? n_items : sm_count();
-    attn_bwd_dkdv_kernel<D, PRECISE, F16><<<grid, kBwdThreads, C::kSmemBytes, stream>>>(
-        tq, tk, tv, tdo, tdq, rowstats, dq_accum, dk, dv, T, BH, n_kvtiles, n_items, scale,
-        scale * kLog2e, causal, grad_f32);
-    return cudaGetLastError();
+    return launch_dependent(attn_bwd_dkdv_kernel<D, PRECISE, F16>, dim3(grid), dim3(kBwdThreads),
+                            C::kSmemBytes, stream, tq, tk, tv, tdo, tdq, rowstats, dq_accum, dk,
+                            dv, T, BH, n_kvtiles, n_items, scale, scale * kLog2e, causal,
+                            grad_f32);
 }
 
 template <int D, bool O_F32, bool F16>
-void launch_pre(const void* o, const void* dO, const float* lse, float* rowstats,
+cudaError_t launch_pre(const void* o, const void* dO, const float* lse, float* rowstats,
                 float* dq_accum, int BH, int T, cudaStream_t stream) {
     const int t_pad = ((T + kTile - 1) / kTile) * kTile;
     const long long padded_rows = (long long)BH * t_pad;
     const int threads = 256;
     const long long total = padded_rows * (D / 8);
     const unsigned blocks = (unsigned)((total + threads - 1) / threads);
-    attn_bwd_preprocess_kernel<D, O_F32, F16><<<blocks, threads, 0, stream>>>(
-        o, static_cast<const uint16_t*>(dO), lse, rowstats, dq_accum, T, t_pad, padded_rows);
+    return launch_dependent(attn_bwd_preprocess_kernel<D, O_F32, F16>, dim3(blocks), dim3(threads),
+                     0, stream, o, static_cast<const uint16_t*>(dO), lse, rowstats, dq_accum, T,
+                     t_pad, padded_rows);
 }
 
 template <int D>
-void launch_pre_d(const void* o, const void* dO, const float* lse, float* rowstats,
-                  float* dq_accum, int BH, int T, int o_f32, int f16, cudaStream_t stream) {
+cudaError_t launch_pre_d(const void* o, const void* dO, const float* lse, float* rowstats,
+                         float* dq_accum, int BH, int T, int o_f32, int f16, cudaStream_t stream) {
     if (o_f32) {
-        if (f16) launch_pre<D, true, true>(o, dO, lse, rowstats, dq_accum, BH, T, stream);
-        else launch_pre<D, true, false>(o, dO, lse, rowstats, dq_accum, BH, T, stream);
-    } else {
-        if (f16) launch_pre<D, false, true>(o, dO, lse, rowstats, dq_accum, BH, T, stream);
-        else launch_pre<D, false, false>(o, dO, lse, rowstats, dq_accum, BH, T, stream);
+        if (f16) return launch_pre<D, true, true>(o, dO, lse, rowstats, dq_accum, BH, T, stream);
+        return launch_pre<D, true, false>(o, dO, lse, rowstats, dq_accum, BH, T, stream);
     }
+    if (f16) return launch_pre<D, false, true>(o, dO, lse, rowstats, dq_accum, BH, T, stream);
+    return launch_pre<D, false, false>(o, dO, lse, rowstats, dq_accum, BH, T, stream);
 }
 
 template <int D>
@@ -982,9 +990,8 @@ cudaError_t launch_dkdv_d(const CUtensorMap& tq, const CUtensorMap& tk, const CU
 cudaError_t launch_bwd_preprocess(const void* o, const void* dO, const float* lse,
                                   float* rowstats, float* dq_accum, int BH, int T, int d,
                                   int o_f32, int f16, cudaStream_t stream) {
-    if (d == 64) launch_pre_d<64>(o, dO, lse, rowstats, dq_accum, BH, T, o_f32, f16, stream);
-    else launch_pre_d<128>(o, dO, lse, rowstats, dq_accum, BH, T, o_f32, f16, stream);
-    return cudaGetLastError();
+    if (d == 64) return launch_pre_d<64>(o, dO, lse, rowstats, dq_accum, BH, T, o_f32, f16, stream);
+    return launch_pre_d<128>(o, dO, lse, rowstats, dq_accum, BH, T, o_f32, f16, stream);
 }
 
 cudaError_t launch_bwd_dkdv(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
@@ -1005,12 +1012,10 @@ cudaError_t launch_bwd_dq_convert(const float* dq_accum, void* dq, long long n, 
     const int threads = 256;
     const unsigned blocks = (unsigned)((n8 + threads - 1) / threads);
     if (f16)
-        attn_bwd_dq_convert_kernel<true><<<blocks, threads, 0, stream>>>(
-            dq_accum, static_cast<uint16_t*>(dq), n8);
-    else
-        attn_bwd_dq_convert_kernel<false><<<blocks, threads, 0, stream>>>(
-            dq_accum, static_cast<uint16_t*>(dq), n8);
-    return cudaGetLastError();
+        return launch_dependent(attn_bwd_dq_convert_kernel<true>, dim3(blocks), dim3(threads), 0,
+                                stream, dq_accum, static_cast<uint16_t*>(dq), n8);
+    return launch_dependent(attn_bwd_dq_convert_kernel<false>, dim3(blocks), dim3(threads), 0,
+                            stream, dq_accum, static_cast<uint16_t*>(dq), n8);
 }
 
 cudaError_t read_and_clear_device_error_bwd(unsigned int* value) {

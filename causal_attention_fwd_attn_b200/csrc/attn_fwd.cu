@@ -169,6 +169,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = bars->tmem_base;
+    // the prologue above overlaps the previous kernel's tail; inputs are read only now
+    grid_dependency_wait();
+    allow_dependents_launch();
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
@@ -536,10 +539,9 @@ cudaError_t launch_fwd_dp(const CUtensorMap& tq, const CUtensorMap& tk, const CU
     const int n_qtiles = (T + kTile - 1) / kTile;
     const int n_items = BH * n_qtiles;
     const int grid = n_items < sm_count() ? n_items : sm_count();
-    attn_fwd_kernel<D, PRECISE, F16><<<grid, kFwdThreads, C::kSmemBytes, stream>>>(
-        tq, tk, tv, o, lse, T, BH, n_qtiles, n_items, fabsf(scale) * kLog2e,
-        scale < 0.f ? 1 : 0, causal, o_f32);
-    return cudaGetLastError();
+    return launch_dependent(attn_fwd_kernel<D, PRECISE, F16>, dim3(grid), dim3(kFwdThreads),
+                            C::kSmemBytes, stream, tq, tk, tv, o, lse, T, BH, n_qtiles, n_items,
+                            fabsf(scale) * kLog2e, scale < 0.f ? 1 : 0, causal, o_f32);
 }
 
 template <int D>

@@ -31,6 +31,25 @@ cudaError_t set_max_dynamic_smem(Kernel* kernel, int bytes,
     return e;
 }
 
+// Launches `kernel` with programmatic stream serialisation: its CTAs may be scheduled
+// while the previous kernel in the stream runs its last CTAs, and they wait in
+// grid_dependency_wait() (sm100_ptx.cuh) until that kernel has completed.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                             cudaStream_t stream, Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args&&>(args)...);
+}
+
 // Number of SMs of the current device: the persistent kernels launch one CTA per SM.
 // Cached per device ordinal (devices 64 and up query on every call); concurrent
 // first calls may both query, which is harmless.

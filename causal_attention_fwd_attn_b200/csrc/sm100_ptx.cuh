@@ -58,6 +58,20 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 __device__ __forceinline__ uint32_t lane_id() { return threadIdx.x & 31; }
 __device__ __forceinline__ uint32_t warp_id() { return threadIdx.x >> 5; }
 
+// --------------------------------------------------- programmatic dependent launch --
+// A kernel launched with programmatic stream serialisation may start before the
+// kernel ahead of it in the stream has finished.  grid_dependency_wait() returns once
+// that kernel has completed and its memory writes are visible (immediately when the
+// launch had no such dependency); every thread calls it before touching global memory.
+// allow_dependents_launch() lets the next kernel of the stream be scheduled (it then
+// waits in its own grid_dependency_wait()).
+__device__ __forceinline__ void grid_dependency_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void allow_dependents_launch() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- mbarrier --
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
