@@ -256,9 +256,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         dst[1] = make_float4(__uint_as_float(r[8 * gq + 4]), __uint_as_float(r[8 * gq + 5]),
                                              __uint_as_float(r[8 * gq + 6]), __uint_as_float(r[8 * gq + 7]));
                     } else {
+                        // two 16-byte vector reductions (N % 8 == 0 keeps them aligned)
                         float* dst = static_cast<float*>(c_out) + off;
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) atomicAdd(dst + e, __uint_as_float(r[8 * gq + e]));
+                        red_add_v4(dst, __uint_as_float(r[8 * gq]), __uint_as_float(r[8 * gq + 1]),
+                                   __uint_as_float(r[8 * gq + 2]), __uint_as_float(r[8 * gq + 3]));
+                        red_add_v4(dst + 4, __uint_as_float(r[8 * gq + 4]),
+                                   __uint_as_float(r[8 * gq + 5]), __uint_as_float(r[8 * gq + 6]),
+                                   __uint_as_float(r[8 * gq + 7]));
                     }
                 }
             }

@@ -188,6 +188,14 @@ __device__ __forceinline__ void tma_reduce_add_3d(const void* map, const void* s
         : "memory");
 }
 
+// Four consecutive fp32 values added into global memory by one vector reduction (no
+// return value); addr 16-byte aligned.
+__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b),
+                 "f"(c), "f"(d)
+                 : "memory");
+}
+
 // 3-D tiled store shared -> global (rows outside the tensor are clipped by TMA).
 __device__ __forceinline__ void tma_store_3d(const void* map, const void* smem_src, int c0, int c1,
                                              int c2) {
