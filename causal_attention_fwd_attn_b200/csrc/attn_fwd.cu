@@ -16,18 +16,23 @@
 // heaviest first, zigzag over the CTAs, and every role walks the same item sequence,
 // so one item's epilogue and the next item's Q load overlap the neighbouring item's
 // products.
-//   warp 0      TMA producer: Q per item into one of two buffers (d = 64; one at
-//               d = 128), once the item that used the buffer before has finished its
-//               score products, then K/V tiles into an NS-stage ring.
-//   warp 1      MMA issuer (converged warp, one elected lane issues): S = Q K^T into
-//               TMEM, then O += P V with P read from TMEM (tcgen05.mma with A in
-//               tensor memory).  An item's first P V waits until the previous
-//               item's O has been read out.
+//   warp 0      TMA producer: Q per item into one of two shared-memory buffers
+//               (d = 64; one at d = 128), once the buffer's previous Q has been
+//               copied to tensor memory, then K/V tiles into an NS-stage ring.
+//   warp 1      MMA issuer (converged warp, one elected lane issues): copies the
+//               item's Q into tensor memory (tcgen05.cp), then S = Q K^T with Q read
+//               from tensor memory as the A operand and K from shared memory (so a
+//               score product reads one operand's bytes from shared memory, not
+//               two), and O += P V with P read from tensor memory.  An item's first
+//               P V waits until the previous item's O has been read out.
 //   warps 2..5  softmax: thread r owns query row r (TMEM lane r): loads its S row,
 //               masks, updates the running max/sum, writes P (bf16) back to TMEM,
 //               and in the epilogue normalises its O row and writes it and its LSE
-//               to global memory.
-// Tensor memory (512 columns): S0 [0,128) | S1 [128,256) | O [256, 256+d).  Key tile g
+//               to global memory.  From an item's third tile on, the tile's max is
+//               taken in the same pass as its exponentials (against the running max),
+//               and the tile is redone in the rare case that it moves the max.
+// Tensor memory (512 columns): S0 [0,128) | S1 [128,256) | O [256, 256+d) | Q0, Q1
+// [256+d, 256+2d) (d/2 columns each).  Key tile g
 // uses S buffer g & 1, and its P is written over that S (the softmax thread holds
 // its whole S row in registers by then): hi = bf16(p) in the buffer's first 64
 // columns and, in precise mode, where P enters P V as two bf16 terms, lo =
@@ -36,7 +41,10 @@
 // still on tile g, so the softmax never waits for a score product.  S(g+2) reuses
 // the buffer of P(g), so it is issued once P V(g) has completed (its commit).
 // The running max is rescaled lazily: O and the row sum are corrected only when
-// the max grows by more than 2^8 (all values stay finite and exact to rounding).
+// the max grows by more than 2^64 (2^15 with fp16 P); all values stay finite and
+// exact to rounding.
+#include <type_traits>
+
 #include "forge_internal.h"
 #include "sm100_ptx.cuh"
 
@@ -46,7 +54,12 @@ namespace {
 constexpr int kFwdThreads = 192;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
-constexpr float kRescaleThreshold = 8.0f;  // log2 units
+// The running max is moved (and O, the row sum rescaled) only when a tile raises it by
+// more than this many log2 units, so P <= 2^bound: 2^64 with bf16 P (P, O and the row
+// sum stay far inside the bf16 / fp32 range; the relative precision does not depend on
+// the magnitude), 2^15 with fp16 P (below the fp16 maximum, 65504).
+template <bool F16>
+constexpr float kRescaleThreshold = F16 ? 15.0f : 64.0f;
 
 // Which pairs of a row's exponentials go to the FMA-pipe polynomial (exp2_poly2)
 // instead of the MUFU unit.  None: every share tried (1/8 to 6/8) measured slower;
@@ -81,7 +94,11 @@ struct FwdCfg {
     // two S buffers; tile g uses buffer g & 1, and its P (bf16, 64 columns; the lo
     // half of precise mode in the next 64) is written over the S it came from
     static constexpr uint32_t kColS0 = 0, kColBuf = 128, kColPlo = 64, kColO = 256;
+    // Q of the item in tensor memory (bf16 pairs, d/2 columns), two buffers by item
+    // parity: the score product's A operand
+    static constexpr uint32_t kColQ = kColO + D;
     static constexpr uint32_t kTmemCols = 512;
+    static_assert(kColQ + 2 * (D / 2) <= kTmemCols, "tensor memory budget");
     // Q, K, V and P are all bf16, or all fp16 (F16)
     static constexpr uint32_t kIdescS = idesc_f16kind_f32(128, 128, false, false, F16);
     static constexpr uint32_t kIdescPV = idesc_f16kind_f32(128, D, false, true, F16);
@@ -260,14 +277,29 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                     c.n_tiles = c.valid ? tiles_of(qt_) : 0;
                 }
             };
-            // S(g) = Q K(g)^T into buffer g & 1, once P V(g-2) has read the P there
+            // S(g) = Q K(g)^T into buffer g & 1, once P V(g-2) has read the P there.  An
+            // item's first score product is preceded by the copy of its Q from shared
+            // into tensor memory (buffer item & 1), after which the shared-memory Q
+            // buffer goes back to the producer.  Tensor-memory buffer item & 1 was last
+            // read by the score products of item - 2, complete before P V(g-2) (each
+            // tile's P V waits for its softmax, which waits for its S).
             auto issue_s = [&](const Cursor& c) -> bool {
                 const int g = c.g;
                 const int st = g % C::kStages;
                 const int qb = c.item % C::kQBufs;
-                if (c.n == 0 &&
-                    !warp_wait(&bars->q_full[qb], (c.item / C::kQBufs) & 1, kSiteQ, abort))
-                    return false;
+                const uint32_t tQ = tmem + C::kColQ + (c.item & 1) * (D / 2);
+                if (c.n == 0) {
+                    if (!warp_wait(&bars->q_full[qb], (c.item / C::kQBufs) & 1, kSiteQ, abort))
+                        return false;
+                    tc_fence_after();
+                    const uint32_t q_addr = smem_u32(smem + C::kOffQ + qb * C::kTileBytes);
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t koff = (kk >> 2) * C::kChunkBytes + (kk & 3) * 32;
+                        tmem_cp_128x256b_warp(tQ + kk * 8, sdesc_sw128(q_addr + koff, 16, 1024));
+                    }
+                    mma_commit_warp(&bars->q_empty[qb]);
+                }
                 if (!warp_wait(&bars->k_full[st], (g / C::kStages) & 1, kSiteKFull, abort))
                     return false;
                 if (g >= 2 && !warp_wait(&bars->pv_done, (g - 2) & 1, kSiteSFree, abort))
@@ -275,17 +307,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 tc_fence_after();
                 const uint32_t tS = tmem + C::kColS0 + (g & 1) * C::kColBuf;
                 const uint32_t k_addr = smem_u32(smem + C::kOffK + st * C::kTileBytes);
-                const uint32_t q_addr = smem_u32(smem + C::kOffQ + qb * C::kTileBytes);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t koff = (kk >> 2) * C::kChunkBytes + (kk & 3) * 32;
-                    const uint64_t adesc = sdesc_sw128(q_addr + koff, 16, 1024);
                     const uint64_t bdesc = sdesc_sw128(k_addr + koff, 16, 1024);
-                    mma_ss_warp(tS, adesc, bdesc, idesc_s, kk > 0 ? 1u : 0u);
+                    mma_ts_warp(tS, tQ + kk * 8, bdesc, idesc_s, kk > 0 ? 1u : 0u);
                 }
                 mma_commit_warp(&bars->s_full[g & 1]);
-                // the item's last score product is the last reader of Q
-                if (c.n == c.n_tiles - 1) mma_commit_warp(&bars->q_empty[qb]);
                 return true;
             };
             // O += P(g) V(g).  An item's first P V overwrites O, so it waits until the
@@ -362,9 +390,6 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             for (int c = 0; c < kTile / 32; ++c) tmem_ld32(tS + c * 32, sraw + c * 32);
             tmem_wait_ld();
 
-            // Row max of the raw scores over the keys this row may see.  scale_log2 is
-            // >= 0 (a negative scale is applied by negating Q in the MMA), so the max
-            // of the scaled scores is scale_log2 times the raw max.
             const bool diag = causal && j == qt;
             const bool tail = !causal && (j + 1) * kTile > T;
             const bool masked_tile = diag || tail;
@@ -372,40 +397,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             float s[kTile];
 #pragma unroll
             for (int c = 0; c < kTile; ++c) s[c] = __uint_as_float(sraw[c]);
-            if (masked_tile) {  // the same for every thread of the CTA
-#pragma unroll
-                for (int c = 0; c < kTile; ++c)
-                    if (c > key_lim) s[c] = -INFINITY;
-            }
-            // eight independent chains of three-input max (16 values each), then 8 -> 1
-            float mx[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                mx[e] = fmaxf(s[16 * e], s[16 * e + 1]);
-#pragma unroll
-                for (int c = 2; c < 16; c += 2) mx[e] = fmax3(mx[e], s[16 * e + c], s[16 * e + c + 1]);
-            }
-            const float mt =
-                fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7])) *
-                scale_log2;
 
-            float alpha = 1.f;
-            bool need = false;
-            if (n == 0) {
-                m_run = mt;
-            } else if (mt > m_run + kRescaleThreshold) {
-                need = true;
-                alpha = ex2_approx(m_run - mt);
-                m_run = mt;
-                l_run *= alpha;
-            }
-            if (n > 0 && __any_sync(0xffffffffu, need)) {
-                // O must include P(n-1) V before it is rescaled
+            // O *= alpha (this thread's row), once O includes P(n-1) V
+            auto rescale_o = [&](float alpha) -> bool {
                 if (!__all_sync(0xffffffffu,
-                                mbar_wait(&bars->pv_done, (g - 1) & 1, kSitePV, abort))) {
-                    ok = false;
-                    break;
-                }
+                                mbar_wait(&bars->pv_done, (g - 1) & 1, kSitePV, abort)))
+                    return false;
                 tc_fence_after();
 #pragma unroll
                 for (int c = 0; c < D / 32; ++c) {
@@ -418,47 +415,118 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                     tmem_st32(tO + c * 32, r);
                 }
                 tmem_wait_st();
-            }
-
-            // P = exp2(s * scale_log2 - m), row sum, pack to bf16 pairs, store to TMEM
-            // P over the S it came from (this thread has all of its S row in registers)
-            const uint32_t tP = tS;
-            const uint32_t tPlo = tS + C::kColPlo;
-            const float neg_m = -m_run;
-            const float2 sl2 = make_float2(scale_log2, scale_log2);
-            const float2 nm2 = make_float2(neg_m, neg_m);
-            float2 ls[4];
+                return true;
+            };
+            // P = exp2(s * scale_log2 - m_run), its row sum, P packed to bf16 pairs
+            // and stored to TMEM over the S it came from (this thread has all of its S
+            // row in registers).  With kTrack the same pass also takes the row's raw
+            // max (eight independent three-input chains).
+            float2 lsum;
+            float mraw = -INFINITY;
+            auto exp_pass = [&](auto track) {
+                constexpr bool kTrack = decltype(track)::value;
+                const float2 sl2 = make_float2(scale_log2, scale_log2);
+                const float2 nm2 = make_float2(-m_run, -m_run);
+                float2 ls[4];
+                float mx[8];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) ls[e] = make_float2(0.f, 0.f);
+                for (int e = 0; e < 4; ++e) ls[e] = make_float2(0.f, 0.f);
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                uint32_t pk[32], pl[32];
+                for (int e = 0; e < 8; ++e) mx[e] = -INFINITY;
 #pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const int c = half * 64 + 2 * e;
-                    const float2 x = ffma2(make_float2(s[c], s[c + 1]), sl2, nm2);
-                    float2 p;
-                    if (!PRECISE && use_poly_pair(e)) {
-                        p = exp2_poly2(x);
-                    } else {
-                        p.x = ex2_approx(x.x);
-                        p.y = ex2_approx(x.y);
+                for (int qr = 0; qr < 4; ++qr) {  // 32 keys = 16 columns of P at a time
+                    uint32_t pk[16], pl[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const int c = qr * 32 + 2 * e;
+                        if (kTrack) mx[e & 7] = fmax3(mx[e & 7], s[c], s[c + 1]);
+                        const float2 x = ffma2(make_float2(s[c], s[c + 1]), sl2, nm2);
+                        float2 p;
+                        if (!PRECISE && use_poly_pair(e)) {
+                            p = exp2_poly2(x);
+                        } else {
+                            p.x = ex2_approx(x.x);
+                            p.y = ex2_approx(x.y);
+                        }
+                        if (masked_tile) {  // also covers scale 0, where -inf * 0 is NaN
+                            p.x = c > key_lim ? 0.f : p.x;
+                            p.y = c + 1 > key_lim ? 0.f : p.y;
+                        }
+                        ls[e & 3] = fadd2(ls[e & 3], p);
+                        pk[e] = pack16x2<F16>(p.x, p.y);
+                        if (PRECISE)
+                            pl[e] = pack_bf16x2(p.x - bf16_lo_to_float(pk[e]),
+                                                p.y - bf16_hi_to_float(pk[e]));
                     }
-                    if (masked_tile) {  // also covers scale 0, where -inf * 0 is NaN
-                        p.x = c > key_lim ? 0.f : p.x;
-                        p.y = c + 1 > key_lim ? 0.f : p.y;
-                    }
-                    ls[e & 3] = fadd2(ls[e & 3], p);
-                    pk[e] = pack16x2<F16>(p.x, p.y);
-                    if (PRECISE)
-                        pl[e] = pack_bf16x2(p.x - bf16_lo_to_float(pk[e]),
-                                            p.y - bf16_hi_to_float(pk[e]));
+                    tmem_st16(tS + qr * 16, pk);
+                    if (PRECISE) tmem_st16(tS + C::kColPlo + qr * 16, pl);
                 }
-                tmem_st32(tP + half * 32, pk);
-                if (PRECISE) tmem_st32(tPlo + half * 32, pl);
+                lsum = fadd2(fadd2(ls[0], ls[1]), fadd2(ls[2], ls[3]));
+                if (kTrack)
+                    mraw = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]),
+                                 fmaxf(mx[6], mx[7]));
+            };
+
+            // scale_log2 is >= 0 (a negative scale is applied by negating Q in the MMA),
+            // so the max of the scaled scores is scale_log2 times the raw max.
+            if (n > 1 && !masked_tile) {
+                // From an item's third tile on (its first is the only one with masked
+                // keys, and after two tiles the running max has seen at least 129 keys
+                // of the row) a tile is exponentiated against the running max straight
+                // away, taking the tile's max in the same pass: the max is off the
+                // critical path.  The result stands unless the tile raises some row's
+                // max by more than the lazy-rescale bound; then those rows move to the
+                // new max, O is rescaled, and the warp recomputes the tile.
+                exp_pass(std::true_type{});
+                const float mt = mraw * scale_log2;
+                const bool need = mt > m_run + kRescaleThreshold<F16>;
+                if (__any_sync(0xffffffffu, need)) {
+                    float alpha = 1.f;
+                    if (need) {
+                        alpha = ex2_approx(m_run - mt);
+                        m_run = mt;
+                        l_run *= alpha;
+                    }
+                    if (!rescale_o(alpha)) {
+                        ok = false;
+                        break;
+                    }
+                    exp_pass(std::false_type{});
+                }
+            } else {
+                // Row max of the raw scores over the keys this row may see, first.
+                if (masked_tile) {  // the same for every thread of the CTA
+#pragma unroll
+                    for (int c = 0; c < kTile; ++c)
+                        if (c > key_lim) s[c] = -INFINITY;
+                }
+                float mx[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    mx[e] = fmaxf(s[16 * e], s[16 * e + 1]);
+#pragma unroll
+                    for (int c = 2; c < 16; c += 2)
+                        mx[e] = fmax3(mx[e], s[16 * e + c], s[16 * e + c + 1]);
+                }
+                const float mt = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]),
+                                       fmaxf(mx[6], mx[7])) *
+                                 scale_log2;
+                float alpha = 1.f;
+                bool need = false;
+                if (n == 0) {
+                    m_run = mt;
+                } else if (mt > m_run + kRescaleThreshold<F16>) {
+                    need = true;
+                    alpha = ex2_approx(m_run - mt);
+                    m_run = mt;
+                    l_run *= alpha;
+                }
+                if (n > 0 && __any_sync(0xffffffffu, need) && !rescale_o(alpha)) {
+                    ok = false;
+                    break;
+                }
+                exp_pass(std::false_type{});
             }
-            const float2 ls01 = fadd2(ls[0], ls[1]), ls23 = fadd2(ls[2], ls[3]);
-            const float2 lsum = fadd2(ls01, ls23);
             l_run += lsum.x + lsum.y;
             tmem_wait_st();
             tc_fence_before();

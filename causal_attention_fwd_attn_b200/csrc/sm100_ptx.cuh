@@ -285,6 +285,18 @@ __device__ __forceinline__ void mma_ts_warp(uint32_t d_tmem, uint32_t a_tmem, ui
         "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
+// Copy of a 128-row x 256-bit (16 bf16 / fp16 per row) matrix from shared memory (a
+// matrix descriptor, as for an MMA operand) into tensor memory: row r to lane r, eight
+// consecutive 32-bit columns, the layout of an A operand read from tensor memory.  Warp-
+// collective like the MMAs; ordered with the MMAs this thread issues after it.
+__device__ __forceinline__ void tmem_cp_128x256b_warp(uint32_t taddr, uint64_t s_desc) {
+    asm volatile(
+        "{\n\t.reg .pred e;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "@e tcgen05.cp.cta_group::1.128x256b [%0], %1;\n\t}" ::"r"(taddr),
+        "l"(s_desc)
+        : "memory");
+}
 __device__ __forceinline__ void mma_commit_warp(uint64_t* bar) {
     asm volatile(
         "{\n\t.reg .pred e;\n\t"

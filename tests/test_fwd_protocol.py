@@ -2,8 +2,9 @@
 
 The forward (attn_fwd.cu) runs three roles per CTA over the CTA's item sequence: a
 TMA producer (Q per item into one of kQBufs buffers, K/V tiles into a ring), an MMA
-issuer (score products two key tiles ahead of the P V products, S buffer g & 1 for
-the CTA's g-th key tile) and the softmax warps (one row per thread, every key tile in
+issuer (the item's Q copied into tensor memory before its first score product, which
+frees the shared-memory Q buffer; score products two key tiles ahead of the P V
+products, S buffer g & 1 for the CTA's g-th key tile) and the softmax warps (one row per thread, every key tile in
 order, the item's epilogue at its end).  Every wait is an mbarrier parity wait, which
 is only sound if the waiter is never two phases ahead of the barrier (the parity of
 phase k + 2 equals that of phase k).  This test restates each role's sequence of
@@ -72,12 +73,11 @@ def simulate(items, d, causal, n_kv, rescale, item_relative_rescale=False):
             if kind == "s":
                 if n == 0:
                     yield f"q_full{qb}", item // q_bufs
+                    bars[f"q_empty{qb}"].arrive()    # Q copied to tensor memory
                 yield f"k_full{st}", g // stages
                 if g >= 2:
                     yield "pv_done", g - 2
                 bars[f"s_full{g & 1}"].arrive()
-                if n == tiles[item] - 1:
-                    bars[f"q_empty{qb}"].arrive()
             else:
                 yield f"p_full{g & 1}", g >> 1
                 yield f"v_full{st}", g // stages

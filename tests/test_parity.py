@@ -90,6 +90,46 @@ def test_precise_mode_sharp_softmax(orc, d):
                  o_dtype=torch.float32, grad_dtype=torch.float32, precise=True)
 
 
+def _growing_max_inputs(w, seed, factor, dtype=torch.bfloat16):
+    """Keys 0..127 scaled by `factor` (a power of two: exact): the key tile the forward
+    reaches last (causal: tile 0, after the diagonal; full attention: tile 0 again, the
+    kernel walks the key tiles from the last) raises most rows' running max past the
+    kernel's lazy-rescale bound (2^64 with bf16 P: factor 32; 2^15 with fp16 P: factor
+    8), so the exponentials it took against the earlier max are redone."""
+    x = wl.make_inputs(0, w, seed_offset=seed, dtype=dtype)
+    x["k"] = x["k"].clone()
+    x["k"][:, :, :128] *= factor
+    return x
+
+
+def _forward_compare(orc, w, x):
+    got = run_gpu(x, w.scale, w.causal, bwd=False)
+    f = as_f64(x)
+    o, lse = orc.fwd(f["q"], f["k"], f["v"], w.scale, w.causal, threads=4)
+    assert_close("o", got["o"], o, w.describe())
+    assert_close("lse", got["lse"], lse, w.describe())
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [1, 0])
+def test_running_max_grows_across_tiles(orc, d, causal):
+    w = wl.custom(1, 2, 700, d, causal=causal)
+    full_compare(orc, w, _growing_max_inputs(w, 19 + d + causal, 32), o_dtype=torch.float32,
+                 grad_dtype=torch.float32, precise=True)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_running_max_grows_across_tiles_default_mode_forward(orc, d):
+    w = wl.custom(2, 3, 600, d)
+    _forward_compare(orc, w, _growing_max_inputs(w, 23 + d, 32))
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_running_max_grows_across_tiles_fp16_forward(orc, d):
+    w = wl.custom(2, 3, 600, d)
+    _forward_compare(orc, w, _growing_max_inputs(w, 29 + d, 8, torch.float16))
+
+
 # ------------------------------------------------------------ fp16 operands --
 # The fp16-operand mode: q, k, v, dO in fp16, P and dS fp16 in the tensor-core
 # products, fp16 outputs; the oracle reads the exact values of the same fp16 inputs.
