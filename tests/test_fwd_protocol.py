@@ -30,21 +30,37 @@ class Bar:
             self.done += 1
 
 
-def simulate(items, d, causal, n_kv, rescale, item_relative_rescale=False):
+def simulate(items, d, causal, n_kv, rescale, item_relative_rescale=False, seed=None,
+             rescale_every=1, s_bufs=2):
     """items: query-tile index of each of the CTA's items.  Returns (finished, errors).
-    item_relative_rescale plants a plausible mistake for the sensitivity check: the
-    rescale wait names the P V phase by the tile's index within its item."""
+    With rescale, the softmax rescales O (waiting for the previous tile's P V) on every
+    rescale_every-th key tile of the CTA, past an item's first.
+
+    Tensor-core work is modelled as an in-order pipe: the MMA role issues products and
+    commits, and a separate pipe role completes them one at a time (a commit arrives
+    once every product issued before it has completed).  With seed None every role
+    runs as far as it can in a fixed order; with a seed the next role to take one step
+    (the pipe included) is drawn at random, which reaches schedules where the pipe
+    lags far behind the MMA issuer.  Planted mistakes for the sensitivity checks:
+    item_relative_rescale names the rescale's P V phase by the tile's index within its
+    item; s_bufs = 3 runs the score products three tiles ahead with the same single
+    P V-done barrier (the softmax's wait for P V(g-1) can then be two phases ahead)."""
+    import collections
+    import random
     q_bufs, stages = (2, 4) if d == 64 else (1, 3)
     bars = {}
     for b in range(2):
-        for name, count in (("q_full", 1), ("q_empty", 1), ("s_full", 1), ("p_full", 4)):
-            bars[f"{name}{b}"] = Bar(count)
+        for name in ("q_full", "q_empty"):
+            bars[f"{name}{b}"] = Bar(1)
+    for b in range(s_bufs):
+        bars[f"s_full{b}"], bars[f"p_full{b}"] = Bar(1), Bar(4)
     for s in range(stages):
         for name in ("k_full", "v_full", "kv_empty"):
             bars[f"{name}{s}"] = Bar(1)
     bars["pv_done"], bars["o_done"], bars["o_free"] = Bar(1), Bar(1), Bar(4)
     tiles = [qt + 1 if causal else n_kv for qt in items]
     seq = [(it, n) for it in range(len(items)) for n in range(tiles[it])]
+    pipe = collections.deque()   # commits in issue order
 
     def producer():
         g = 0
@@ -62,41 +78,41 @@ def simulate(items, d, causal, n_kv, rescale, item_relative_rescale=False):
                 g += 1
 
     def mma():
-        order = [("s", g) for g in range(min(2, len(seq)))]
+        order = [("s", g) for g in range(min(s_bufs, len(seq)))]
         for g in range(len(seq)):
             order.append(("pv", g))
-            if g + 2 < len(seq):
-                order.append(("s", g + 2))
+            if g + s_bufs < len(seq):
+                order.append(("s", g + s_bufs))
         for kind, g in order:
             item, n = seq[g]
-            st, qb = g % stages, item % q_bufs
+            st, qb, sb = g % stages, item % q_bufs, g % s_bufs
             if kind == "s":
                 if n == 0:
                     yield f"q_full{qb}", item // q_bufs
-                    bars[f"q_empty{qb}"].arrive()    # Q copied to tensor memory
+                    pipe.append(f"q_empty{qb}")    # Q copied to tensor memory
                 yield f"k_full{st}", g // stages
-                if g >= 2:
-                    yield "pv_done", g - 2
-                bars[f"s_full{g & 1}"].arrive()
+                if g >= s_bufs:
+                    yield "pv_done", g - s_bufs
+                pipe.append(f"s_full{sb}")
             else:
-                yield f"p_full{g & 1}", g >> 1
+                yield f"p_full{sb}", g // s_bufs
                 yield f"v_full{st}", g // stages
                 if n == 0 and item > 0:
                     yield "o_free", item - 1
-                bars["pv_done"].arrive()
-                bars[f"kv_empty{st}"].arrive()
+                pipe.append("pv_done")
+                pipe.append(f"kv_empty{st}")
                 if n == tiles[item] - 1:
-                    bars["o_done"].arrive()
+                    pipe.append("o_done")
 
     def softmax():
         g = 0
         for item in range(len(items)):
             for n in range(tiles[item]):
-                yield f"s_full{g & 1}", g >> 1
-                if rescale and n > 0:
+                yield f"s_full{g % s_bufs}", g // s_bufs
+                if rescale and n > 0 and g % rescale_every == 0:
                     yield "pv_done", (n - 1) if item_relative_rescale else g - 1
                 for _ in range(4):
-                    bars[f"p_full{g & 1}"].arrive()
+                    bars[f"p_full{g % s_bufs}"].arrive()
                 g += 1
             yield "o_done", item
             for _ in range(4):
@@ -106,25 +122,51 @@ def simulate(items, d, causal, n_kv, rescale, item_relative_rescale=False):
     waiting = [None] * len(roles)
     finished = [False] * len(roles)
     errors = []
-    progress = True
-    while progress:
-        progress = False
-        for i, role in enumerate(roles):
-            while not finished[i]:
-                if waiting[i] is not None:
-                    name, phase = waiting[i]
-                    b = bars[name]
-                    passes = (b.done & 1) != (phase & 1)   # what the hardware checks
-                    if passes != (b.done > phase) or b.done > phase + 1:
-                        errors.append((i, name, phase, b.done))
-                    if not passes:
-                        break
-                try:
-                    waiting[i] = next(role)
+
+    def ready(i):
+        """Checks role i's pending wait (recording a wrong pass); True if it may step."""
+        if finished[i]:
+            return False
+        if waiting[i] is None:
+            return True
+        name, phase = waiting[i]
+        b = bars[name]
+        passes = (b.done & 1) != (phase & 1)   # what the hardware checks
+        if passes != (b.done > phase) or b.done > phase + 1:
+            errors.append((i, name, phase, b.done))
+        return passes
+
+    def step(i):
+        try:
+            waiting[i] = next(roles[i])
+        except StopIteration:
+            finished[i] = True
+
+    if seed is None:
+        progress = True
+        while progress:
+            progress = False
+            while pipe:
+                bars[pipe.popleft()].arrive()
+                progress = True
+            for i in range(len(roles)):
+                while ready(i):
+                    step(i)
                     progress = True
-                except StopIteration:
-                    finished[i] = True
-    return all(finished), errors
+    else:
+        rng = random.Random(seed)
+        while True:
+            choices = [i for i in range(len(roles)) if ready(i)]
+            if pipe:
+                choices.append(-1)
+            if not choices:
+                break
+            i = rng.choice(choices)
+            if i < 0:
+                bars[pipe.popleft()].arrive()
+            else:
+                step(i)
+    return all(finished) and not pipe, errors
 
 
 def cta_items(b, n_ctas, n_items, BH, nq):
@@ -168,3 +210,35 @@ def test_model_catches_a_misnamed_phase():
     workload."""
     w = wl.WORKLOADS[1]
     assert run_all((w.B, w.H, w.T, w.d, 1), True, item_relative_rescale=True)
+
+
+RANDOM_SHAPES = [(1, 2, 1000, 64, 1), (1, 2, 1000, 128, 1), (1, 3, 700, 128, 0), (2, 3, 600, 64, 0)]
+
+
+@pytest.mark.parametrize("shape", RANDOM_SHAPES, ids=lambda s: "b{}h{}t{}d{}c{}".format(*s))
+def test_forward_protocol_under_random_schedules(shape):
+    """Random interleavings of the roles and of the tensor pipe's completions (the
+    pipe may lag the MMA issuer by many products), several CTAs' item sequences."""
+    B, H, T, d, causal = shape
+    BH, nq = B * H, -(-T // 128)
+    n_items = BH * nq
+    n_ctas = min(n_items, SMS)
+    for b in range(0, n_ctas, max(1, n_ctas // 4)):
+        items = cta_items(b, n_ctas, n_items, BH, nq)
+        for seed in range(12):
+            ok, errors = simulate(items, d, causal, nq, True, seed=seed,
+                                  rescale_every=1 + seed % 4)
+            assert ok and not errors, (b, seed, errors[:2])
+
+
+def test_random_schedules_catch_three_buffers_on_one_pv_barrier():
+    """Sensitivity: with the score products three tiles ahead (three S buffers) and the
+    same single P V-done barrier, the pipe can still be on P V(g-2) when the softmax of
+    tile g waits for P V(g-1); random schedules flag it, the kernel's two buffers not."""
+    bad = good = 0
+    for seed in range(40):
+        _, errors = simulate([7, 6, 5], 128, 1, 8, True, seed=seed, rescale_every=3, s_bufs=3)
+        bad += bool(errors)
+        ok, errors = simulate([7, 6, 5], 128, 1, 8, True, seed=seed, rescale_every=3)
+        good += ok and not errors
+    assert bad > 0 and good == 40
