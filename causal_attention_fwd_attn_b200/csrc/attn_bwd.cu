@@ -95,10 +95,15 @@ struct BwdCfg {
     // dQ_n leaves tensor memory through 128-byte-swizzled fp32 staging in shared
     // memory, 32-column slices at a time, and a TMA reduce-add.  Default mode: a
     // staging buffer of its own (two slices; two rounds per step at d = 128).
-    // Precise mode has no room for it and stages through the dS^T buffer, which
-    // dQ_n's products have finished reading once dQ_n is complete (the compute warps
-    // then wait for the drain before writing the next dS^T).
+    // Precise mode has no room for it.  At d = 128 it stages dQ_n in the shared
+    // memory of Q_n, dead once dK_n (issued before dQ_n) has read it: two rounds of
+    // two slices, both loaded from tensor memory before the first round's reduce is
+    // waited for, and Q_n's stage goes back to the producer (a second arrival on its
+    // empty barrier) once the reduces have read it.  At d = 64 it stages through the
+    // dS^T buffer, which dQ_n's products have finished reading once dQ_n is complete
+    // (the compute warps then wait for the drain before writing the next dS^T).
     static constexpr bool kStageOwn = !PRECISE;
+    static constexpr bool kStageInQ = PRECISE && D == 128;
     // P^T goes back into tensor memory (bf16 pairs) as the A operand of dV: into
     // columns of its own where 64 are left (d = 64 default), otherwise over the S^T
     // columns it was computed from (each 64-query half into the first 32 (hi) and
@@ -117,12 +122,12 @@ struct BwdCfg {
     static constexpr int kDQStageBytes = kTile * 32 * 4;  // one slice: [128 rows][32 fp32]
     static constexpr int kStageSlicesDS = kSplit * kScoreBytes / kDQStageBytes;
     static constexpr int kStageSlices =  // per round
-        kStageOwn ? 2 : (kStageSlicesDS < D / 32 ? kStageSlicesDS : D / 32);
+        (kStageOwn || kStageInQ) ? 2 : (kStageSlicesDS < D / 32 ? kStageSlicesDS : D / 32);
     static constexpr int kDrainRounds = (D / 32) / kStageSlices;
     static_assert(kDrainRounds * kStageSlices == D / 32, "dQ staging slices");
     // slices moved out of tensor memory per load group: the last group's load frees
     // the columns, before any wait for the staging
-    static constexpr int kLoadGroup = kStageOwn ? 2 : (kDrainRounds > 1 ? 2 : 1);
+    static constexpr int kLoadGroup = (kStageOwn || kStageInQ) ? 2 : 1;
     // K/V buffers.  One: the next item's K_j, V_j load after this item's last dQ,
     // and its first S^T waits for them.  (Two buffers at d = 64 measured slower, with
     // the next item's first S^T issued at the top of the item's last step, ahead of
@@ -151,9 +156,9 @@ struct BwdCfg {
         return kPAliasS ? kColS + (kk >> 2) * 64 + (kk & 3) * 8 : kColP + kk * 8;
     }
     // registers per thread after setmaxnreg (the launch gives 512 x 128): the precise
-    // d = 128 MMA issuer needs more, its drain (one slice at a time) less
-    static constexpr uint32_t kRegsDrain = (D == 128 && PRECISE) ? 80 : 96;
-    static constexpr uint32_t kRegsCompute = 168;
+    // d = 128 MMA issuer needs more, paid for by its compute warps
+    static constexpr uint32_t kRegsDrain = 96;
+    static constexpr uint32_t kRegsCompute = (D == 128 && PRECISE) ? 160 : 168;
     static constexpr uint32_t kRegsCtl = (D == 128 && PRECISE) ? 96 : 80;
     static_assert(128 * kRegsDrain + 256 * kRegsCompute + 128 * kRegsCtl <=
                       kBwdThreads * kLaunchRegs,
@@ -251,7 +256,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         mbar_init(&bars->acc_free, kDrainWarps);
         for (int s = 0; s < 3; ++s) {
             mbar_init(&bars->q_full[s], 1);
-            mbar_init(&bars->q_empty[s], 1);
+            mbar_init(&bars->q_empty[s], C::kStageInQ ? 2 : 1);
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(&bars->do_full[s], 1);
@@ -303,6 +308,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             if (!warp_wait(&bars->dq_full, g & 1, kSiteDQFull, abort)) { run = false; break; }
             tc_fence_after();
             bool fine = true;
+            // dQ staging: a buffer of its own, Q_i's stage, or the dS^T buffer
+            const int stage_off =
+                C::kStageInQ ? C::kOffQ + (g % C::kStagesQ) * C::kTileBytes : C::kOffStage;
             constexpr int kG = C::kLoadGroup;
             constexpr int kGroups = D / 32 / kG;
             constexpr int kGroupsPerRound = C::kStageSlices / kG;
@@ -335,7 +343,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 }
 #pragma unroll
                 for (int h = 0; h < kG; ++h) {
-                    uint8_t* stage = smem + C::kOffStage + (sl0 + h) * C::kDQStageBytes;
+                    uint8_t* stage = smem + stage_off + (sl0 + h) * C::kDQStageBytes;
 #pragma unroll
                     for (int ch = 0; ch < 8; ++ch)
                         *reinterpret_cast<float4*>(stage + sw128_offset(row, ch)) = make_float4(
@@ -357,7 +365,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
                             for (int sl = 0; sl < C::kStageSlices; ++sl)
                                 tma_reduce_add_3d(&tmap_dq,
-                                                  smem + C::kOffStage + sl * C::kDQStageBytes,
+                                                  smem + stage_off + sl * C::kDQStageBytes,
                                                   (rd * C::kStageSlices + sl) * 32, i * kTile, bh);
                             tma_store_commit();
                         }
@@ -367,11 +375,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             }
             if (!fine) { run = false; break; }
             if constexpr (!C::kStageOwn) {
-                // the dS^T buffer goes back to the compute warps once the reduces have
-                // read it
+                // the dS^T buffer goes back to the compute warps, or Q_i's stage to the
+                // producer, once the reduces have read it
                 if (leader) {
                     tma_store_wait_all_read();
-                    mbar_arrive(&bars->stage_done);
+                    mbar_arrive(C::kStageInQ ? &bars->q_empty[g % C::kStagesQ]
+                                             : &bars->stage_done);
                 }
             }
         }
@@ -531,7 +540,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             if (!warp_wait(&bars->dp_full, g & 1, kSiteDPFull, abort)) { ok = false; break; }
             // dS^T buffer: free once dK and dQ of the previous iteration have read it
             // and, where it stages dQ, once the drain is done with it
-            constexpr bool kStaged = !C::kStageOwn;
+            constexpr bool kStaged = !C::kStageOwn && !C::kStageInQ;
             if (g > 0 && !warp_wait(kStaged ? &bars->stage_done : &bars->ds_free, (g - 1) & 1,
                                     kStaged ? kSiteStageDone : kSiteDSFree, abort)) {
                 ok = false;
@@ -732,8 +741,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     const bool next_step = !last || have_next;  // a step g + 1 exists
                     const int kb1 = last ? nkb : kb;            // its K/V buffer
                     // with one K/V buffer the next item's K/V arrive only after this
-                    // item's last dQ has released them: its first S is issued after that
-                    const bool s_late = last && C::kKVBufs == 1;
+                    // item's last dQ has released them: its first S is issued after that.
+                    // With dQ staged in Q's shared memory every S_{g+1} goes after dK_g and
+                    // dQ_g: it may wait for Q_{g+1}, whose stage the reduces of dQ_{g-1}
+                    // release, and dK_g, dQ_g must not queue behind that wait.
+                    const bool s_late = C::kStageInQ || (last && C::kKVBufs == 1);
                     // S_{g+1}; a new item's first also waits for that item's K/V
                     auto issue_s = [&]() -> bool {
                         if (last && !warp_wait(&bars->kv_full[nkb], ((item + 1) / C::kKVBufs) & 1,
