@@ -129,9 +129,9 @@ struct BwdCfg {
     // the columns, before any wait for the staging
     static constexpr int kLoadGroup = (kStageOwn || kStageInQ) ? 2 : 1;
     // K/V buffers.  One: the next item's K_j, V_j load after this item's last dQ,
-    // and its first S^T waits for them.  (Two buffers at d = 64 measured slower, with
-    // the next item's first S^T issued at the top of the item's last step, ahead of
-    // that step's dV, dQ and dK; two buffers with that S^T kept late are untried.)
+    // and its first S^T waits for them.  (Two buffers at d = 64 measured slower, both
+    // with the next item's first S^T issued at the top of the item's last step, ahead
+    // of that step's dV, dQ and dK, and with it kept after them.)
     static constexpr int kKVBufs = 1;
     static constexpr int kOffK = 0;
     static constexpr int kOffV = kOffK + kKVBufs * kTileBytes;
