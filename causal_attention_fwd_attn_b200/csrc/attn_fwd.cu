@@ -11,8 +11,11 @@
 // diagonal-matrix trick for the rescale is not needed here: in tensor memory a
 // row of the accumulator is one lane, owned by one thread.
 //
-// Blackwell design (persistent CTAs, one per SM at most, 6 warps; used for every head
-// dimension and mode).  A work item is one (head, query tile); items are dealt
+// Blackwell design (persistent CTAs; used for every head dimension and mode).  At
+// d = 128 one CTA per SM with 6 warps and two S buffers.  At d = 64 two CTAs share an
+// SM, each with 8 warps (a control and a softmax warpgroup, registers moved to the
+// softmax by setmaxnreg), one S buffer and half of tensor memory: the two CTAs'
+// softmax warps overlap on every sub-partition.  A work item is one (head, query tile); items are dealt
 // heaviest first, zigzag over the CTAs, and every role walks the same item sequence,
 // so one item's epilogue and the next item's Q load overlap the neighbouring item's
 // products.
@@ -25,21 +28,25 @@
 //               score product reads one operand's bytes from shared memory, not
 //               two), and O += P V with P read from tensor memory.  An item's first
 //               P V waits until the previous item's O has been read out.
-//   warps 2..5  softmax: thread r owns query row r (TMEM lane r): loads its S row,
+//   warps 2, 3  (d = 64) idle: they complete the control warpgroup.
+//   warps 2..5 (d = 128), 4..7 (d = 64)
+//               softmax: thread r owns query row r (TMEM lane r): loads its S row,
 //               masks, updates the running max/sum, writes P (bf16) back to TMEM,
 //               and in the epilogue normalises its O row and writes it and its LSE
 //               to global memory.  From an item's third tile on, the tile's max is
 //               taken in the same pass as its exponentials (against the running max),
 //               and the tile is redone in the rare case that it moves the max.
-// Tensor memory (512 columns): S0 [0,128) | S1 [128,256) | O [256, 256+d) | Q0, Q1
-// [256+d, 256+2d) (d/2 columns each).  Key tile g
-// uses S buffer g & 1, and its P is written over that S (the softmax thread holds
+// Tensor memory: d = 128, 512 columns: S0 [0,128) | S1 [128,256) | O [256,384) | Q0, Q1
+// [384,512); d = 64, 256 columns per CTA: S0 [0,128) | O [128,192) | Q0, Q1 [192,256)
+// (Q: d/2 columns each).  Key tile g uses S buffer g % (number of buffers), and its P
+// is written over that S (the softmax thread holds
 // its whole S row in registers by then): hi = bf16(p) in the buffer's first 64
 // columns and, in precise mode, where P enters P V as two bf16 terms, lo =
 // bf16(p - hi) in the next 64.  The score products run two key tiles ahead of the
-// P V products (S0 S1 PV0 S2 PV1 S3 ...): S(g+1) is complete while the softmax is
-// still on tile g, so the softmax never waits for a score product.  S(g+2) reuses
-// the buffer of P(g), so it is issued once P V(g) has completed (its commit).
+// P V products with two buffers (S0 S1 PV0 S2 PV1 S3 ...): S(g+1) is complete while the
+// softmax is still on tile g.  S(g+2) reuses the buffer of P(g), so it is issued once
+// P V(g) has completed (its commit).  With one buffer (d = 64) S(g+1) follows P V(g)
+// and the SM's other CTA fills the gap.
 // The running max is rescaled lazily: O and the row sum are corrected only when
 // the max grows by more than 2^64 (2^15 with fp16 P); all values stay finite and
 // exact to rounding.
@@ -51,7 +58,6 @@
 namespace forge {
 namespace {
 
-constexpr int kFwdThreads = 192;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 // The running max is moved (and O, the row sum rescaled) only when a tile raises it by
@@ -75,10 +81,24 @@ enum : uint32_t {
 
 template <int D, bool F16>
 struct FwdCfg {
+    // d = 64: two CTAs share an SM, each with one S buffer and half of tensor memory,
+    // so each sub-partition runs two softmax warps (of different CTAs) whose latencies
+    // overlap.  Eight warps per CTA (two whole warpgroups, for the register split).
+    // d = 128: one CTA per SM with two S buffers, six warps.
+    static constexpr bool kTwoPerSM = D == 64;
+    static constexpr int kCtasPerSM = kTwoPerSM ? 2 : 1;
+    static constexpr int kThreads = kTwoPerSM ? 256 : 192;
+    static constexpr uint32_t kWarpSoftmax0 = kTwoPerSM ? 4 : 2;  // first softmax warp
+    static constexpr int kSBufs = kTwoPerSM ? 1 : 2;
+    // registers per thread after setmaxnreg (two CTAs of 256 threads leave 128 each at
+    // launch): the control warpgroup gives most of them to the softmax warpgroup
+    static constexpr uint32_t kRegsCtl = 48, kRegsSoftmax = 208;
+    static_assert(!kTwoPerSM || 128 * kRegsCtl + 128 * kRegsSoftmax <= 65536 / kCtasPerSM,
+                  "register split exceeds the block's launch allocation");
     static constexpr int kChunks = D / 64;               // 128-byte column chunks per row
     static constexpr int kChunkBytes = kTile * 128;      // 128 rows x 128 bytes
     static constexpr int kTileBytes = kChunks * kChunkBytes;
-    static constexpr int kStages = D == 64 ? 4 : 3;
+    static constexpr int kStages = D == 64 ? 2 : 3;
     // Q buffers: with two (d = 64), the next item's Q is loaded while this item runs,
     // so its first score product never waits for the load; d = 128 has room for one.
     static constexpr int kQBufs = D == 64 ? 2 : 1;
@@ -90,14 +110,17 @@ struct FwdCfg {
     // 1 KB of slack for aligning the dynamic shared memory base to 1024 bytes.
     static constexpr int kSmemBytes = kOffBar + kBarBytes + 1024;
     static_assert(kSmemBytes <= 232448, "shared memory budget");
+    static_assert(kSmemBytes * kCtasPerSM <= 233472 - 1024 * kCtasPerSM,
+                  "shared memory budget of the SM");
     // tensor memory columns
-    // two S buffers; tile g uses buffer g & 1, and its P (bf16, 64 columns; the lo
-    // half of precise mode in the next 64) is written over the S it came from
-    static constexpr uint32_t kColS0 = 0, kColBuf = 128, kColPlo = 64, kColO = 256;
+    // kSBufs S buffers; tile g uses buffer g % kSBufs, and its P (bf16, 64 columns;
+    // the lo half of precise mode in the next 64) is written over the S it came from
+    static constexpr uint32_t kColS0 = 0, kColBuf = 128, kColPlo = 64;
+    static constexpr uint32_t kColO = kSBufs * kColBuf;
     // Q of the item in tensor memory (bf16 pairs, d/2 columns), two buffers by item
     // parity: the score product's A operand
     static constexpr uint32_t kColQ = kColO + D;
-    static constexpr uint32_t kTmemCols = 512;
+    static constexpr uint32_t kTmemCols = kTwoPerSM ? 256 : 512;
     static_assert(kColQ + 2 * (D / 2) <= kTmemCols, "tensor memory budget");
     // Q, K, V and P are all bf16, or all fp16 (F16)
     static constexpr uint32_t kIdescS = idesc_f16kind_f32(128, 128, false, false, F16);
@@ -123,8 +146,21 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, uint32
     return __all_sync(0xffffffffu, mbar_wait(bar, parity, site, abort));
 }
 
+// Register split of the two-CTAs-per-SM configuration (every warp of a warpgroup
+// executes it in its own role's branch); a no-op otherwise.
+template <int D, bool F16, bool kSoftmax>
+__device__ __forceinline__ void fwd_set_regs() {
+    using C = FwdCfg<D, F16>;
+    if constexpr (C::kTwoPerSM) {
+        if constexpr (kSoftmax)
+            regs_inc<C::kRegsSoftmax>();
+        else
+            regs_dec<C::kRegsCtl>();
+    }
+}
+
 template <int D, bool PRECISE, bool F16>
-__global__ void __launch_bounds__(kFwdThreads, 1)
+__global__ void __launch_bounds__(FwdCfg<D, F16>::kThreads, FwdCfg<D, F16>::kCtasPerSM)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
                     const __grid_constant__ CUtensorMap tmap_k,
                     const __grid_constant__ CUtensorMap tmap_v,
@@ -192,6 +228,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
+        fwd_set_regs<D, F16, false>();
         if (lane == 0) {
             tma_prefetch_desc(&tmap_q);
             tma_prefetch_desc(&tmap_k);
@@ -247,6 +284,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     } else if (warp == 1) {
         // --------------------------------------------------------- MMA issuer
         // The whole warp runs this loop; one elected lane issues each MMA.
+        fwd_set_regs<D, F16, false>();
         {
             const uint32_t tO = tmem + C::kColO;
             // bit 13 of the instruction descriptor negates A: S = (-Q) K^T for scale < 0
@@ -302,10 +340,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 }
                 if (!warp_wait(&bars->k_full[st], (g / C::kStages) & 1, kSiteKFull, abort))
                     return false;
-                if (g >= 2 && !warp_wait(&bars->pv_done, (g - 2) & 1, kSiteSFree, abort))
+                if (g >= C::kSBufs &&
+                    !warp_wait(&bars->pv_done, (g - C::kSBufs) & 1, kSiteSFree, abort))
                     return false;
                 tc_fence_after();
-                const uint32_t tS = tmem + C::kColS0 + (g & 1) * C::kColBuf;
+                const uint32_t tS = tmem + C::kColS0 + (g % C::kSBufs) * C::kColBuf;
                 const uint32_t k_addr = smem_u32(smem + C::kOffK + st * C::kTileBytes);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
@@ -313,7 +352,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                     const uint64_t bdesc = sdesc_sw128(k_addr + koff, 16, 1024);
                     mma_ts_warp(tS, tQ + kk * 8, bdesc, idesc_s, kk > 0 ? 1u : 0u);
                 }
-                mma_commit_warp(&bars->s_full[g & 1]);
+                mma_commit_warp(&bars->s_full[g % C::kSBufs]);
                 return true;
             };
             // O += P(g) V(g).  An item's first P V overwrites O, so it waits until the
@@ -321,14 +360,16 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             auto issue_pv = [&](const Cursor& c) -> bool {
                 const int g = c.g;
                 const int st = g % C::kStages;
-                if (!warp_wait(&bars->p_full[g & 1], (g >> 1) & 1, kSitePFull, abort)) return false;
+                if (!warp_wait(&bars->p_full[g % C::kSBufs], (g / C::kSBufs) & 1, kSitePFull,
+                               abort))
+                    return false;
                 if (!warp_wait(&bars->v_full[st], (g / C::kStages) & 1, kSiteVFull, abort))
                     return false;
                 if (c.n == 0 && c.item > 0 &&
                     !warp_wait(&bars->o_free, (c.item - 1) & 1, kSiteOFree, abort))
                     return false;
                 tc_fence_after();
-                const uint32_t tP = tmem + C::kColS0 + (g & 1) * C::kColBuf;
+                const uint32_t tP = tmem + C::kColS0 + (g % C::kSBufs) * C::kColBuf;
                 const uint32_t v_addr = smem_u32(smem + C::kOffV + st * C::kTileBytes);
 #pragma unroll
                 for (int kk = 0; kk < kTile / 16; ++kk) {
@@ -346,7 +387,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             start(cs);
             start(cp);
             bool ok = true;
-            for (int i = 0; ok && i < 2 && cs.valid; ++i) {
+            for (int i = 0; ok && i < C::kSBufs && cs.valid; ++i) {
                 ok = issue_s(cs);
                 advance(cs);
             }
@@ -362,8 +403,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             mma_commit_warp(&bars->mma_final);
             mbar_wait_drain(&bars->mma_final, 0);
         }
+    } else if (warp < C::kWarpSoftmax0) {
+        fwd_set_regs<D, F16, false>();  // idle: completes the control warpgroup
     } else {
         // ------------------------------------------------------------ softmax
+        fwd_set_regs<D, F16, true>();
         const uint32_t row = ((warp & 3) << 5) + lane;  // TMEM lane owned by this thread
         const uint32_t lane_off = ((warp & 3) << 5) << 16;
         const uint32_t tO = tmem + lane_off + C::kColO;
@@ -378,9 +422,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         for (int n = 0; n < n_tiles; ++n) {
             const int g = g0 + n;
             const int j = causal ? qt - n : n_kvtiles_total - 1 - n;
-            const uint32_t tS = tmem + lane_off + C::kColS0 + (g & 1) * C::kColBuf;
-            if (!__all_sync(0xffffffffu,
-                            mbar_wait(&bars->s_full[g & 1], (g >> 1) & 1, kSiteSFull, abort))) {
+            const uint32_t tS = tmem + lane_off + C::kColS0 + (g % C::kSBufs) * C::kColBuf;
+            if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full[g % C::kSBufs],
+                                                   (g / C::kSBufs) & 1, kSiteSFull, abort))) {
                 ok = false;
                 break;
             }
@@ -531,7 +575,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bars->p_full[g & 1]);
+            if (lane == 0) mbar_arrive(&bars->p_full[g % C::kSBufs]);
         }
 
         if (!ok) break;
@@ -606,8 +650,9 @@ cudaError_t launch_fwd_dp(const CUtensorMap& tq, const CUtensorMap& tk, const CU
     if (e != cudaSuccess) return e;
     const int n_qtiles = (T + kTile - 1) / kTile;
     const int n_items = BH * n_qtiles;
-    const int grid = n_items < sm_count() ? n_items : sm_count();
-    return launch_dependent(attn_fwd_kernel<D, PRECISE, F16>, dim3(grid), dim3(kFwdThreads),
+    const int slots = sm_count() * C::kCtasPerSM;
+    const int grid = n_items < slots ? n_items : slots;
+    return launch_dependent(attn_fwd_kernel<D, PRECISE, F16>, dim3(grid), dim3(C::kThreads),
                             C::kSmemBytes, stream, tq, tk, tv, o, lse, T, BH, n_qtiles, n_items,
                             fabsf(scale) * kLog2e, scale < 0.f ? 1 : 0, causal, o_f32);
 }

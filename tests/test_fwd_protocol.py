@@ -3,8 +3,9 @@
 The forward (attn_fwd.cu) runs three roles per CTA over the CTA's item sequence: a
 TMA producer (Q per item into one of kQBufs buffers, K/V tiles into a ring), an MMA
 issuer (the item's Q copied into tensor memory before its first score product, which
-frees the shared-memory Q buffer; score products two key tiles ahead of the P V
-products, S buffer g & 1 for the CTA's g-th key tile) and the softmax warps (one row per thread, every key tile in
+frees the shared-memory Q buffer; score products one (d = 64, two CTAs per SM) or two
+(d = 128) key tiles ahead of the P V products, S buffer g mod the buffer count for the
+CTA's g-th key tile) and the softmax warps (one row per thread, every key tile in
 order, the item's epilogue at its end).  Every wait is an mbarrier parity wait, which
 is only sound if the waiter is never two phases ahead of the barrier (the parity of
 phase k + 2 equals that of phase k).  This test restates each role's sequence of
@@ -31,7 +32,7 @@ class Bar:
 
 
 def simulate(items, d, causal, n_kv, rescale, item_relative_rescale=False, seed=None,
-             rescale_every=1, s_bufs=2):
+             rescale_every=1, s_bufs=None):
     """items: query-tile index of each of the CTA's items.  Returns (finished, errors).
     With rescale, the softmax rescales O (waiting for the previous tile's P V) on every
     rescale_every-th key tile of the CTA, past an item's first.
@@ -47,7 +48,9 @@ def simulate(items, d, causal, n_kv, rescale, item_relative_rescale=False, seed=
     P V-done barrier (the softmax's wait for P V(g-1) can then be two phases ahead)."""
     import collections
     import random
-    q_bufs, stages = (2, 4) if d == 64 else (1, 3)
+    # d = 64: two CTAs per SM, each with one S buffer and a two-stage K/V ring
+    q_bufs, stages, s_bufs_kernel = (2, 2, 1) if d == 64 else (1, 3, 2)
+    s_bufs = s_bufs or s_bufs_kernel
     bars = {}
     for b in range(2):
         for name in ("q_full", "q_empty"):
