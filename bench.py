@@ -646,43 +646,76 @@ def run_ours(args, rank, world, local_rank):
 
 def run_e2e(args, w, ci, mode, causal, dev, p, world):
     """Same metric through the public C ABI (forge_attn_fwd_ex, forge_attn_bwd_ex), with
-    each step's inputs copied from pinned host memory and its outputs copied back,
-    all inside the timed region."""
+    each step's inputs copied from pinned host memory and all its outputs (O, LSE, dQ,
+    dK, dV) copied back, all inside the timed region.  The copies run on streams of
+    their own, as a caller would drive the API: step k+1's inputs go up and step
+    k-1's outputs come down while step k computes (two device buffer sets)."""
     L = p.lib
     B, H, T, d = w.B, w.H, w.T, w.d
     x = wl.make_inputs(ci, w, seed_offset=7)
     host_in = {n: t.pin_memory() for n, t in x.items()}
-    dev_in = {n: torch.empty_like(t, device=dev) for n, t in x.items()}
-    dev_out = {"o": p.o, "lse": p.lse, "dq": p.dq, "dk": p.dk, "dv": p.dv}
-    host_out = {n: torch.empty_like(t, device="cpu").pin_memory() for n, t in dev_out.items()}
+    dev_in = [{n: torch.empty_like(t, device=dev) for n, t in x.items()} for _ in range(2)]
+    out0 = {"o": p.o, "lse": p.lse, "dq": p.dq, "dk": p.dk, "dv": p.dv}
+    dev_out = [out0, {n: torch.empty_like(t) for n, t in out0.items()}]
+    host_out = {n: torch.empty_like(t, device="cpu").pin_memory() for n, t in out0.items()}
     h2d = sum(t.numel() * t.element_size() for t in host_in.values())
     d2h = sum(t.numel() * t.element_size() for t in host_out.values())
-    s = p.stream.cuda_stream
+    comp = p.stream
+    up = torch.cuda.Stream(device=dev)
+    down = torch.cuda.Stream(device=dev)
+    s = comp.cuda_stream
 
-    def step():
-        for n in host_in:
-            dev_in[n].copy_(host_in[n], non_blocking=True)
-        q, k, v, dO = dev_in["q"], dev_in["k"], dev_in["v"], dev_in["dO"]
-        L.check(L.forge_attn_fwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), p.o.data_ptr(),
-                                    p.lse.data_ptr(), B, H, T, d, w.scale, causal, p.fwd_flags,
-                                    s), "fwd")
-        L.check(L.forge_attn_bwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), p.o.data_ptr(),
-                                    dO.data_ptr(), p.lse.data_ptr(), p.dq.data_ptr(),
-                                    p.dk.data_ptr(), p.dv.data_ptr(), p.ws.data_ptr(), p.ws_n,
-                                    B, H, T, d, w.scale, causal, p.bwd_flags, s), "bwd")
-        for n in host_out:
-            host_out[n].copy_(dev_out[n], non_blocking=True)
+    def ev():
+        return torch.cuda.Event()
+
+    def run(steps, first_event=None):
+        """Issues `steps` pipelined steps; returns the event that completes the last
+        download (on the compute stream's timeline once waited for)."""
+        in_ready, comp_done, out_done = {}, {}, {}
+        if first_event is not None:
+            up.wait_event(first_event)
+            down.wait_event(first_event)
+        for k in range(steps):
+            b = k % 2
+            with torch.cuda.stream(up):
+                if k >= 2:
+                    up.wait_event(comp_done[k - 2])      # buffer set b's inputs are free
+                for n in host_in:
+                    dev_in[b][n].copy_(host_in[n], non_blocking=True)
+                in_ready[k] = ev()
+                in_ready[k].record(up)
+            comp.wait_event(in_ready[k])
+            if k >= 2:
+                comp.wait_event(out_done[k - 2])         # buffer set b's outputs are read
+            q, kk, v, dO = (dev_in[b][n] for n in ("q", "k", "v", "dO"))
+            o = dev_out[b]
+            L.check(L.forge_attn_fwd_ex(q.data_ptr(), kk.data_ptr(), v.data_ptr(),
+                                        o["o"].data_ptr(), o["lse"].data_ptr(), B, H, T, d,
+                                        w.scale, causal, p.fwd_flags, s), "fwd")
+            L.check(L.forge_attn_bwd_ex(q.data_ptr(), kk.data_ptr(), v.data_ptr(),
+                                        o["o"].data_ptr(), dO.data_ptr(), o["lse"].data_ptr(),
+                                        o["dq"].data_ptr(), o["dk"].data_ptr(),
+                                        o["dv"].data_ptr(), p.ws.data_ptr(), p.ws_n, B, H, T, d,
+                                        w.scale, causal, p.bwd_flags, s), "bwd")
+            comp_done[k] = ev()
+            comp_done[k].record(comp)
+            with torch.cuda.stream(down):
+                down.wait_event(comp_done[k])
+                for n in host_out:
+                    host_out[n].copy_(o[n], non_blocking=True)
+                out_done[k] = ev()
+                out_done[k].record(down)
+        comp.wait_event(out_done[steps - 1])
+        comp.wait_event(in_ready[steps - 1])
 
     steps = max(3, min(args.steps, 20))
-    for _ in range(2):
-        step()
+    run(2)
     torch.cuda.synchronize()
     barrier(world)
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    t0.record(p.stream)
-    for _ in range(steps):
-        step()
-    t1.record(p.stream)
+    t0.record(comp)
+    run(steps, first_event=t0)
+    t1.record(comp)
     torch.cuda.synchronize()
     p.check_device("in the end-to-end run")
     ms = max_over_ranks(t0.elapsed_time(t1), world, dev)
@@ -690,7 +723,9 @@ def run_e2e(args, w, ci, mode, causal, dev, p, world):
     value = job_tflops(fwd_flops + bwd_flops, steps, world, ms)
     return {"value": round(value, 2), "unit": UNIT, "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "steps": steps, "ms_per_step": round(ms / steps, 4),
-            "api": "forge_attn_fwd_ex + forge_attn_bwd_ex"}
+            "api": "forge_attn_fwd_ex + forge_attn_bwd_ex",
+            "copies": "own streams: step k+1's inputs up and step k-1's outputs down while "
+                      "step k computes (two device buffer sets)"}
 
 
 # ---------------------------------------------------------- CPU oracle leg ----
