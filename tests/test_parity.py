@@ -205,6 +205,7 @@ MULTI_ITEM = [
     ("ragged_d64", _multi(2, 40, 1000, 64), "default"),
     ("precise_d64", _multi(4, 16, 1024, 64, sv=1.0), "accuracy"),
     ("precise_d128", _multi(4, 16, 1024, 128, sv=1.0), "accuracy"),
+    ("precise_full_d64", _multi(4, 16, 1024, 64, causal=0, sv=1.0), "accuracy"),
     ("precise_full_d128", _multi(4, 16, 1024, 128, causal=0, sv=1.0), "accuracy"),
     ("precise_ragged_d128", _multi(2, 40, 1000, 128, sv=1.0), "accuracy"),
 ]
