@@ -311,29 +311,6 @@ cudaError_t launch_gemm_layout(const CUtensorMap& ta, const CUtensorMap& tb, voi
 #undef FORGE_GEMM_OUT
 }
 
-// Tile width: the one whose last wave of tiles is fuller (fewer idle SMs), 256 on a tie.
-int pick_bn(int M, int N) {
-    const int sms = sm_count();
-    auto waste = [&](int bn) {
-        const long long tiles = (long long)((M + kBM - 1) / kBM) * ((N + bn - 1) / bn);
-        const long long waves = (tiles + sms - 1) / sms;
-        // idle tile slots in units of 128 x 128 tiles
-        return (waves * sms - tiles) * (bn / 128);
-    };
-    return (N <= 128 || waste(128) < waste(256)) ? 128 : 256;
-}
-
-bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-
-int check_dims(int tokens, int in_f, int out_f) {
-    if (tokens < 1 || in_f < 1 || out_f < 1) return FORGE_ATTN_ERR_INVALID_ARG;
-    if (tokens % 8 || in_f % 8 || out_f % 8) return FORGE_ATTN_ERR_UNSUPPORTED;
-    if ((long long)tokens * in_f >= (1ll << 31) || (long long)tokens * out_f >= (1ll << 31) ||
-        (long long)out_f * in_f >= (1ll << 31))
-        return FORGE_ATTN_ERR_UNSUPPORTED;
-    return FORGE_ATTN_OK;
-}
-
 GemmShape make_shape(int M, int N, int K, int BN, int splits) {
     GemmShape s;
     s.M = M;
@@ -348,6 +325,46 @@ GemmShape make_shape(int M, int N, int K, int BN, int splits) {
     s.splits = (s.k_blocks + s.kb_per_split - 1) / s.kb_per_split;  // no empty split
     s.units = s.splits * s.tiles_m * s.tiles_n;
     return s;
+}
+
+// Split of a reduction of K over (split, tile) units when none is asked for: enough units
+// to give every SM about two, each split at least eight k-blocks (512) deep.
+int auto_splits(int M, int N, int K, int bn) {
+    const long long tiles = (long long)((M + kBM - 1) / kBM) * ((N + bn - 1) / bn);
+    const int k_blocks = (K + kBK - 1) / kBK;
+    long long splits = (2LL * sm_count() + tiles - 1) / tiles;
+    const long long max_splits = k_blocks / 8 > 0 ? k_blocks / 8 : 1;
+    if (splits > max_splits) splits = max_splits;
+    return splits < 1 ? 1 : (int)splits;
+}
+
+// Tile width.  A 128 x 256 tile does twice the work of a 128 x 128 one for 1.5 times
+// its operand bytes per k-block (A 16 KB + B 32 KB against 16 + 16 KB), and the
+// operand stream from L2 sets the pace of both, so a 256-wide k-block costs 1.5 of a
+// 128-wide one (1.4-1.55 measured on linear-layer shapes).  A width's cost is then the
+// k-blocks of the most loaded CTA (units are dealt round robin), weighted so: fewer,
+// wider tiles win unless they leave many more SMs idle.  256 on a tie.  splits = 0
+// takes auto_splits for each width.
+int pick_bn(int M, int N, int K, int splits) {
+    if (N <= 128) return 128;
+    const int sms = sm_count();
+    auto cost = [&](int bn) {
+        const int sp = splits > 0 ? splits : auto_splits(M, N, K, bn);
+        const GemmShape s = make_shape(M, N, K, bn, sp);
+        return (long long)((s.units + sms - 1) / sms) * s.kb_per_split * (bn == 256 ? 3 : 2);
+    };
+    return cost(256) <= cost(128) ? 256 : 128;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_dims(int tokens, int in_f, int out_f) {
+    if (tokens < 1 || in_f < 1 || out_f < 1) return FORGE_ATTN_ERR_INVALID_ARG;
+    if (tokens % 8 || in_f % 8 || out_f % 8) return FORGE_ATTN_ERR_UNSUPPORTED;
+    if ((long long)tokens * in_f >= (1ll << 31) || (long long)tokens * out_f >= (1ll << 31) ||
+        (long long)out_f * in_f >= (1ll << 31))
+        return FORGE_ATTN_ERR_UNSUPPORTED;
+    return FORGE_ATTN_OK;
 }
 
 int status_of(cudaError_t e) { return e == cudaSuccess ? FORGE_ATTN_OK : FORGE_ATTN_ERR_CUDA; }
@@ -372,7 +389,7 @@ int forge_linear_fwd(const void* x, const void* w, void* y, int tokens, int in_f
     if (flags & ~(FORGE_ATTN_OUT_F32 | FORGE_ATTN_FP16)) return FORGE_ATTN_ERR_INVALID_ARG;
     if (!aligned16(x) || !aligned16(w) || !aligned16(y)) return FORGE_ATTN_ERR_MISALIGNED;
     const bool f16 = (flags & FORGE_ATTN_FP16) != 0;
-    const int bn = pick_bn(tokens, out_features);
+    const int bn = pick_bn(tokens, out_features, in_features, 1);
     CUtensorMap ta, tb;
     if (encode_map_2d16(&ta, x, in_features, tokens, 64, kBM, f16) != cudaSuccess ||
         encode_map_2d16(&tb, w, in_features, out_features, 64, bn, f16) != cudaSuccess)
@@ -391,7 +408,7 @@ int forge_linear_bwd_dx(const void* dy, const void* w, void* dx, int tokens, int
     if (flags & ~(FORGE_ATTN_OUT_F32 | FORGE_ATTN_FP16)) return FORGE_ATTN_ERR_INVALID_ARG;
     if (!aligned16(dy) || !aligned16(w) || !aligned16(dx)) return FORGE_ATTN_ERR_MISALIGNED;
     const bool f16 = (flags & FORGE_ATTN_FP16) != 0;
-    const int bn = pick_bn(tokens, in_features);
+    const int bn = pick_bn(tokens, in_features, out_features, 1);
     CUtensorMap ta, tb;
     // A = dY [tokens][out] (k = out contiguous); B = W [out = k][in = n], MN-major
     if (encode_map_2d16(&ta, dy, out_features, tokens, 64, kBM, f16) != cudaSuccess ||
@@ -405,17 +422,8 @@ int forge_linear_bwd_dx(const void* dy, const void* w, void* dx, int tokens, int
 
 int forge_linear_split_k(int tokens, int in_features, int out_features) {
     if (check_dims(tokens, in_features, out_features) != FORGE_ATTN_OK) return 0;
-    const int bn = pick_bn(out_features, in_features);
-    const long long tiles =
-        (long long)((out_features + kBM - 1) / kBM) * ((in_features + bn - 1) / bn);
-    const int k_blocks = (tokens + kBK - 1) / kBK;
-    const int sms = sm_count();
-    // enough (split, tile) units to fill every SM about twice, each split at least eight
-    // k-blocks (512 tokens) deep
-    long long splits = (2LL * sms + tiles - 1) / tiles;
-    const long long max_splits = k_blocks / 8 > 0 ? k_blocks / 8 : 1;
-    if (splits > max_splits) splits = max_splits;
-    return splits < 1 ? 1 : (int)splits;
+    const int bn = pick_bn(out_features, in_features, tokens, 0);
+    return auto_splits(out_features, in_features, tokens, bn);
 }
 
 int forge_linear_bwd_dw(const void* dy, const void* x, float* dw, int tokens, int in_features,
@@ -427,8 +435,8 @@ int forge_linear_bwd_dw(const void* dy, const void* x, float* dw, int tokens, in
     if (flags & ~FORGE_ATTN_FP16) return FORGE_ATTN_ERR_INVALID_ARG;
     if (!aligned16(dy) || !aligned16(x) || !aligned16(dw)) return FORGE_ATTN_ERR_MISALIGNED;
     const bool f16 = (flags & FORGE_ATTN_FP16) != 0;
-    const int bn = pick_bn(out_features, in_features);
-    if (split_k == 0) split_k = forge_linear_split_k(tokens, in_features, out_features);
+    const int bn = pick_bn(out_features, in_features, tokens, split_k);
+    if (split_k == 0) split_k = auto_splits(out_features, in_features, tokens, bn);
     const GemmShape sh = make_shape(out_features, in_features, tokens, bn, split_k);
     CUtensorMap ta, tb;
     // A = dY^T: dY [tokens = k][out = m], MN-major; B = X [tokens = k][in = n], MN-major
