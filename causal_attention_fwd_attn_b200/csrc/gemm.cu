@@ -17,14 +17,17 @@
 // The transposes are descriptor choices (the operand-role exchange the paper uses for
 // its transposed attention products), never data movement.
 //
-// Design (persistent, one CTA per SM, 6 warps):
+// Design (persistent, one CTA per SM, 6 warps; tiles of BM x BN = 128 x 128, 128 x 256
+// or 256 x 256):
 //   warp 0      TMA producer: A and B k-blocks (64 deep) into a kStages ring.
 //   warp 1      MMA issuer (converged warp, one elected lane): 128 x BN x 16
-//               tcgen05 products into one of two tensor-memory accumulators, so one
-//               tile's epilogue overlaps the next tile's products.
-//   warps 2..5  epilogue: warp w reads TMEM lanes 32 (w % 4).. (its 32 rows of the
-//               tile), converts and stores them, or adds them (fp32 reductions) into C
-//               for split-K and accumulation.
+//               tcgen05 products, BM / 128 of them per 16-deep step sharing the B
+//               operand (one per 128-row half of the tile), into tensor memory: two
+//               accumulators when the tile fits twice (128-row tiles), so one tile's
+//               epilogue overlaps the next tile's products, else one (256 x 256).
+//   warps 2..5  epilogue: warp w reads TMEM lanes 32 (w % 4).. (its 32 rows of each
+//               128-row half), converts and stores them, or adds them (fp32
+//               reductions) into C for split-K and accumulation.
 // Work units are (split, tile) pairs walked by all CTAs in the same order; tiles are
 // grouped eight M-rows at a time so the CTAs live at once share operand panels in L2.
 #include "forge_internal.h"
@@ -42,17 +45,22 @@ constexpr int kGroupM = 8;
 enum : uint32_t { kGSiteFull = 1, kGSiteEmpty, kGSiteAccFull, kGSiteAccEmpty };
 enum OutMode : int { kOut16 = 0, kOutF32 = 1, kOutF32Add = 2 };
 
-template <int BN>
+template <int BM, int BN>
 struct GemmCfg {
-    static constexpr int kABytes = kBM * kBK * 2;  // 16 KB
-    static constexpr int kBBytes = BN * kBK * 2;   // 16 or 32 KB
+    static constexpr int kHalves = BM / kBM;          // 128-row halves of a tile
+    static constexpr int kHalfBytes = kBM * kBK * 2;  // 16 KB of A per half
+    static constexpr int kABytes = kHalves * kHalfBytes;
+    static constexpr int kBBytes = BN * kBK * 2;      // 16 or 32 KB
     static constexpr int kStageBytes = kABytes + kBBytes;
-    static constexpr int kStages = BN == 256 ? 4 : 6;
+    static constexpr int kStages = kStageBytes >= 65536 ? 3 : (kStageBytes >= 49152 ? 4 : 6);
     static constexpr int kChunkBytes = kBK * 128;  // one 64-element MN chunk of a k-block
     static constexpr int kOffBar = kStages * kStageBytes;
     static constexpr int kSmemBytes = kOffBar + 256 + 1024;
     static_assert(kSmemBytes <= 232448, "shared memory budget");
-    static constexpr uint32_t kTmemCols = 2 * BN;  // two accumulators
+    static constexpr int kAccCols = kHalves * BN;  // one accumulator
+    static constexpr int kAccBufs = 2 * kAccCols <= 512 ? 2 : 1;
+    static constexpr uint32_t kTmemCols = kAccBufs * kAccCols;
+    static_assert(kTmemCols <= 512 && kStages <= 6, "tensor memory / barrier budget");
 };
 
 struct GemmBarriers {
@@ -92,12 +100,12 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, uint32
     return __all_sync(0xffffffffu, mbar_wait(bar, parity, site, abort));
 }
 
-template <int BN, bool A_MN, bool B_MN, int OUT, bool F16>
+template <int BM, int BN, bool A_MN, bool B_MN, int OUT, bool F16>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                 const __grid_constant__ CUtensorMap tmap_b, void* __restrict__ c_out,
                 const GemmShape shape) {
-    using C = GemmCfg<BN>;
+    using C = GemmCfg<BM, BN>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -149,11 +157,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     uint8_t* sb = sa + C::kABytes;
                     mbar_arrive_expect_tx(&bars->full[st], C::kStageBytes);
                     if constexpr (A_MN) {
-                        for (int c = 0; c < kBM / 64; ++c)
+                        for (int c = 0; c < BM / 64; ++c)
                             tma_load_2d(sa + c * C::kChunkBytes, &tmap_a, &bars->full[st],
-                                        tm * kBM + 64 * c, kb * kBK);
+                                        tm * BM + 64 * c, kb * kBK);
                     } else {
-                        tma_load_2d(sa, &tmap_a, &bars->full[st], kb * kBK, tm * kBM);
+                        for (int h = 0; h < C::kHalves; ++h)
+                            tma_load_2d(sa + h * C::kHalfBytes, &tmap_a, &bars->full[st],
+                                        kb * kBK, tm * BM + kBM * h);
                     }
                     if constexpr (B_MN) {
                         for (int c = 0; c < BN / 64; ++c)
@@ -177,15 +187,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         for (int u = blockIdx.x; ok && u < shape.units; u += gridDim.x, ++n_unit) {
             int tm, tn, kb0, kb1;
             unit_of(shape, u, tm, tn, kb0, kb1);
-            const int buf = n_unit & 1, use = n_unit >> 1;
-            // the accumulator must have been read out by the epilogue of two units ago
+            const int buf = C::kAccBufs == 2 ? n_unit & 1 : 0;
+            const int use = C::kAccBufs == 2 ? n_unit >> 1 : n_unit;
+            // the accumulator must have been read out by the epilogue of the unit that
+            // used it last (two units ago, or the previous one with a single accumulator)
             if (use > 0 &&
                 !warp_wait(&bars->acc_empty[buf], (use - 1) & 1, kGSiteAccEmpty, abort)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
-            const uint32_t tacc = tmem + buf * BN;
+            const uint32_t tacc = tmem + buf * C::kAccCols;
             for (int kb = kb0; kb < kb1; ++kb, ++it) {
                 const int st = it % C::kStages;
                 if (!warp_wait(&bars->full[st], (it / C::kStages) & 1, kGSiteFull, abort)) {
@@ -199,11 +211,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 for (int kk = 0; kk < kBK / 16; ++kk) {
                     // K-major: 16 k-values = 32 bytes along the swizzled row;
                     // MN-major: 16 k-rows = two 8-row groups of 1024 bytes
-                    const uint64_t ad = A_MN ? sdesc_sw128(a_addr + kk * 2048, C::kChunkBytes, 1024)
-                                             : sdesc_sw128(a_addr + kk * 32, 16, 1024);
                     const uint64_t bd = B_MN ? sdesc_sw128(b_addr + kk * 2048, C::kChunkBytes, 1024)
                                              : sdesc_sw128(b_addr + kk * 32, 16, 1024);
-                    mma_ss_warp(tacc, ad, bd, kIdesc, (kb > kb0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+                    for (int h = 0; h < C::kHalves; ++h) {
+                        const uint32_t ah = a_addr + h * C::kHalfBytes;
+                        const uint64_t ad = A_MN ? sdesc_sw128(ah + kk * 2048, C::kChunkBytes, 1024)
+                                                 : sdesc_sw128(ah + kk * 32, 16, 1024);
+                        mma_ss_warp(tacc + h * BN, ad, bd, kIdesc, (kb > kb0 || kk > 0) ? 1u : 0u);
+                    }
                 }
                 mma_commit_warp(&bars->empty[st]);
             }
@@ -219,50 +235,61 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         for (int u = blockIdx.x; u < shape.units; u += gridDim.x, ++n_unit) {
             int tm, tn, kb0, kb1;
             unit_of(shape, u, tm, tn, kb0, kb1);
-            const int buf = n_unit & 1;
-            if (!warp_wait(&bars->acc_full[buf], (n_unit >> 1) & 1, kGSiteAccFull, abort)) break;
+            const int buf = C::kAccBufs == 2 ? n_unit & 1 : 0;
+            const int use = C::kAccBufs == 2 ? n_unit >> 1 : n_unit;
+            if (!warp_wait(&bars->acc_full[buf], use & 1, kGSiteAccFull, abort)) break;
             tc_fence_after();
-            const int row = tm * kBM + (int)(quarter * 32 + lane);
+            // 32-column chunks of the accumulator, four loads in flight per wait
+            constexpr int kChunks = C::kHalves * (BN / 32), kG = 4;
+            static_assert(kChunks % kG == 0, "epilogue load groups");
 #pragma unroll 1
-            for (int c = 0; c < BN / 32; ++c) {
-                uint32_t r[32];
-                tmem_ld32(tmem + lane_off + buf * BN + c * 32, r);
+            for (int g = 0; g < kChunks / kG; ++g) {
+                uint32_t r[32 * kG];
+#pragma unroll
+                for (int j = 0; j < kG; ++j) {
+                    const int hc = g * kG + j, h = hc / (BN / 32), c = hc % (BN / 32);
+                    tmem_ld32(tmem + lane_off + buf * C::kAccCols + h * BN + c * 32, r + 32 * j);
+                }
                 tmem_wait_ld();
-                if (c == BN / 32 - 1) {  // the accumulator has been read
+                if (g == kChunks / kG - 1) {  // the accumulator has been read
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&bars->acc_empty[buf]);
                 }
-                const int col0 = tn * BN + c * 32;
 #pragma unroll
-                for (int gq = 0; gq < 4; ++gq) {  // groups of 8 columns (N % 8 == 0)
-                    const int col = col0 + 8 * gq;
-                    if (row >= shape.M || col >= shape.N) continue;
-                    const size_t off = (size_t)row * shape.N + col;
-                    if constexpr (OUT == kOut16) {
-                        *reinterpret_cast<uint4*>(static_cast<uint16_t*>(c_out) + off) =
-                            make_uint4(pack16x2<F16>(__uint_as_float(r[8 * gq]),
-                                                     __uint_as_float(r[8 * gq + 1])),
-                                       pack16x2<F16>(__uint_as_float(r[8 * gq + 2]),
-                                                     __uint_as_float(r[8 * gq + 3])),
-                                       pack16x2<F16>(__uint_as_float(r[8 * gq + 4]),
-                                                     __uint_as_float(r[8 * gq + 5])),
-                                       pack16x2<F16>(__uint_as_float(r[8 * gq + 6]),
-                                                     __uint_as_float(r[8 * gq + 7])));
-                    } else if constexpr (OUT == kOutF32) {
-                        float4* dst = reinterpret_cast<float4*>(static_cast<float*>(c_out) + off);
-                        dst[0] = make_float4(__uint_as_float(r[8 * gq]), __uint_as_float(r[8 * gq + 1]),
-                                             __uint_as_float(r[8 * gq + 2]), __uint_as_float(r[8 * gq + 3]));
-                        dst[1] = make_float4(__uint_as_float(r[8 * gq + 4]), __uint_as_float(r[8 * gq + 5]),
-                                             __uint_as_float(r[8 * gq + 6]), __uint_as_float(r[8 * gq + 7]));
-                    } else {
-                        // two 16-byte vector reductions (N % 8 == 0 keeps them aligned)
-                        float* dst = static_cast<float*>(c_out) + off;
-                        red_add_v4(dst, __uint_as_float(r[8 * gq]), __uint_as_float(r[8 * gq + 1]),
-                                   __uint_as_float(r[8 * gq + 2]), __uint_as_float(r[8 * gq + 3]));
-                        red_add_v4(dst + 4, __uint_as_float(r[8 * gq + 4]),
-                                   __uint_as_float(r[8 * gq + 5]), __uint_as_float(r[8 * gq + 6]),
-                                   __uint_as_float(r[8 * gq + 7]));
+                for (int j = 0; j < kG; ++j) {
+                    const int hc = g * kG + j, h = hc / (BN / 32), c = hc % (BN / 32);
+                    const int row = tm * BM + h * kBM + (int)(quarter * 32 + lane);
+                    const int col0 = tn * BN + c * 32;
+                    const uint32_t* q = r + 32 * j;
+#pragma unroll
+                    for (int gq = 0; gq < 4; ++gq) {  // groups of 8 columns (N % 8 == 0)
+                        const int col = col0 + 8 * gq;
+                        if (row >= shape.M || col >= shape.N) continue;
+                        const size_t off = (size_t)row * shape.N + col;
+                        const uint32_t* v = q + 8 * gq;
+                        if constexpr (OUT == kOut16) {
+                            *reinterpret_cast<uint4*>(static_cast<uint16_t*>(c_out) + off) =
+                                make_uint4(
+                                    pack16x2<F16>(__uint_as_float(v[0]), __uint_as_float(v[1])),
+                                    pack16x2<F16>(__uint_as_float(v[2]), __uint_as_float(v[3])),
+                                    pack16x2<F16>(__uint_as_float(v[4]), __uint_as_float(v[5])),
+                                    pack16x2<F16>(__uint_as_float(v[6]), __uint_as_float(v[7])));
+                        } else if constexpr (OUT == kOutF32) {
+                            float4* dst =
+                                reinterpret_cast<float4*>(static_cast<float*>(c_out) + off);
+                            dst[0] = make_float4(__uint_as_float(v[0]), __uint_as_float(v[1]),
+                                                 __uint_as_float(v[2]), __uint_as_float(v[3]));
+                            dst[1] = make_float4(__uint_as_float(v[4]), __uint_as_float(v[5]),
+                                                 __uint_as_float(v[6]), __uint_as_float(v[7]));
+                        } else {
+                            // two 16-byte vector reductions (N % 8 == 0 keeps them aligned)
+                            float* dst = static_cast<float*>(c_out) + off;
+                            red_add_v4(dst, __uint_as_float(v[0]), __uint_as_float(v[1]),
+                                       __uint_as_float(v[2]), __uint_as_float(v[3]));
+                            red_add_v4(dst + 4, __uint_as_float(v[4]), __uint_as_float(v[5]),
+                                       __uint_as_float(v[6]), __uint_as_float(v[7]));
+                        }
                     }
                 }
             }
@@ -279,12 +306,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
 }
 
-template <int BN, bool A_MN, bool B_MN, int OUT, bool F16>
+template <int BM, int BN, bool A_MN, bool B_MN, int OUT, bool F16>
 cudaError_t launch_gemm_t(const CUtensorMap& ta, const CUtensorMap& tb, void* c,
                           const GemmShape& s, cudaStream_t stream) {
-    using C = GemmCfg<BN>;
+    using C = GemmCfg<BM, BN>;
     static std::atomic<unsigned long long> configured{0};
-    auto* kernel = gemm_kernel<BN, A_MN, B_MN, OUT, F16>;
+    auto* kernel = gemm_kernel<BM, BN, A_MN, B_MN, OUT, F16>;
     cudaError_t e = set_max_dynamic_smem(kernel, C::kSmemBytes, configured);
     if (e != cudaSuccess) return e;
     const int grid = s.units < sm_count() ? s.units : sm_count();
@@ -292,32 +319,41 @@ cudaError_t launch_gemm_t(const CUtensorMap& ta, const CUtensorMap& tb, void* c,
     return cudaGetLastError();
 }
 
+// Tile shape of a launch: 128 x 128, 128 x 256 or 256 x 256.
+struct Tile {
+    int bm, bn;
+};
+
 template <bool A_MN, bool B_MN>
 cudaError_t launch_gemm_layout(const CUtensorMap& ta, const CUtensorMap& tb, void* c,
-                               const GemmShape& s, int bn, int out, bool f16,
+                               const GemmShape& s, Tile t, int out, bool f16,
                                cudaStream_t stream) {
-#define FORGE_GEMM_OUT(BN_, F16_)                                                               \
-    switch (out) {                                                                              \
-        case kOut16: return launch_gemm_t<BN_, A_MN, B_MN, kOut16, F16_>(ta, tb, c, s, stream);  \
-        case kOutF32: return launch_gemm_t<BN_, A_MN, B_MN, kOutF32, F16_>(ta, tb, c, s, stream);\
-        default: return launch_gemm_t<BN_, A_MN, B_MN, kOutF32Add, F16_>(ta, tb, c, s, stream); \
+#define FORGE_GEMM_OUT(BM_, BN_, F16_)                                                         \
+    switch (out) {                                                                             \
+        case kOut16:                                                                           \
+            return launch_gemm_t<BM_, BN_, A_MN, B_MN, kOut16, F16_>(ta, tb, c, s, stream);    \
+        case kOutF32:                                                                          \
+            return launch_gemm_t<BM_, BN_, A_MN, B_MN, kOutF32, F16_>(ta, tb, c, s, stream);   \
+        default:                                                                               \
+            return launch_gemm_t<BM_, BN_, A_MN, B_MN, kOutF32Add, F16_>(ta, tb, c, s, stream);\
     }
-    if (bn == 256) {
-        if (f16) { FORGE_GEMM_OUT(256, true) }
-        FORGE_GEMM_OUT(256, false)
-    }
-    if (f16) { FORGE_GEMM_OUT(128, true) }
-    FORGE_GEMM_OUT(128, false)
+#define FORGE_GEMM_TILE(BM_, BN_)                 \
+    if (f16) { FORGE_GEMM_OUT(BM_, BN_, true) }   \
+    FORGE_GEMM_OUT(BM_, BN_, false)
+    if (t.bm == 256) { FORGE_GEMM_TILE(256, 256) }
+    if (t.bn == 256) { FORGE_GEMM_TILE(128, 256) }
+    FORGE_GEMM_TILE(128, 128)
+#undef FORGE_GEMM_TILE
 #undef FORGE_GEMM_OUT
 }
 
-GemmShape make_shape(int M, int N, int K, int BN, int splits) {
+GemmShape make_shape(int M, int N, int K, Tile t, int splits) {
     GemmShape s;
     s.M = M;
     s.N = N;
     s.K = K;
-    s.tiles_m = (M + kBM - 1) / kBM;
-    s.tiles_n = (N + BN - 1) / BN;
+    s.tiles_m = (M + t.bm - 1) / t.bm;
+    s.tiles_n = (N + t.bn - 1) / t.bn;
     s.k_blocks = (K + kBK - 1) / kBK;
     if (splits < 1) splits = 1;
     if (splits > s.k_blocks) splits = s.k_blocks;
@@ -329,8 +365,8 @@ GemmShape make_shape(int M, int N, int K, int BN, int splits) {
 
 // Split of a reduction of K over (split, tile) units when none is asked for: enough units
 // to give every SM about two, each split at least eight k-blocks (512) deep.
-int auto_splits(int M, int N, int K, int bn) {
-    const long long tiles = (long long)((M + kBM - 1) / kBM) * ((N + bn - 1) / bn);
+int auto_splits(int M, int N, int K, Tile t) {
+    const long long tiles = (long long)((M + t.bm - 1) / t.bm) * ((N + t.bn - 1) / t.bn);
     const int k_blocks = (K + kBK - 1) / kBK;
     long long splits = (2LL * sm_count() + tiles - 1) / tiles;
     const long long max_splits = k_blocks / 8 > 0 ? k_blocks / 8 : 1;
@@ -338,22 +374,30 @@ int auto_splits(int M, int N, int K, int bn) {
     return splits < 1 ? 1 : (int)splits;
 }
 
-// Tile width.  A 128 x 256 tile does twice the work of a 128 x 128 one for 1.5 times
-// its operand bytes per k-block (A 16 KB + B 32 KB against 16 + 16 KB), and the
-// operand stream from L2 sets the pace of both, so a 256-wide k-block costs 1.5 of a
-// 128-wide one (1.4-1.55 measured on linear-layer shapes).  A width's cost is then the
-// k-blocks of the most loaded CTA (units are dealt round robin), weighted so: fewer,
-// wider tiles win unless they leave many more SMs idle.  256 on a tie.  splits = 0
-// takes auto_splits for each width.
-int pick_bn(int M, int N, int K, int splits) {
-    if (N <= 128) return 128;
+// Tile shape.  Shared-memory traffic sets the pace of a k-block: the TMA writes of its
+// operands plus the tensor cores' reads of them (each 128 x BN x 16 product reads its A
+// and B slices), 64, 96 and 160 KB for 128 x 128, 128 x 256 and 256 x 256 tiles
+// (weights 2, 3, 5) for 1, 2 and 4 times the work; measured times per unit of work
+// were 1 : 0.76 : 0.67 (square 8192), where these bytes give 1 : 0.75 : 0.63 and the
+// tensor-core time alone would give 1 : 1 : 1.  A 256 x 256 tile's accumulator fills
+// tensor memory alone, so the next tile's products wait for its epilogue: weight 32
+// more per tile (fitted on linear-layer shapes).  A shape costs what its most loaded
+// CTA does (units are dealt round robin); the larger tile on a tie.  splits = 0 takes
+// auto_splits for each shape.
+Tile pick_tile(int M, int N, int K, int splits) {
+    Tile best{128, 128};
+    if (N <= 128) return best;
     const int sms = sm_count();
-    auto cost = [&](int bn) {
-        const int sp = splits > 0 ? splits : auto_splits(M, N, K, bn);
-        const GemmShape s = make_shape(M, N, K, bn, sp);
-        return (long long)((s.units + sms - 1) / sms) * s.kb_per_split * (bn == 256 ? 3 : 2);
+    auto cost = [&](Tile t) {
+        const int sp = splits > 0 ? splits : auto_splits(M, N, K, t);
+        const GemmShape s = make_shape(M, N, K, t, sp);
+        const int w = t.bm == 256 ? 5 : (t.bn == 256 ? 3 : 2);
+        return (long long)((s.units + sms - 1) / sms) *
+               ((long long)s.kb_per_split * w + (t.bm == 256 ? 32 : 0));
     };
-    return cost(256) <= cost(128) ? 256 : 128;
+    for (const Tile t : {Tile{128, 256}, Tile{256, 256}})
+        if (cost(t) <= cost(best)) best = t;
+    return best;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -389,14 +433,14 @@ int forge_linear_fwd(const void* x, const void* w, void* y, int tokens, int in_f
     if (flags & ~(FORGE_ATTN_OUT_F32 | FORGE_ATTN_FP16)) return FORGE_ATTN_ERR_INVALID_ARG;
     if (!aligned16(x) || !aligned16(w) || !aligned16(y)) return FORGE_ATTN_ERR_MISALIGNED;
     const bool f16 = (flags & FORGE_ATTN_FP16) != 0;
-    const int bn = pick_bn(tokens, out_features, in_features, 1);
+    const Tile t = pick_tile(tokens, out_features, in_features, 1);
     CUtensorMap ta, tb;
     if (encode_map_2d16(&ta, x, in_features, tokens, 64, kBM, f16) != cudaSuccess ||
-        encode_map_2d16(&tb, w, in_features, out_features, 64, bn, f16) != cudaSuccess)
+        encode_map_2d16(&tb, w, in_features, out_features, 64, t.bn, f16) != cudaSuccess)
         return FORGE_ATTN_ERR_CUDA;
-    const GemmShape sh = make_shape(tokens, out_features, in_features, bn, 1);
+    const GemmShape sh = make_shape(tokens, out_features, in_features, t, 1);
     return status_of(launch_gemm_layout<false, false>(
-        ta, tb, y, sh, bn, (flags & FORGE_ATTN_OUT_F32) ? kOutF32 : kOut16, f16,
+        ta, tb, y, sh, t, (flags & FORGE_ATTN_OUT_F32) ? kOutF32 : kOut16, f16,
         static_cast<cudaStream_t>(stream)));
 }
 
@@ -408,22 +452,22 @@ int forge_linear_bwd_dx(const void* dy, const void* w, void* dx, int tokens, int
     if (flags & ~(FORGE_ATTN_OUT_F32 | FORGE_ATTN_FP16)) return FORGE_ATTN_ERR_INVALID_ARG;
     if (!aligned16(dy) || !aligned16(w) || !aligned16(dx)) return FORGE_ATTN_ERR_MISALIGNED;
     const bool f16 = (flags & FORGE_ATTN_FP16) != 0;
-    const int bn = pick_bn(tokens, in_features, out_features, 1);
+    const Tile t = pick_tile(tokens, in_features, out_features, 1);
     CUtensorMap ta, tb;
     // A = dY [tokens][out] (k = out contiguous); B = W [out = k][in = n], MN-major
     if (encode_map_2d16(&ta, dy, out_features, tokens, 64, kBM, f16) != cudaSuccess ||
         encode_map_2d16(&tb, w, in_features, out_features, 64, 64, f16) != cudaSuccess)
         return FORGE_ATTN_ERR_CUDA;
-    const GemmShape sh = make_shape(tokens, in_features, out_features, bn, 1);
+    const GemmShape sh = make_shape(tokens, in_features, out_features, t, 1);
     return status_of(launch_gemm_layout<false, true>(
-        ta, tb, dx, sh, bn, (flags & FORGE_ATTN_OUT_F32) ? kOutF32 : kOut16, f16,
+        ta, tb, dx, sh, t, (flags & FORGE_ATTN_OUT_F32) ? kOutF32 : kOut16, f16,
         static_cast<cudaStream_t>(stream)));
 }
 
 int forge_linear_split_k(int tokens, int in_features, int out_features) {
     if (check_dims(tokens, in_features, out_features) != FORGE_ATTN_OK) return 0;
-    const int bn = pick_bn(out_features, in_features, tokens, 0);
-    return auto_splits(out_features, in_features, tokens, bn);
+    const Tile t = pick_tile(out_features, in_features, tokens, 0);
+    return auto_splits(out_features, in_features, tokens, t);
 }
 
 int forge_linear_bwd_dw(const void* dy, const void* x, float* dw, int tokens, int in_features,
@@ -435,9 +479,9 @@ int forge_linear_bwd_dw(const void* dy, const void* x, float* dw, int tokens, in
     if (flags & ~FORGE_ATTN_FP16) return FORGE_ATTN_ERR_INVALID_ARG;
     if (!aligned16(dy) || !aligned16(x) || !aligned16(dw)) return FORGE_ATTN_ERR_MISALIGNED;
     const bool f16 = (flags & FORGE_ATTN_FP16) != 0;
-    const int bn = pick_bn(out_features, in_features, tokens, split_k);
-    if (split_k == 0) split_k = auto_splits(out_features, in_features, tokens, bn);
-    const GemmShape sh = make_shape(out_features, in_features, tokens, bn, split_k);
+    const Tile t = pick_tile(out_features, in_features, tokens, split_k);
+    if (split_k == 0) split_k = auto_splits(out_features, in_features, tokens, t);
+    const GemmShape sh = make_shape(out_features, in_features, tokens, t, split_k);
     CUtensorMap ta, tb;
     // A = dY^T: dY [tokens = k][out = m], MN-major; B = X [tokens = k][in = n], MN-major
     if (encode_map_2d16(&ta, dy, out_features, tokens, 64, 64, f16) != cudaSuccess ||
@@ -452,7 +496,7 @@ int forge_linear_bwd_dw(const void* dy, const void* x, float* dw, int tokens, in
             cudaMemsetAsync(dw, 0, (size_t)out_features * in_features * sizeof(float), st);
         if (e != cudaSuccess) return FORGE_ATTN_ERR_CUDA;
     }
-    return status_of(launch_gemm_layout<true, true>(ta, tb, dw, sh, bn,
+    return status_of(launch_gemm_layout<true, true>(ta, tb, dw, sh, t,
                                                     add ? kOutF32Add : kOutF32, f16, st));
 }
 

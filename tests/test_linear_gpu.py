@@ -102,3 +102,20 @@ def test_fp32_outputs():
 
 def test_fp16_operands():
     run(1032, 264, 392, seed=59, dtype=torch.float16)
+
+
+# Shapes whose products take the wider tiles on a 148-SM B200 (by the library's tile
+# cost model), with rows and columns that end inside a tile:
+#   (3000, 776, 776)    Y, dX and dW on 128 x 256 tiles
+#   (3000, 2056, 1544)  Y on 256 x 256 tiles (dX, dW 128 x 256)
+#   (3000, 1544, 2056)  dX on 256 x 256 tiles
+#   (4040, 3080, 3080)  dW on 256 x 256 tiles, split over the tokens
+@pytest.mark.parametrize("shape", [(3000, 776, 776), (3000, 2056, 1544), (3000, 1544, 2056),
+                                   (4040, 3080, 3080)])
+def test_wide_tiles_on_ragged_shapes(shape):
+    run(*shape, seed=61 + shape[1] % 7)
+
+
+def test_wide_tiles_fp16_and_fp32_outputs():
+    run(3000, 2056, 1544, seed=67, dtype=torch.float16)
+    run(3000, 1544, 2056, seed=71, out_f32=True)
