@@ -363,40 +363,54 @@ GemmShape make_shape(int M, int N, int K, Tile t, int splits) {
     return s;
 }
 
-// Split of a reduction of K over (split, tile) units when none is asked for: enough units
-// to give every SM about two, each split at least eight k-blocks (512) deep.
-int auto_splits(int M, int N, int K, Tile t) {
-    const long long tiles = (long long)((M + t.bm - 1) / t.bm) * ((N + t.bn - 1) / t.bn);
-    const int k_blocks = (K + kBK - 1) / kBK;
-    long long splits = (2LL * sm_count() + tiles - 1) / tiles;
-    const long long max_splits = k_blocks / 8 > 0 ? k_blocks / 8 : 1;
-    if (splits > max_splits) splits = max_splits;
-    return splits < 1 ? 1 : (int)splits;
+// Tile shape and split of the reduction over K for a launch.
+struct Plan {
+    Tile tile;
+    int splits;
+};
+
+// Cost model of a plan, fitted on linear-layer shapes.  Shared-memory traffic sets the
+// pace of a k-block: the TMA writes of its operands plus the tensor cores' reads of them
+// (each 128 x BN x 16 product reads its A and B slices), 64, 96 and 160 KB for 128 x 128,
+// 128 x 256 and 256 x 256 tiles (weights 2, 3, 5) for 1, 2 and 4 times the work;
+// measured times per unit of work were 1 : 0.76 : 0.67 (square 8192), where these bytes
+// give 1 : 0.75 : 0.63 and the tensor-core time alone would give 1 : 1 : 1.  A 256 x 256
+// tile's accumulator fills tensor memory alone, so the next tile's products wait for its
+// epilogue: weight 32 more per tile.  A plan costs what its most loaded CTA does (units
+// are dealt round robin), plus, with more than one split, the fp32 reductions of every
+// split's partial output in L2 (after a memset of C): weight 1e-5 per output element and
+// split.
+double plan_cost(int M, int N, int K, Tile t, int splits, int sms) {
+    const GemmShape s = make_shape(M, N, K, t, splits);
+    const int w = t.bm == 256 ? 5 : (t.bn == 256 ? 3 : 2);
+    double c = (double)((s.units + sms - 1) / sms) *
+               ((double)s.kb_per_split * w + (t.bm == 256 ? 32.0 : 0.0));
+    if (s.splits > 1) c += 1e-5 * s.splits * (double)M * N;
+    return c;
 }
 
-// Tile shape.  Shared-memory traffic sets the pace of a k-block: the TMA writes of its
-// operands plus the tensor cores' reads of them (each 128 x BN x 16 product reads its A
-// and B slices), 64, 96 and 160 KB for 128 x 128, 128 x 256 and 256 x 256 tiles
-// (weights 2, 3, 5) for 1, 2 and 4 times the work; measured times per unit of work
-// were 1 : 0.76 : 0.67 (square 8192), where these bytes give 1 : 0.75 : 0.63 and the
-// tensor-core time alone would give 1 : 1 : 1.  A 256 x 256 tile's accumulator fills
-// tensor memory alone, so the next tile's products wait for its epilogue: weight 32
-// more per tile (fitted on linear-layer shapes).  A shape costs what its most loaded
-// CTA does (units are dealt round robin); the larger tile on a tie.  splits = 0 takes
-// auto_splits for each shape.
-Tile pick_tile(int M, int N, int K, int splits) {
-    Tile best{128, 128};
-    if (N <= 128) return best;
+// The cheapest plan: over the three tiles (128 x 128 alone when N <= 128) and, when
+// splits = 0, every split whose parts are at least eight k-blocks (512) deep; else the
+// split given.  Ties go to the larger tile, then to fewer splits.
+Plan pick_plan(int M, int N, int K, int splits) {
     const int sms = sm_count();
-    auto cost = [&](Tile t) {
-        const int sp = splits > 0 ? splits : auto_splits(M, N, K, t);
-        const GemmShape s = make_shape(M, N, K, t, sp);
-        const int w = t.bm == 256 ? 5 : (t.bn == 256 ? 3 : 2);
-        return (long long)((s.units + sms - 1) / sms) *
-               ((long long)s.kb_per_split * w + (t.bm == 256 ? 32 : 0));
-    };
-    for (const Tile t : {Tile{128, 256}, Tile{256, 256}})
-        if (cost(t) <= cost(best)) best = t;
+    const int k_blocks = (K + kBK - 1) / kBK;
+    const int lo = splits > 0 ? splits : 1;
+    const int hi = splits > 0 ? splits : (k_blocks / 8 > 1 ? k_blocks / 8 : 1);
+    Plan best{Tile{128, 128}, lo};
+    double best_c = 0.0;
+    bool have = false;
+    for (const Tile t : {Tile{256, 256}, Tile{128, 256}, Tile{128, 128}}) {
+        if (N <= 128 && t.bn != 128) continue;
+        for (int sp = lo; sp <= hi; ++sp) {
+            const double c = plan_cost(M, N, K, t, sp, sms);
+            if (!have || c < best_c) {
+                best = Plan{t, sp};
+                best_c = c;
+                have = true;
+            }
+        }
+    }
     return best;
 }
 
@@ -433,7 +447,7 @@ int forge_linear_fwd(const void* x, const void* w, void* y, int tokens, int in_f
     if (flags & ~(FORGE_ATTN_OUT_F32 | FORGE_ATTN_FP16)) return FORGE_ATTN_ERR_INVALID_ARG;
     if (!aligned16(x) || !aligned16(w) || !aligned16(y)) return FORGE_ATTN_ERR_MISALIGNED;
     const bool f16 = (flags & FORGE_ATTN_FP16) != 0;
-    const Tile t = pick_tile(tokens, out_features, in_features, 1);
+    const Tile t = pick_plan(tokens, out_features, in_features, 1).tile;
     CUtensorMap ta, tb;
     if (encode_map_2d16(&ta, x, in_features, tokens, 64, kBM, f16) != cudaSuccess ||
         encode_map_2d16(&tb, w, in_features, out_features, 64, t.bn, f16) != cudaSuccess)
@@ -452,7 +466,7 @@ int forge_linear_bwd_dx(const void* dy, const void* w, void* dx, int tokens, int
     if (flags & ~(FORGE_ATTN_OUT_F32 | FORGE_ATTN_FP16)) return FORGE_ATTN_ERR_INVALID_ARG;
     if (!aligned16(dy) || !aligned16(w) || !aligned16(dx)) return FORGE_ATTN_ERR_MISALIGNED;
     const bool f16 = (flags & FORGE_ATTN_FP16) != 0;
-    const Tile t = pick_tile(tokens, in_features, out_features, 1);
+    const Tile t = pick_plan(tokens, in_features, out_features, 1).tile;
     CUtensorMap ta, tb;
     // A = dY [tokens][out] (k = out contiguous); B = W [out = k][in = n], MN-major
     if (encode_map_2d16(&ta, dy, out_features, tokens, 64, kBM, f16) != cudaSuccess ||
@@ -466,8 +480,7 @@ int forge_linear_bwd_dx(const void* dy, const void* w, void* dx, int tokens, int
 
 int forge_linear_split_k(int tokens, int in_features, int out_features) {
     if (check_dims(tokens, in_features, out_features) != FORGE_ATTN_OK) return 0;
-    const Tile t = pick_tile(out_features, in_features, tokens, 0);
-    return auto_splits(out_features, in_features, tokens, t);
+    return pick_plan(out_features, in_features, tokens, 0).splits;
 }
 
 int forge_linear_bwd_dw(const void* dy, const void* x, float* dw, int tokens, int in_features,
@@ -479,9 +492,9 @@ int forge_linear_bwd_dw(const void* dy, const void* x, float* dw, int tokens, in
     if (flags & ~FORGE_ATTN_FP16) return FORGE_ATTN_ERR_INVALID_ARG;
     if (!aligned16(dy) || !aligned16(x) || !aligned16(dw)) return FORGE_ATTN_ERR_MISALIGNED;
     const bool f16 = (flags & FORGE_ATTN_FP16) != 0;
-    const Tile t = pick_tile(out_features, in_features, tokens, split_k);
-    if (split_k == 0) split_k = auto_splits(out_features, in_features, tokens, t);
-    const GemmShape sh = make_shape(out_features, in_features, tokens, t, split_k);
+    const Plan plan = pick_plan(out_features, in_features, tokens, split_k);
+    const Tile t = plan.tile;
+    const GemmShape sh = make_shape(out_features, in_features, tokens, t, plan.splits);
     CUtensorMap ta, tb;
     // A = dY^T: dY [tokens = k][out = m], MN-major; B = X [tokens = k][in = n], MN-major
     if (encode_map_2d16(&ta, dy, out_features, tokens, 64, 64, f16) != cudaSuccess ||

@@ -52,9 +52,11 @@ int forge_linear_bwd_dx(const void* dy, const void* w, void* dx, int tokens, int
 int forge_linear_bwd_dw(const void* dy, const void* x, float* dw, int tokens, int in_features,
                         int out_features, int split_k, int accumulate, int flags, void* stream);
 
-/* The split of forge_linear_bwd_dw's token reduction chosen for split_k = 0: enough
- * (part, tile) units to give every SM about two, each part at least 512 tokens deep.
- * 0 for arguments forge_linear_bwd_dw would reject. */
+/* The split of forge_linear_bwd_dw's token reduction chosen for split_k = 0: with the
+ * tile shape, the plan a cost model rates cheapest (the k-blocks of the most loaded SM,
+ * weighted by the tile's shared-memory traffic, plus the fp32 reductions of every
+ * part's partial dW), each part at least 512 tokens deep.  0 for arguments
+ * forge_linear_bwd_dw would reject. */
 int forge_linear_split_k(int tokens, int in_features, int out_features);
 
 #ifdef __cplusplus

@@ -104,14 +104,16 @@ def test_fp16_operands():
     run(1032, 264, 392, seed=59, dtype=torch.float16)
 
 
-# Shapes whose products take the wider tiles on a 148-SM B200 (by the library's tile
+# Shapes whose products take the wider tiles on a 148-SM B200 (by the library's plan
 # cost model), with rows and columns that end inside a tile:
-#   (3000, 776, 776)    Y, dX and dW on 128 x 256 tiles
+#   (3000, 776, 776)    Y and dX on 128 x 256 tiles (dW 128 x 128, split 3)
 #   (3000, 2056, 1544)  Y on 256 x 256 tiles (dX, dW 128 x 256)
 #   (3000, 1544, 2056)  dX on 256 x 256 tiles
-#   (4040, 3080, 3080)  dW on 256 x 256 tiles, split over the tokens
+#   (2056, 1544, 3080)  dW on 256 x 256 tiles, one split (stored)
+#   (12040, 264, 3080)  dW on 256 x 256 tiles, split 5 (fp32 reductions)
+#   (3000, 264, 2056)   dW on 128 x 256 tiles, split 4
 @pytest.mark.parametrize("shape", [(3000, 776, 776), (3000, 2056, 1544), (3000, 1544, 2056),
-                                   (4040, 3080, 3080)])
+                                   (2056, 1544, 3080), (12040, 264, 3080), (3000, 264, 2056)])
 def test_wide_tiles_on_ragged_shapes(shape):
     run(*shape, seed=61 + shape[1] % 7)
 
