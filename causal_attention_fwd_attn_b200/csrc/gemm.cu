@@ -390,13 +390,15 @@ double plan_cost(int M, int N, int K, Tile t, int splits, int sms) {
 }
 
 // The cheapest plan: over the three tiles (128 x 128 alone when N <= 128) and, when
-// splits = 0, every split whose parts are at least eight k-blocks (512) deep; else the
-// split given.  Ties go to the larger tile, then to fewer splits.
+// splits = 0, every split whose parts are at least eight k-blocks (512) deep, up to two
+// per SM (more cannot shorten the most loaded CTA's share); else the split given.  Ties
+// go to the larger tile, then to fewer splits.
 Plan pick_plan(int M, int N, int K, int splits) {
     const int sms = sm_count();
     const int k_blocks = (K + kBK - 1) / kBK;
     const int lo = splits > 0 ? splits : 1;
-    const int hi = splits > 0 ? splits : (k_blocks / 8 > 1 ? k_blocks / 8 : 1);
+    int hi = splits > 0 ? splits : (k_blocks / 8 > 1 ? k_blocks / 8 : 1);
+    if (splits == 0 && hi > 2 * sms) hi = 2 * sms;
     Plan best{Tile{128, 128}, lo};
     double best_c = 0.0;
     bool have = false;
