@@ -54,12 +54,15 @@ L2_BYTES = 126 * 1024 * 1024
 PROFILES = os.path.join(ROOT, "profiles")
 # Sub-results beside the headline: (workload, mode, causal).  Every causal workload
 # in the mode its parity tests use, the long workload also in the default bf16 mode
-# (context: outside the tolerance there), and full attention at two shapes.
+# (context: outside the tolerance there) and in the fp16-operand accuracy mode (which
+# meets the tolerance there too, with its bf16 -> fp16 input conversion in the step),
+# and full attention at two shapes.
 SUB_RESULTS = [
     ("gpt2small_b8h12t1024d64", "default", 1),
     ("decoder200m_b4h16t2048d64", "default", 1),
     ("hd128_b2h16t4096d128", "default", 1),
     ("ragged_b1h32t8000d128", "default", 1),
+    ("ragged_b1h32t8000d128", "accuracy_fp16", 1),
     ("gpt2small_b8h12t1024d64", "default", 0),
     ("hd128_b2h16t4096d128", "default", 0),
 ]
@@ -277,49 +280,71 @@ class Pass:
         # with fp32 gradients the dQ accumulator is dq itself, and there is no conversion
         self.acc = (self.dq.data_ptr() if m["grad_f32"]
                     else self.ws.data_ptr() + _lib.rowstats_bytes(B, H, T))
-        p = _lib.PRECISE if m["precise"] else 0
+        # the fp16-operand mode converts each step's bf16 inputs into these first
+        self.fp16 = m["fp16"]
+        self.x16 = ({n: torch.empty((B, H, T, d), dtype=torch.float16, device=dev)
+                     for n in ("q", "k", "v", "dO")} if self.fp16 else None)
+        self.overflow = torch.zeros(1, dtype=torch.int32, device=dev)
+        p = (_lib.PRECISE if m["precise"] else 0) | (_lib.FP16 if self.fp16 else 0)
         self.fwd_flags = (_lib.OUT_F32 if m["o_f32"] else 0) | p
-        self.pre_flags = _lib.O_IN_F32 if m["o_f32"] else 0
+        self.pre_flags = (_lib.O_IN_F32 if m["o_f32"] else 0) | (_lib.FP16 if self.fp16 else 0)
         self.dkdv_flags = (_lib.OUT_F32 if m["grad_f32"] else 0) | p
         self.bwd_flags = self.pre_flags | self.dkdv_flags
-        self.kernels = ["fwd", "pre", "dkdv"] + ([] if m["grad_f32"] else ["cvt"])
+        # timed stages in step order ("in": the four input conversions)
+        self.kernels = ((["in"] if self.fp16 else []) + ["fwd", "pre", "dkdv"]
+                        + ([] if m["grad_f32"] else ["cvt"]))
+        self.launches_per_step = len(self.kernels) + (3 if self.fp16 else 0)
         self.stream = torch.cuda.current_stream(dev)
 
+    def to_fp16(self, x):
+        """The library's bf16 -> fp16 conversion of q, k, v, dO into self.x16."""
+        L, s = self.lib, self.stream.cuda_stream
+        for n in ("q", "k", "v", "dO"):
+            L.check(L.forge_attn_bf16_to_fp16(x[n].data_ptr(), self.x16[n].data_ptr(),
+                                              x[n].numel(), self.overflow.data_ptr(), s),
+                    "bf16_to_fp16")
+        return self.x16
+
     def step(self, x, ev=None):
+        """One step; with `ev` (five events) an event before the first stage and after
+        each stage of self.kernels."""
         L, w, s = self.lib, self.w, self.stream.cuda_stream
         B, H, T, d = w.B, w.H, w.T, w.d
+        marks = iter(ev or [])
+
+        def mark():
+            if ev:
+                next(marks).record(self.stream)
+
+        mark()
+        if self.fp16:
+            x = self.to_fp16(x)
+            mark()
         q, k, v, dO = x["q"], x["k"], x["v"], x["dO"]
-        if ev:
-            ev[0].record(self.stream)
         L.check(L.forge_attn_fwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), self.o.data_ptr(),
                                     self.lse.data_ptr(), B, H, T, d, w.scale, self.causal,
                                     self.fwd_flags, s), "fwd")
-        if ev:
-            ev[1].record(self.stream)
+        mark()
         L.check(L.forge_attn_bwd_preprocess(self.o.data_ptr(), dO.data_ptr(), self.lse.data_ptr(),
                                             self.rowstats, self.acc, B, H, T, d, self.pre_flags,
                                             s), "pre")
-        if ev:
-            ev[2].record(self.stream)
+        mark()
         L.check(L.forge_attn_bwd_dkdv(q.data_ptr(), k.data_ptr(), v.data_ptr(), dO.data_ptr(),
                                       self.rowstats, self.acc, self.dk.data_ptr(),
                                       self.dv.data_ptr(), B, H, T, d, w.scale, self.causal,
                                       self.dkdv_flags, s), "dkdv")
-        if ev:
-            ev[3].record(self.stream)
+        mark()
         if "cvt" in self.kernels:
             L.check(L.forge_attn_bwd_dq_convert(self.acc, self.dq.data_ptr(), B, H, T, d, s),
                     "cvt")
-        if ev:
-            ev[4].record(self.stream)
+            mark()
 
     def kernel_times(self, evs):
-        """Mean CUDA-event time (ms) of each kernel over the steps of `evs`."""
+        """Mean CUDA-event time (ms) of each stage over the steps of `evs`."""
         per = {k: [] for k in self.kernels}
         for e in evs:
-            for a, k in enumerate(("fwd", "pre", "dkdv", "cvt")):
-                if k in per:
-                    per[k].append(e[a].elapsed_time(e[a + 1]))
+            for a, k in enumerate(self.kernels):
+                per[k].append(e[a].elapsed_time(e[a + 1]))
         return {k: sum(v) / len(v) for k, v in per.items()}
 
     def check_device(self, when):
@@ -356,6 +381,8 @@ def timed_run(p, sets, warmup, steps, world, dev, clocks):
     hi = clocks.now()
     barrier(world)
     p.check_device("in the timed region")
+    if p.fp16 and int(p.overflow.item()) != 0:
+        raise RuntimeError("inputs beyond fp16's range in the fp16-operand mode")
     max_ms = max_over_ranks(t0.elapsed_time(t1), world, dev)
     return max_ms, p.kernel_times(evs), clocks.stats(lo, hi)
 
@@ -387,7 +414,7 @@ def result_fields(w, causal, steps, world, max_ms, avg, peaks):
     """Throughput fields shared by the headline and the sub-results."""
     fwd_flops, bwd_flops = causal_flops(w, causal)
     value = job_tflops(fwd_flops + bwd_flops, steps, world, max_ms)
-    bwd_ms = sum(v for k, v in avg.items() if k != "fwd")
+    bwd_ms = sum(v for k, v in avg.items() if k not in ("fwd", "in"))
     return {
         "value": round(value, 2),
         "ms_per_step": round(max_ms / steps, 4),
@@ -419,7 +446,7 @@ def ours_line(w, mode, causal, steps, warmup, world, max_ms, avg, clk, e2e, laun
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "bf16",
+        "dtype": "f16" if wl.MODES[mode]["fp16"] else "bf16",
         "data": "synthetic",
         "config": config_of(w, mode, causal, world),
         "mode_desc": wl.MODES[mode]["desc"],
@@ -442,6 +469,7 @@ def sub_result(w, mode, causal, steps, world, max_ms, avg, clk, peaks):
     _, bwd_flops = causal_flops(w, causal)
     dkdv_tf = bwd_flops / (avg["dkdv"] * 1e-3) / 1e12
     r.update({"workload": w.name, "mode": mode, "causal": causal, "steps": steps,
+              "dtype": "f16" if wl.MODES[mode]["fp16"] else "bf16",
               "dominant_kernel": dominant(avg),
               "dkdv_frac": round(dkdv_tf / peaks["bf16_tflops"], 4),
               "clocks": {k: clk.get(k) for k in ("sm_mhz", "samples", "reasons")}})
@@ -640,7 +668,7 @@ def run_ours(args, rank, world, local_rank):
         return None
     traffic = recorded_traffic("attn_bwd_dkdv", f"{w.name}/{mode}")
     return ours_line(w, mode, causal, args.steps, args.warmup, world, max_ms, avg, clk, e2e,
-                     len(p.kernels), peaks, traffic,
+                     p.launches_per_step, peaks, traffic,
                      os.path.relpath(_lib.library_path(), ROOT), subs)
 
 
@@ -687,7 +715,8 @@ def run_e2e(args, w, ci, mode, causal, dev, p, world):
             comp.wait_event(in_ready[k])
             if k >= 2:
                 comp.wait_event(out_done[k - 2])         # buffer set b's outputs are read
-            q, kk, v, dO = (dev_in[b][n] for n in ("q", "k", "v", "dO"))
+            xin = p.to_fp16(dev_in[b]) if p.fp16 else dev_in[b]
+            q, kk, v, dO = (xin[n] for n in ("q", "k", "v", "dO"))
             o = dev_out[b]
             L.check(L.forge_attn_fwd_ex(q.data_ptr(), kk.data_ptr(), v.data_ptr(),
                                         o["o"].data_ptr(), o["lse"].data_ptr(), B, H, T, d,

@@ -37,6 +37,7 @@ EXPORTED = [
     "forge_attn_check_device_error", "forge_attn_version", "forge_probe_mma", "forge_probe_wait_timeout",
     "forge_attn_bwd_noalloc", "forge_adamw_workspace_size", "forge_adamw_step",
     "forge_linear_fwd", "forge_linear_bwd_dx", "forge_linear_bwd_dw", "forge_linear_split_k",
+    "forge_attn_bf16_to_fp16",
 ]
 
 ADAMW_MAX_TENSORS_PER_LAUNCH = 256
@@ -79,6 +80,7 @@ _SIGNATURES = {
     "forge_linear_bwd_dx": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _vp]),
     "forge_linear_bwd_dw": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp]),
     "forge_linear_split_k": (_i, [_i, _i, _i]),
+    "forge_attn_bf16_to_fp16": (_i, [_vp, _vp, ctypes.c_longlong, _vp, _vp]),
     "forge_adamw_step": (_i, [ctypes.POINTER(AdamWTensor), _i, _f, _f, _f, _f, _f, _i, _f, _vp,
                               _vp, _sz, _vp]),
 }
@@ -214,6 +216,10 @@ def forge_linear_bwd_dw(dy, x, dw, tokens, in_features, out_features, split_k, a
 
 def forge_linear_split_k(tokens, in_features, out_features):
     return load().forge_linear_split_k(tokens, in_features, out_features)
+
+
+def forge_attn_bf16_to_fp16(src, dst, n, overflow, stream):
+    return load().forge_attn_bf16_to_fp16(src, dst, n, overflow, stream)
 
 
 def forge_attn_check_device_error(stream):

@@ -20,7 +20,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIBRARY = os.path.join(PKG, "libforge_attn.so")
 SOURCES = ["forge_attn_api.cu", "attn_fwd.cu", "attn_bwd.cu", "tc_probe.cu", "forge_attn_noalloc.cu",
-           "adamw.cu", "gemm.cu"]
+           "adamw.cu", "gemm.cu", "convert.cu"]
 HEADERS = ["sm100_ptx.cuh", "forge_internal.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

@@ -72,12 +72,19 @@ WORKLOADS = [
 ]
 
 # Option settings of each mode (the library's option bits are named after them).
+# "accuracy_fp16" runs the bf16 inputs through the library's bf16 -> fp16 conversion
+# (part of the step) and the fp16-operand kernels.
 MODES = {
-    "default": {"o_f32": False, "grad_f32": False, "precise": False,
+    "default": {"o_f32": False, "grad_f32": False, "precise": False, "fp16": False,
                 "desc": "bf16 O, dQ, dK, dV; P and dS enter the tensor-core products as bf16"},
-    "accuracy": {"o_f32": True, "grad_f32": True, "precise": True,
+    "accuracy": {"o_f32": True, "grad_f32": True, "precise": True, "fp16": False,
                  "desc": "fp32 O, dQ, dK, dV; D from the fp32 O; P and dS enter the "
                          "tensor-core products as two bf16 terms hi + lo"},
+    "accuracy_fp16": {"o_f32": True, "grad_f32": True, "precise": False, "fp16": True,
+                      "desc": "bf16 Q, K, V, dO converted to fp16 in the step (exact for "
+                              "magnitudes in [2^-14, 65504]); fp32 O, dQ, dK, dV; D from the "
+                              "fp32 O; every tensor-core operand fp16 (P and dS with 11 "
+                              "significant bits)"},
 }
 
 TENSOR_INDEX = {"q": 0, "k": 1, "v": 2, "dO": 3}

@@ -200,6 +200,22 @@ int forge_attn_bwd_noalloc(const void* q, const void* k, const void* v, const vo
                            const void* dO, const float* lse, void* dq, void* dk, void* dv,
                            int B, int H, int T, int d, float scale, int causal, void* stream);
 
+/*
+ * bf16 -> fp16 conversion of n values, for running bf16 tensors through the
+ * FORGE_ATTN_FP16 path (whose P and dS then enter the tensor-core products with fp16's
+ * 11 significant bits instead of bf16's 8, so fp32 outputs and D from the fp32 O meet
+ * the tolerances at T = 8000 without FORGE_ATTN_PRECISE's split products).  src, dst:
+ * device pointers, caller-owned, 16-byte aligned, not overlapping.  Each value is
+ * rounded to nearest even once: magnitudes in [2^-14, 65504] (and zeros) convert
+ * exactly, smaller ones land on fp16's subnormal grid (absolute error at most 2^-25),
+ * NaN stays NaN, and larger ones (infinities included) become +-inf; when `overflow`
+ * is not NULL the number of those is added atomically to the device counter
+ * *overflow (4-byte aligned), for the caller to read after the stream's work.
+ * n = 0 does nothing.  One kernel launch on `stream`.
+ */
+int forge_attn_bf16_to_fp16(const void* src, void* dst, long long n, unsigned int* overflow,
+                            void* stream);
+
 /* Human-readable name of a status code (static string, never NULL). */
 const char* forge_attn_status_string(int status);
 

@@ -31,14 +31,29 @@ def assert_close(name, gpu, ref, what=""):
     return rel, mx
 
 
-def run_gpu(x, scale, causal, o_dtype=None, grad_dtype=None, bwd=True, precise=False):
+def to_fp16_on_device(t, s):
+    """bf16 device tensor -> fp16 through the library's conversion (no value may leave
+    fp16's range)."""
+    out = torch.empty_like(t, dtype=torch.float16)
+    over = torch.zeros(1, dtype=torch.int32, device=t.device)
+    _lib.check(_lib.forge_attn_bf16_to_fp16(t.data_ptr(), out.data_ptr(), t.numel(),
+                                            over.data_ptr(), s), "bf16_to_fp16")
+    assert int(over.item()) == 0, "values beyond fp16's range"
+    return out
+
+
+def run_gpu(x, scale, causal, o_dtype=None, grad_dtype=None, bwd=True, precise=False,
+            fp16=False):
     """Forward (and backward) through the C ABI on cuda:0.  x: dict of CPU bf16 (or fp16:
-    the fp16-operand mode) tensors.  Outputs default to the inputs' dtype.  With an
-    fp32 O the backward reads that fp32 O for its D pre-pass."""
+    the fp16-operand mode) tensors; fp16=True converts bf16 inputs to fp16 on the device
+    with the library first.  Outputs default to the kernels' input dtype.  With an fp32 O
+    the backward reads that fp32 O for its D pre-pass."""
     dev = torch.device("cuda", 0)
-    q, k, v, dO = (x[n].to(dev) for n in ("q", "k", "v", "dO"))
-    B, H, T, d = q.shape
     s = torch.cuda.current_stream(dev).cuda_stream
+    q, k, v, dO = (x[n].to(dev) for n in ("q", "k", "v", "dO"))
+    if fp16:
+        q, k, v, dO = (to_fp16_on_device(t, s) for t in (q, k, v, dO))
+    B, H, T, d = q.shape
     o_dtype = o_dtype or q.dtype
     grad_dtype = grad_dtype or q.dtype
     pflag = (_lib.PRECISE if precise else 0) | (_lib.FP16 if q.dtype == torch.float16 else 0)
@@ -72,7 +87,7 @@ def mode_kwargs(mode):
     m = wl.MODES[mode]
     return dict(o_dtype=torch.float32 if m["o_f32"] else torch.bfloat16,
                 grad_dtype=torch.float32 if m["grad_f32"] else torch.bfloat16,
-                precise=m["precise"])
+                precise=m["precise"], fp16=m["fp16"])
 
 
 def oracle_threads(T):

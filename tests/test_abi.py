@@ -179,3 +179,18 @@ def test_linear_rejects_bad_arguments(lib):
         _lib.ERR_INVALID_ARG
     assert _lib.forge_linear_split_k(8192, 768, 3072) >= 1
     assert _lib.forge_linear_split_k(8, 8, 0) == 0
+
+
+def test_bf16_to_fp16_rejects_bad_arguments(lib):
+    # all checked before any launch (no GPU needed); n = 0 is a no-op
+    Q = P + (1 << 20)
+    assert _lib.forge_attn_bf16_to_fp16(P, Q, 0, None, None) == _lib.OK
+    assert _lib.forge_attn_bf16_to_fp16(P, Q, -1, None, None) == _lib.ERR_INVALID_ARG
+    assert _lib.forge_attn_bf16_to_fp16(0, Q, 8, None, None) == _lib.ERR_INVALID_ARG
+    assert _lib.forge_attn_bf16_to_fp16(P, 0, 8, None, None) == _lib.ERR_INVALID_ARG
+    assert _lib.forge_attn_bf16_to_fp16(P + 2, Q, 8, None, None) == _lib.ERR_MISALIGNED
+    assert _lib.forge_attn_bf16_to_fp16(P, Q + 8, 8, None, None) == _lib.ERR_MISALIGNED
+    assert _lib.forge_attn_bf16_to_fp16(P, Q, 8, Q + 2, None) == _lib.ERR_MISALIGNED
+    # overlapping source and destination
+    assert _lib.forge_attn_bf16_to_fp16(P, P + 16, 64, None, None) == _lib.ERR_INVALID_ARG
+    assert _lib.forge_attn_bf16_to_fp16(P + 16, P, 64, None, None) == _lib.ERR_INVALID_ARG

@@ -163,11 +163,25 @@ def test_fp16_operands_fp32_outputs(orc):
 # bound, and where D from a bf16 O and bf16 rounding of P and dS as tensor-core
 # operands each cost 0.01 - 0.05.  So: fp32 O and gradients, D from the fp32 O, and
 # P, dS split into hi + lo bf16 terms.
-def whole_compare(orc, w, x, threads, **kw):
-    got = run_gpu(x, w.scale, w.causal, **kw)
+_ORACLE_CACHE = {}
+
+
+def oracle_outputs(orc, w, x, threads, key=None):
+    """The full oracle's (o, lse, dq, dk, dv); cached under `key` when one is given (the
+    same inputs compared in several modes)."""
+    if key is not None and key in _ORACLE_CACHE:
+        return _ORACLE_CACHE[key]
     f = as_f64(x)
     o, lse = orc.fwd(f["q"], f["k"], f["v"], w.scale, w.causal, threads=threads)
     dq, dk, dv = orc.bwd(f["q"], f["k"], f["v"], f["dO"], w.scale, w.causal, threads=threads)
+    if key is not None:
+        _ORACLE_CACHE[key] = (o, lse, dq, dk, dv)
+    return o, lse, dq, dk, dv
+
+
+def whole_compare(orc, w, x, threads, cache_key=None, **kw):
+    got = run_gpu(x, w.scale, w.causal, **kw)
+    o, lse, dq, dk, dv = oracle_outputs(orc, w, x, threads, cache_key)
     failures = []
     for n, ref in (("o", o), ("lse", lse), ("dq", dq), ("dk", dk), ("dv", dv)):
         rel, mx = errors(got[n], ref)
@@ -183,7 +197,19 @@ def whole_compare(orc, w, x, threads, **kw):
 @pytest.mark.parametrize("ci", [1, 2, 3, 4])
 def test_full_workload_whole_tensors(orc, ci):
     w = wl.WORKLOADS[ci]
-    whole_compare(orc, w, wl.make_inputs(ci), oracle_threads(w.T), **mode_kwargs(w.mode))
+    # the T = 8000 oracle (70 s) is kept for the fp16 accuracy-mode test below
+    whole_compare(orc, w, wl.make_inputs(ci), oracle_threads(w.T),
+                  cache_key=ci if ci == 4 else None, **mode_kwargs(w.mode))
+
+
+def test_long_workload_in_the_fp16_accuracy_mode(orc):
+    """The T = 8000 workload's bf16 inputs converted to fp16 on the device (exact for
+    these magnitudes, at most 16.6) and run through the fp16-operand kernels with fp32
+    outputs and D from the fp32 O, no split products: P and dS keep 11 significant bits,
+    which meets the tolerances where bf16's 8 do not."""
+    w = wl.WORKLOADS[4]
+    whole_compare(orc, w, wl.make_inputs(4), oracle_threads(w.T), cache_key=4,
+                  **mode_kwargs("accuracy_fp16"))
 
 
 # ------------------------------------------------- several items per CTA ----
@@ -208,6 +234,8 @@ MULTI_ITEM = [
     ("precise_full_d64", _multi(4, 16, 1024, 64, causal=0, sv=1.0), "accuracy"),
     ("precise_full_d128", _multi(4, 16, 1024, 128, causal=0, sv=1.0), "accuracy"),
     ("precise_ragged_d128", _multi(2, 40, 1000, 128, sv=1.0), "accuracy"),
+    ("fp16acc_d64", _multi(4, 16, 1024, 64, sv=1.0), "accuracy_fp16"),
+    ("fp16acc_ragged_d128", _multi(2, 40, 1000, 128, sv=1.0), "accuracy_fp16"),
 ]
 
 
