@@ -8,4 +8,5 @@ does, and fails loudly if it is missing.
 """
 from . import workloads  # noqa: F401
 from ._lib import ForgeAttnError, library_path, load  # noqa: F401
-from .attention import attn_bwd, attn_fwd, check_device_error, workspace_bytes  # noqa: F401
+from .attention import (attn_bwd, attn_fwd, check_device_error, to_fp16,  # noqa: F401
+                        workspace_bytes)

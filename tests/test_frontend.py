@@ -39,3 +39,21 @@ def test_cpu_inputs_are_refused_before_any_library_call():
         A.attn_bwd(q, q, q, q, q, torch.zeros((1, 1, 8)))
     with pytest.raises(ValueError, match=r"\[B, H, T, d\]"):
         A.attn_fwd(torch.zeros((8, 64), dtype=torch.bfloat16), q, q)
+
+
+def test_k_v_must_share_q_dtype():
+    # what _check_qkv applies to k and v (it needs CUDA tensors itself)
+    q = torch.zeros((1, 1, 8, 64), dtype=torch.bfloat16)
+    k = torch.zeros((1, 1, 8, 64), dtype=torch.float16)
+    with pytest.raises(ValueError, match="dtype"):
+        A._check_tensor(k, "k", q.shape, (q.dtype,), CPU)
+
+
+def test_fp16_inputs_take_fp16_or_fp32_outputs():
+    assert A._out_dtypes(torch.float16) == (torch.float16, torch.float32)
+    assert A._out_dtypes(torch.bfloat16) == (torch.bfloat16, torch.float32)
+
+
+def test_to_fp16_refuses_cpu_tensors():
+    with pytest.raises(ValueError, match="CUDA"):
+        A.to_fp16(torch.zeros(8, dtype=torch.bfloat16))
