@@ -33,9 +33,12 @@
 //               softmax: thread r owns query row r (TMEM lane r): loads its S row,
 //               masks, updates the running max/sum, writes P (bf16) back to TMEM,
 //               and in the epilogue normalises its O row and writes it and its LSE
-//               to global memory.  From an item's third tile on, the tile's max is
-//               taken in the same pass as its exponentials (against the running max),
-//               and the tile is redone in the rare case that it moves the max.
+//               to global memory.  With bf16 P, from an item's third tile on, the
+//               tile's max is taken in the same pass as its exponentials (against the
+//               running max), and the tile is redone in the rare case that it moves
+//               the max past the lazy-rescale bound.  With fp16 P that bound is 2^15
+//               (fp16's range), which logits of a few nats' spread cross on a large
+//               share of tiles, so the fp16 kernels take every tile's max first.
 // Tensor memory: d = 128, 512 columns: S0 [0,128) | S1 [128,256) | O [256,384) | Q0, Q1
 // [384,512); d = 64, 256 columns per CTA: S0 [0,128) | O [128,192) | Q0, Q1 [192,256)
 // (Q: d/2 columns each).  Key tile g uses S buffer g % (number of buffers), and its P
@@ -513,14 +516,17 @@ __global__ void __launch_bounds__(FwdCfg<D, F16>::kThreads, FwdCfg<D, F16>::kCta
 
             // scale_log2 is >= 0 (a negative scale is applied by negating Q in the MMA),
             // so the max of the scaled scores is scale_log2 times the raw max.
-            if (n > 1 && !masked_tile) {
+            if (!F16 && n > 1 && !masked_tile) {
                 // From an item's third tile on (its first is the only one with masked
                 // keys, and after two tiles the running max has seen at least 129 keys
                 // of the row) a tile is exponentiated against the running max straight
                 // away, taking the tile's max in the same pass: the max is off the
                 // critical path.  The result stands unless the tile raises some row's
                 // max by more than the lazy-rescale bound; then those rows move to the
-                // new max, O is rescaled, and the warp recomputes the tile.
+                // new max, O is rescaled, and the warp recomputes the tile.  (bf16 P
+                // only: under fp16's bound of 2^15 a third of the tiles were recomputed
+                // on logits with a 9-nat spread, and the max-first pass below costs
+                // less than that.)
                 exp_pass(std::true_type{});
                 const float mt = mraw * scale_log2;
                 const bool need = mt > m_run + kRescaleThreshold<F16>;
