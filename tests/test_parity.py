@@ -62,6 +62,15 @@ def test_other_scales(orc, scale):
     full_compare(orc, w, wl.make_inputs(0, w, seed_offset=11), scale=scale)
 
 
+@pytest.mark.parametrize("scale", [0.0, -0.2, 0.15])
+@pytest.mark.parametrize("d", [64, 128])
+def test_other_scales_fp16_operands(orc, scale, d):
+    # the fp16 kernels take every tile's max first; five key tiles per row
+    w = wl.custom(1, 2, 600, d)
+    x = wl.make_inputs(0, w, seed_offset=13 + d, dtype=torch.float16)
+    full_compare(orc, w, x, scale=scale)
+
+
 def test_several_heads_and_batches(orc):
     w = wl.custom(3, 5, 257, 64)
     full_compare(orc, w, wl.make_inputs(0, w, seed_offset=5))
